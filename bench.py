@@ -1,0 +1,459 @@
+"""Benchmark of the W4 + per-token-gated EC linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one pass of the whole hot path over one batch of the workload: for the default
+workload (decode q/o-projection, N = K = 4096, EC rank 64, 1% outlier channels x20) that is
+one spear_w4ec_gemm call for each decode batch M in {1, 4, 16}; each call runs the EC
+pre-pass and the weight-streaming GEMM.  Packing runs once, before timing.
+
+value   = algorithmic bytes (packed W4 + s/z + A + B + w_g + x + y) / device time, GB/s,
+          inputs resident in HBM; K steps are captured in a CUDA graph and replayed, timed
+          with CUDA events; weights rotate over copies larger than 2x L2.
+e2e     = same metric through the Python API with pinned host x and y: every step copies x
+          host->device and y device->host inside the timed region.
+roofline= the layer call at the largest decode batch, against the measured HBM copy peak.
+cpu_baseline / --impl reference = the CPU oracle timed on this host's cores on a bounded
+          sample of the same workload.
+
+Multi-GPU (torchrun): independent replicas, one per GPU (no data-path collective); the
+timed region is bracketed by barriers and the max over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # name: (config index, batches, kind)
+    "decode-qo": (1, [1, 4, 16], "decode"),
+    "decode-mlp": (2, [1, 8, 32, 64], "decode"),
+    "prefill": (3, [2048], "prefill"),
+}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode-qo", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the secondary prefill measurement")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def layer_bytes(M, N, K, r):
+    w = N * K // 2 + 4 * N
+    ec = (2 * K * r + 2 * r * N + 2 * K) if r else 0
+    return w + ec + 2 * M * K + 2 * M * N
+
+
+def layer_flops(M, N, K, r):
+    f = 2 * M * N * K
+    if r:
+        f += 2 * M * K * r + 2 * M * r * N + 2 * M * K
+    return f
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(widx, seconds, M_list):
+    """Time the CPU oracle on the workload's batches, repeated for about `seconds`."""
+    import oracle
+    from synthetic import config_layers
+    cfg, batches, kind = WORKLOADS[widx]
+    L = config_layers(cfg, M=max(batches))[0]
+    packed, s, z = oracle.pack_w4(L.W)
+    if kind == "prefill":
+        M_list = [64]          # a 64-token slice of the 2048-token batch (rows are independent)
+    total_bytes = total_flops = 0
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        for M in M_list:
+            oracle.w4ec_gemm(L.x(M), packed, s, z, L.A_bits, L.B_bits, L.wg_bits, L.b_g)
+            total_bytes += layer_bytes(M, L.N, L.K, L.rank)
+            total_flops += layer_flops(M, L.N, L.K, L.rank)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"bytes": total_bytes, "flops": total_flops, "seconds": dt, "reps": reps, "M": M_list,
+            "cores": oracle.num_threads()}
+
+
+def cpu_baseline_obj(widx, seconds):
+    cfg, batches, kind = WORKLOADS[widx]
+    r = oracle_sample(widx, seconds, batches)
+    if kind == "prefill":
+        val, unit = r["flops"] / r["seconds"] / 1e12, "TFLOP/s"
+    else:
+        val, unit = r["bytes"] / r["seconds"] / 1e9, "GB/s"
+    return {"value": val, "unit": unit, "cores": r["cores"], "kind": "oracle",
+            "sample": f"{r['reps']} passes over M={r['M']} of the {widx} layer, fp64 C oracle, "
+                      f"{r['seconds']:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def make_device_layer(torch, spear, L, copies):
+    dev = torch.device("cuda")
+    W = torch.from_numpy(L.W).to(dev)
+    packed, scale, zero = spear.spear_pack_w4(W)
+    del W
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    A, B, wg = bf(L.A_bits), bf(L.B_bits), bf(L.wg_bits)
+    sets = []
+    for c in range(copies):
+        if c == 0:
+            sets.append((packed, scale, zero, A, B, wg))
+        else:
+            sets.append(tuple(t.clone() for t in (packed, scale, zero, A, B, wg)))
+    return sets
+
+
+def run_ours(args, rank, world, torch, dist):
+    import w4_gemm_error_channel_b200 as spear
+    from synthetic import config_layers
+
+    cfg, batches, kind = WORKLOADS[args.workload]
+    L = config_layers(cfg, M=max(batches))[0]
+    N, K, r = L.N, L.K, L.rank
+    per_set = layer_bytes(max(batches), N, K, r)
+    copies = max(2, int(np.ceil(2 * L2_BYTES / per_set)) + 1)
+    if kind == "prefill":
+        copies = max(2, int(np.ceil(2 * L2_BYTES / (N * K // 2 + 2 * max(batches) * K))))
+    sets = make_device_layer(torch, spear, L, copies)
+    dev = torch.device("cuda")
+    xs = {M: torch.from_numpy(L.x(M).view(np.int16)).to(dev).view(torch.bfloat16) for M in batches}
+    ys = {M: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for M in batches}
+    plans = {M: spear.spear_gemm_plan(M, N, K, r) for M in batches}
+    ws = spear.alloc_workspace(max(p.workspace_bytes for p in plans.values()))
+    stream = torch.cuda.Stream()
+    calls_per_step = len(batches)
+
+    def step_calls(step_idx, use_ec=True):
+        for j, M in enumerate(batches):
+            p, s, z, A, B, wg = sets[(step_idx * calls_per_step + j) % copies]
+            ec = spear.EC(A, B, wg, L.b_g) if use_ec else None
+            spear.spear_w4ec_gemm(xs[M], p, s, z, ec, y=ys[M], workspace=ws, plan=plans[M], stream=stream)
+
+    def graph_of(n_steps, use_ec=True, only_M=None):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            # warm the path (library attributes, first launches) before capture
+            step_calls(0, use_ec)
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n_steps):
+                    if only_M is None:
+                        step_calls(i, use_ec)
+                    else:
+                        p, s, z, A, B, wg = sets[i % copies]
+                        ec = spear.EC(A, B, wg, L.b_g) if use_ec else None
+                        spear.spear_w4ec_gemm(xs[only_M], p, s, z, ec, y=ys[only_M], workspace=ws,
+                                              plan=plans[only_M], stream=stream)
+        return g
+
+    def time_graph(g, reps=1):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / 1e3
+
+    # Warm-up: W untimed steps (eager), then the graph once.
+    for i in range(args.warmup):
+        with torch.cuda.stream(stream):
+            step_calls(i)
+    stream.synchronize()
+    g_main = graph_of(args.steps)
+    g_main.replay()
+    stream.synchronize()
+
+    # Timed region: barrier + sync on both sides, K steps, max over ranks.
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_main = time_graph(g_main)
+    torch.cuda.synchronize()
+    if world > 1:
+        t = torch.tensor([t_main], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_main = float(t.item())
+        dist.barrier()
+    clocks = clk.summary()
+
+    step_bytes = sum(layer_bytes(M, N, K, r) for M in batches)
+    step_flops = sum(layer_flops(M, N, K, r) for M in batches)
+
+    # Per-batch timings (EC on and off) for the roofline and the EC overhead.
+    per_m = {}
+    n_sub = 64 if kind == "decode" else 8
+    for M in batches:
+        g_on = graph_of(n_sub, True, M)
+        g_off = graph_of(n_sub, False, M)
+        time_graph(g_on)
+        time_graph(g_off)
+        t_on = min(time_graph(g_on) for _ in range(3)) / n_sub
+        t_off = min(time_graph(g_off) for _ in range(3)) / n_sub
+        b_on, b_off = layer_bytes(M, N, K, r), layer_bytes(M, N, K, 0)
+        per_m[M] = {"us": t_on * 1e6, "us_no_ec": t_off * 1e6, "GBps": b_on / t_on / 1e9,
+                    "GBps_no_ec": b_off / t_off / 1e9, "TFLOPs": layer_flops(M, N, K, r) / t_on / 1e12,
+                    "ec_overhead": t_on / t_off - 1.0, "ec_byte_floor": b_on / b_off - 1.0,
+                    "plan": {"kernel": plans[M].kernel_id, "tile_n": plans[M].tile_n,
+                             "split_k": plans[M].split_k, "tile_m": plans[M].tile_m}}
+        del g_on, g_off
+
+    # e2e through the public API with pinned host buffers.
+    hx = {M: torch.from_numpy(L.x(M).view(np.int16)).view(torch.bfloat16).pin_memory() for M in batches}
+    hy = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in batches}
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step(i):
+        for j, M in enumerate(batches):
+            p, s, z, A, B, wg = sets[(i * calls_per_step + j) % copies]
+            xs[M].copy_(hx[M], non_blocking=True)
+            spear.spear_w4ec_gemm(xs[M], p, s, z, spear.EC(A, B, wg, L.b_g), y=ys[M], workspace=ws,
+                                  plan=plans[M], stream=stream)
+            hy[M].copy_(ys[M], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(2):
+            e2e_step(i)
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        e1.record(stream)
+    e1.synchronize()
+    t_e2e = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        t = torch.tensor([t_e2e], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_e2e = float(t.item())
+
+    import json as _json
+    peaks = {}
+    pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk_path):
+        peaks = _json.load(open(pk_path))
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    tc_peak = peaks.get("bf16_tflops", 1590.0)
+    peak_src = "measured" if peaks else "fallback"
+
+    if kind == "decode":
+        metric_val = step_bytes * args.steps * world / t_main / 1e9
+        unit = "GB/s"
+        e2e_val = step_bytes * e2e_steps * world / t_e2e / 1e9
+        Mr = max(b for b in batches if b <= 16) if any(b <= 16 for b in batches) else max(batches)
+        rl = {"bound": "hbm", "achieved": per_m[Mr]["GBps"], "peak": hbm_peak, "unit": "GB/s",
+              "frac": per_m[Mr]["GBps"] / hbm_peak, "traffic": None,
+              "kernel": f"spear_w4ec_gemm M={Mr} (splitk_w4_kernel with the EC pre-pass overlapped)",
+              "peak_source": f"{peak_src} hbm_gbs (copy)", "algorithmic_bytes": layer_bytes(Mr, N, K, r)}
+    else:
+        metric_val = step_flops * args.steps * world / t_main / 1e12
+        unit = "TFLOP/s"
+        e2e_val = step_flops * e2e_steps * world / t_e2e / 1e12
+        M0 = batches[0]
+        ach = per_m[M0]["TFLOPs"]
+        rl = {"bound": "tensor", "achieved": ach, "peak": tc_peak, "unit": "TFLOP/s", "frac": ach / tc_peak,
+              "traffic": None, "kernel": f"spear_w4ec_gemm M={M0}",
+              "peak_source": f"{peak_src} bf16_tflops (burst)", "algorithmic_flops": layer_flops(M0, N, K, r)}
+
+    out = {
+        "metric": "W4+gated-EC GEMM: decode GB/s and prefill TFLOP/s vs B200 roofline, 1 GPU",
+        "value": metric_val, "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_main / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: M in {batches}, N={N}, K={K}, EC rank {r}",
+                   "l2": f"weights rotate over {copies} copies ({copies * per_set / 2**20:.0f} MiB > 2x L2)",
+                   "parallelism": f"replicas x{world}", "timing": "CUDA graph of K steps, CUDA events"},
+        "e2e": {"value": e2e_val, "unit": unit,
+                "h2d_bytes_per_step": sum(2 * M * K for M in batches),
+                "d2h_bytes_per_step": sum(2 * M * N for M in batches)},
+        "gpu_launches": args.steps * sum(2 if r else 1 for _ in batches),
+        "roofline": rl,
+        "clocks": clocks,
+        "detail": {str(M): v for M, v in per_m.items()},
+    }
+    return out
+
+
+def prefill_summary(torch, spear):
+    """Secondary number: the prefill workload's TFLOP/s (M=2048, N=4096, K=14336, r=128)."""
+    from synthetic import config_layers
+    L = config_layers(3)[0]
+    M, N, K, r = 2048, L.N, L.K, L.rank
+    dev = torch.device("cuda")
+    sets = make_device_layer(torch, spear, L, 3)
+    x = torch.from_numpy(L.x(M).view(np.int16)).to(dev).view(torch.bfloat16)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    res = {}
+    for use_ec in (True, False):
+        plan = spear.spear_gemm_plan(M, N, K, r if use_ec else 0)
+        ws = spear.alloc_workspace(plan.workspace_bytes)
+        stream = torch.cuda.Stream()
+
+        def call(i):
+            p, s, z, A, B, wg = sets[i % 3]
+            ec = spear.EC(A, B, wg, L.b_g) if use_ec else None
+            spear.spear_w4ec_gemm(x, p, s, z, ec, y=y, workspace=ws, plan=plan, stream=stream)
+
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                call(i)
+        stream.synchronize()
+        n = 6
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(n):
+                call(i)
+            e1.record(stream)
+        e1.synchronize()
+        t = e0.elapsed_time(e1) / 1e3 / n
+        res["ec" if use_ec else "no_ec"] = {"us": t * 1e6,
+                                            "TFLOPs": layer_flops(M, N, K, r if use_ec else 0) / t / 1e12,
+                                            "plan": {"kernel": plan.kernel_id, "tile_n": plan.tile_n,
+                                                     "split_k": plan.split_k}}
+    res["ec_overhead"] = res["ec"]["us"] / res["no_ec"]["us"] - 1.0
+    return res
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg, batches, kind = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        # The reference arm is the CPU oracle (the pages ship no implementation).  Rank 0 only.
+        if rank != 0:
+            return
+        r = oracle_sample(args.workload, min(args.cpu_seconds, 15.0) / max(1, args.steps) * args.steps, batches)
+        if kind == "prefill":
+            val, unit = r["flops"] / r["seconds"] / 1e12, "TFLOP/s"
+        else:
+            val, unit = r["bytes"] / r["seconds"] / 1e9, "GB/s"
+        from synthetic import config_layers
+        L = config_layers(cfg, M=1)[0]
+        out = {"impl": "reference",
+               "metric": "W4+gated-EC GEMM: decode GB/s and prefill TFLOP/s vs B200 roofline, 1 GPU",
+               "value": val, "unit": unit, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": r["seconds"] / r["reps"] * 1e3, "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+               "config": {"workload": f"{args.workload}: M in {batches}, N={L.N}, K={L.K}, EC rank {L.rank}"},
+               "cpu_baseline": {"value": val, "unit": unit, "cores": r["cores"], "kind": "oracle",
+                                "sample": f"{r['reps']} passes over M={r['M']}, {r['seconds']:.1f} s"},
+               "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(out))
+        return
+
+    # Build the CPU baseline before any CUDA work (the oracle uses OpenMP threads).
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_obj(args.workload, args.cpu_seconds)
+
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    out = run_ours(args, rank, world, torch, dist)
+    if rank == 0 and not args.no_prefill and args.workload != "prefill":
+        import w4_gemm_error_channel_b200 as spear
+        try:
+            out["prefill"] = prefill_summary(torch, spear)
+        except Exception as e:  # secondary figure only; the main line stands on its own
+            out["prefill"] = {"error": str(e)}
+    if cpu is not None:
+        out["cpu_baseline"] = cpu
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    main()

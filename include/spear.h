@@ -1,0 +1,176 @@
+/*
+ * spear.h -- C ABI of the B200 (sm_100a) W4 linear layer with a per-token-gated
+ * low-rank error compensator (EC).
+ *
+ * Source: "SPEAR: A System for Post-Quantization Error-Adaptive Recovery
+ * Enabling Efficient Low-Bit LLM Serving".  The technical summary, section 2.1A
+ * (input-adaptive error compensators), defines the effective weight
+ * W + alpha * B diag(gamma(Ax)) A.  Section 3.1 quantises per output channel with
+ * RTN to 4 bits.  Section 2.2A (phase-adaptive fused kernel dispatch) fuses the
+ * EC into the low-bit GEMM's epilogue at decode and runs it as a separate
+ * kernel at prefill.  The abstract names the per-token gates.  This library
+ * computes, for every token row m of x:
+ *
+ *   y[m,n] = s[n] * sum_k x[m,k] (q[n,k] - z[n])  +  g[m] * sum_j t[m,j] B[j,n]
+ *   t[m,j] = sum_k x[m,k] A[k,j]
+ *   g[m]   = 1 / (1 + exp(-(sum_k x[m,k] w_g[k] + b_g)))
+ *
+ * with alpha = 1, gamma a scalar sigmoid gate, A stored [K, r], B stored [r, N].
+ *
+ * Conventions shared by every call:
+ *   - Pointers marked "device" are CUDA device pointers that the caller
+ *     allocates and owns.  The library keeps no pointer after a call returns.
+ *     Apart from the one-time tensor-map and attribute set-up noted below, it
+ *     allocates no device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Every device call is asynchronous on that stream.
+ *   - Argument errors are detected on the host, before anything is launched.
+ *     A CUDA launch or runtime error returns SPEAR_ERR_CUDA.
+ *   - Row-major layouts throughout.  bf16 = IEEE bfloat16 and fp16 = IEEE
+ *     binary16, both stored as 16-bit patterns.
+ *   - All device pointers must be 16-byte aligned (SPEAR_ERR_MISALIGNED).
+ */
+#ifndef SPEAR_H
+#define SPEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPEAR_API __attribute__((visibility("default")))
+#else
+#define SPEAR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SPEAR_OK = 0,
+    SPEAR_ERR_INVALID_ARG = 1,        /* NULL pointer, bad enum, negative size, ... */
+    SPEAR_ERR_UNSUPPORTED_SHAPE = 2,  /* N % 128, K % 64, rank outside 16..256 or not % 16 */
+    SPEAR_ERR_MISALIGNED = 3,         /* a device pointer is not 16-byte aligned */
+    SPEAR_ERR_WORKSPACE_TOO_SMALL = 4,
+    SPEAR_ERR_CUDA = 5,               /* CUDA runtime / launch failure */
+    SPEAR_ERR_TIMEOUT = 6             /* a bounded in-kernel wait gave up (see spear_get_device_status) */
+} spear_status;
+
+typedef enum { SPEAR_BF16 = 0, SPEAR_FP32 = 1 } spear_dtype;
+
+/* Kernel families the dispatcher chooses from (section 2.2A's two phases). */
+typedef enum {
+    SPEAR_KERNEL_AUTO = 0,      /* let spear_gemm_plan decide */
+    SPEAR_KERNEL_SPLITK = 1,    /* decode: split-K weight-streaming kernel (mma.sync on registers) plus
+                                   a separate EC pass, overlapped by programmatic dependent launch */
+    SPEAR_KERNEL_TC05 = 2       /* prefill: TMA + tcgen05/TMEM kernel, EC applied in its epilogue */
+} spear_kernel;
+
+/* Error compensator of one layer.  Pass NULL for a layer without EC (section
+ * 2.1B: compensators sit only at the selected, error-sensitive modules). */
+typedef struct {
+    const void* A;    /* device, bf16 [K, rank]   down-projection */
+    const void* B;    /* device, bf16 [rank, N]   up-projection */
+    const void* w_g;  /* device, bf16 [K]         gate weights */
+    float b_g;        /* gate bias (host value); -INFINITY gives g = 0 exactly */
+    int32_t rank;     /* r: 16..256, a multiple of 16 */
+} spear_ec;
+
+/* A launch plan.  Produced by spear_gemm_plan and read by spear_w4ec_gemm.  A
+ * caller may override kernel_id/split_k.  Invalid fields are rejected with
+ * SPEAR_ERR_INVALID_ARG. */
+typedef struct {
+    int32_t kernel_id;        /* spear_kernel */
+    int32_t tile_n;           /* weight rows per CTA */
+    int32_t split_k;          /* number of K slices reduced in the workspace (1 = none) */
+    int32_t tile_m;           /* token rows per CTA (or per launch chunk) */
+    int32_t flags;            /* reserved, 0 */
+    int32_t reserved;
+    size_t workspace_bytes;   /* minimum workspace for this (M, N, K, rank) */
+} spear_plan;
+
+/*
+ * spear_pack_w4 -- RTN per-output-channel asymmetric int4 quantisation
+ * (technical summary section 3.1: per-channel W4, RTN backend).
+ *
+ *   W       device, [N, K] fp32 (w_dtype = SPEAR_FP32) or bf16 (SPEAR_BF16)
+ *   packed  device, uint8 [N, K/2]: byte b of row n holds q[n,2b] in bits 0..3
+ *           and q[n,2b+1] in bits 4..7
+ *   scale   device, fp16 [N]    s[n]
+ *   zero    device, fp16 [N]    z[n], an integer in [0, 15]
+ *
+ * Per row, in IEEE fp32 operations, each correctly rounded:
+ *   lo = min(min_k W, 0), hi = max(max_k W, 0); hi == lo -> lo = -1, hi = 1;
+ *   s = fp16_rne((hi - lo) / 15); s == 0 -> row treated as all-zero;
+ *   z = clamp(rint(-lo / s), 0, 15); q = clamp(rint(W / s) + z, 0, 15)
+ *   (rint = round half to even).
+ * Requires N >= 1 and K >= 2 with K even.  Deterministic: the output is
+ * bit-identical on every run.
+ */
+SPEAR_API spear_status spear_pack_w4(const void* W, spear_dtype w_dtype, int64_t N, int64_t K,
+                           void* packed, void* scale, void* zero, void* stream);
+
+/*
+ * spear_debug_unpack_w4 -- test hook: the codes and the exact (q - z) values
+ * that the GEMM kernels feed their tensor-core operands.
+ *
+ *   packed     device, uint8 [N, K/2] (layout of spear_pack_w4)
+ *   zero       device, fp16 [N]
+ *   q_out      device, uint8 [N, K] or NULL
+ *   qz_out     device, bf16 [N, K] holding (q - z), exact in bf16; or NULL
+ */
+SPEAR_API spear_status spear_debug_unpack_w4(const void* packed, const void* zero, int64_t N, int64_t K,
+                                   void* q_out, void* qz_out, void* stream);
+
+/*
+ * spear_gemm_plan -- host-only choice of kernel and tiling for one
+ * (M, N, K, rank) problem (section 2.2A: the phase decides between the fused
+ * epilogue and a separate EC kernel; section 2.2C: decisions come from
+ * precomputed latency tables).  rank = 0 means no compensator.  `device` picks
+ * the SM count used for sizing; pass -1 for the current device.  Launches
+ * nothing.
+ */
+SPEAR_API spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int device,
+                             spear_plan* out);
+
+/*
+ * spear_w4ec_gemm -- y = x dequant(Wq)^T + g(x) * ((x A) B)  (section 2.1A).
+ *
+ *   plan       host, from spear_gemm_plan, or NULL (planned on the fly)
+ *   x          device, bf16 [M, K]
+ *   packed, scale, zero   from spear_pack_w4 for W [N, K]
+ *   ec         host struct with device pointers, or NULL for a plain W4 layer
+ *   y          device, [M, N], bf16 (y_dtype = SPEAR_BF16, one rounding at the
+ *              end) or fp32 (SPEAR_FP32, unrounded: a test/debug output)
+ *   workspace  device, >= plan->workspace_bytes.  Zero-fill it once before its
+ *              first use.  Every call leaves its control words zeroed again.
+ *              Calls that share a workspace must be ordered on one stream.
+ *
+ * Requires N % 128 == 0, K % 64 == 0, M >= 0 (M = 0 launches nothing).  The
+ * accumulation is fp32 throughout (the EC factors u = g t enter the prefill
+ * tensor cores as a bf16 hi/lo pair).  The output is deterministic for a given
+ * plan: no atomics take part in any floating-point sum.
+ */
+SPEAR_API spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, int64_t N, int64_t K,
+                             const void* packed, const void* scale, const void* zero,
+                             const spear_ec* ec, void* y, spear_dtype y_dtype,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * spear_get_device_status -- read (and optionally clear) the error word that
+ * bounded in-kernel waits set when they give up.  Synchronises `stream`.
+ * Returns SPEAR_OK, SPEAR_ERR_TIMEOUT, or SPEAR_ERR_CUDA.
+ */
+SPEAR_API spear_status spear_get_device_status(void* workspace, int clear, void* stream);
+
+/* Static string for a status code (never NULL). */
+SPEAR_API const char* spear_status_string(spear_status status);
+
+/* Library version, as MAJOR * 10000 + MINOR * 100 + PATCH. */
+SPEAR_API int spear_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPEAR_H */

@@ -1,0 +1,127 @@
+"""The C-ABI library on the host: it loads, exports what include/spear.h declares, and
+rejects bad arguments before launching anything (no GPU is needed for any of this)."""
+import ctypes
+import math
+import os
+import re
+import subprocess
+
+import pytest
+
+import w4_gemm_error_channel_b200 as spear
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spear.h")
+
+OK, INVALID, SHAPE, MISALIGNED, WS_SMALL = 0, 1, 2, 3, 4
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SPEAR_API\s+[\w\s\*]+?\b(spear_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for fn in ("spear_pack_w4", "spear_gemm_plan", "spear_w4ec_gemm", "spear_debug_unpack_w4",
+               "spear_status_string", "spear_get_device_status", "spear_version"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(spear.LIB_PATH)
+    for fn in declared_functions():
+        assert hasattr(lib, fn), fn
+    out = subprocess.run(["nm", "-D", "--defined-only", spear.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    missing = [fn for fn in declared_functions() if fn not in exported]
+    assert not missing, missing
+
+
+def test_status_strings_and_version():
+    for code in range(7):
+        assert spear.spear_status_string(code)
+    assert spear.spear_status_string(99) == "unknown status"
+    assert spear.spear_version() >= 100
+
+
+def _plan(M, N, K, r):
+    p = spear.spear_plan()
+    return spear._lib.spear_gemm_plan(M, N, K, r, -1, ctypes.byref(p)), p
+
+
+@pytest.mark.parametrize("M,N,K,r", [(1, 4096, 4096, 64), (16, 4096, 4096, 64), (64, 22016, 4096, 64),
+                                     (2048, 4096, 14336, 128), (4, 512, 512, 16), (4096, 16384, 2048, 0),
+                                     (256, 2048, 8192, 32), (7, 128, 64, 0)])
+def test_plan_is_consistent(M, N, K, r):
+    st, p = _plan(M, N, K, r)
+    assert st == OK
+    assert p.kernel_id in (spear.SPEAR_KERNEL_SPLITK, spear.SPEAR_KERNEL_TC05)
+    assert N % p.tile_n == 0 and K % (p.split_k * 64) == 0
+    assert p.workspace_bytes >= 128 * 1024
+    if r:
+        assert p.workspace_bytes >= 128 * 1024 + 4 * M * r
+
+
+@pytest.mark.parametrize("M,N,K,r,want", [(1, 100, 4096, 0, SHAPE), (1, 4096, 100, 0, SHAPE),
+                                          (1, 4096, 4096, 8, SHAPE), (1, 4096, 4096, 72, SHAPE),
+                                          (1, 4096, 4096, 512, SHAPE), (-1, 4096, 4096, 0, INVALID),
+                                          (1, 0, 4096, 0, INVALID), (70000, 4096, 4096, 0, SHAPE)])
+def test_plan_rejects_bad_shapes(M, N, K, r, want):
+    st, _ = _plan(M, N, K, r)
+    assert st == want
+
+
+def _gemm(M=4, N=512, K=512, x=0x1000, packed=0x2000, scale=0x3000, zero=0x4000, y=0x5000, ws=0x6000,
+          ws_bytes=1 << 30, ec=None, y_dtype=0, plan=None):
+    P = ctypes.c_void_p
+    return spear._lib.spear_w4ec_gemm(plan, P(x), M, N, K, P(packed), P(scale), P(zero), ec, P(y), y_dtype, P(ws),
+                                      ws_bytes, None)
+
+
+def test_gemm_host_checks_return_before_launch():
+    # Fake, never-dereferenced addresses: every case below must fail (or finish) on the host.
+    assert _gemm(x=0) == INVALID
+    assert _gemm(y=0) == INVALID
+    assert _gemm(ws=0) == INVALID
+    assert _gemm(y_dtype=7) == INVALID
+    assert _gemm(N=500) == SHAPE
+    assert _gemm(K=100) == SHAPE
+    assert _gemm(x=0x1008) == MISALIGNED
+    assert _gemm(packed=0x2001) == MISALIGNED
+    assert _gemm(ws=0x6004) == MISALIGNED
+    assert _gemm(ws_bytes=1024) == WS_SMALL
+    assert _gemm(M=0) == OK               # empty batch: nothing to launch
+    ec = spear.spear_ec(0x7000, 0x8000, 0x9000, 0.0, 16)
+    assert _gemm(ec=ctypes.byref(ec), ws_bytes=1024) == WS_SMALL
+    bad = spear.spear_ec(0x7000, 0, 0x9000, 0.0, 16)
+    assert _gemm(ec=ctypes.byref(bad)) == INVALID
+    nan = spear.spear_ec(0x7000, 0x8000, 0x9000, math.nan, 16)
+    assert _gemm(ec=ctypes.byref(nan)) == INVALID
+    r8 = spear.spear_ec(0x7000, 0x8000, 0x9000, 0.0, 8)
+    assert _gemm(ec=ctypes.byref(r8)) == SHAPE
+    mis = spear.spear_ec(0x7008, 0x8000, 0x9000, 0.0, 16)
+    assert _gemm(ec=ctypes.byref(mis)) == MISALIGNED
+
+
+def test_gemm_rejects_bad_plans():
+    st, p = _plan(4, 512, 512, 0)
+    assert st == OK
+    for field, val in (("kernel_id", 9), ("split_k", 0), ("split_k", 3), ("tile_n", 48), ("tile_m", 12)):
+        q = spear.spear_plan.from_buffer_copy(p)
+        setattr(q, field, val)
+        assert _gemm(plan=ctypes.byref(q)) == INVALID, field
+
+
+def test_pack_and_unpack_host_checks():
+    P = ctypes.c_void_p
+    lib = spear._lib
+    assert lib.spear_pack_w4(P(0), 1, 8, 8, P(0x2000), P(0x3000), P(0x4000), None) == INVALID
+    assert lib.spear_pack_w4(P(0x1000), 5, 8, 8, P(0x2000), P(0x3000), P(0x4000), None) == INVALID
+    assert lib.spear_pack_w4(P(0x1000), 1, 8, 7, P(0x2000), P(0x3000), P(0x4000), None) == SHAPE
+    assert lib.spear_pack_w4(P(0x1000), 1, 0, 8, P(0x2000), P(0x3000), P(0x4000), None) == INVALID
+    assert lib.spear_pack_w4(P(0x1004), 1, 8, 8, P(0x2000), P(0x3000), P(0x4000), None) == MISALIGNED
+    assert lib.spear_debug_unpack_w4(P(0x1000), P(0x2000), 8, 8, P(0), P(0), None) == INVALID
+    assert lib.spear_debug_unpack_w4(P(0x1000), P(0x2000), 8, 9, P(0x3000), P(0), None) == SHAPE
+    assert lib.spear_get_device_status(P(0), 0, None) == INVALID

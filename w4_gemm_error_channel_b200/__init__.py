@@ -1,0 +1,198 @@
+"""Python binding of ``libspear.so``: the B200 W4 linear layer with a per-token-gated
+low-rank error compensator (SPEAR: Post-Quantization Error-Adaptive Recovery,
+technical summary section 2.1A).
+
+Argument marshalling only.  Every step of the layer runs in the library's CUDA
+kernels; PyTorch supplies device memory and streams.  The names match the C ABI
+in ``include/spear.h``.  There is no CPU fallback: if the library is missing or
+fails to load, importing this package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libspear.so")
+
+SPEAR_OK = 0
+SPEAR_BF16, SPEAR_FP32 = 0, 1
+SPEAR_KERNEL_AUTO, SPEAR_KERNEL_SPLITK, SPEAR_KERNEL_TC05 = 0, 1, 2
+STATUS_NAMES = {0: "SPEAR_OK", 1: "SPEAR_ERR_INVALID_ARG", 2: "SPEAR_ERR_UNSUPPORTED_SHAPE",
+                3: "SPEAR_ERR_MISALIGNED", 4: "SPEAR_ERR_WORKSPACE_TOO_SMALL", 5: "SPEAR_ERR_CUDA",
+                6: "SPEAR_ERR_TIMEOUT"}
+EXPORTED = ["spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_w4ec_gemm",
+            "spear_get_device_status", "spear_status_string", "spear_version"]
+
+
+class SpearError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)} ({spear_status_string(status)})")
+
+
+class spear_plan(ctypes.Structure):
+    _fields_ = [("kernel_id", ctypes.c_int32), ("tile_n", ctypes.c_int32), ("split_k", ctypes.c_int32),
+                ("tile_m", ctypes.c_int32), ("flags", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+    def __repr__(self):
+        return (f"spear_plan(kernel_id={self.kernel_id}, tile_n={self.tile_n}, split_k={self.split_k}, "
+                f"tile_m={self.tile_m}, workspace_bytes={self.workspace_bytes})")
+
+
+class spear_ec(ctypes.Structure):
+    _fields_ = [("A", ctypes.c_void_p), ("B", ctypes.c_void_p), ("w_g", ctypes.c_void_p),
+                ("b_g", ctypes.c_float), ("rank", ctypes.c_int32)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m w4_gemm_error_channel_b200.build` "
+                          "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    lib.spear_pack_w4.argtypes = [P, ctypes.c_int, I64, I64, P, P, P, P]
+    lib.spear_debug_unpack_w4.argtypes = [P, P, I64, I64, P, P, P]
+    lib.spear_gemm_plan.argtypes = [I64, I64, I64, ctypes.c_int32, ctypes.c_int, ctypes.POINTER(spear_plan)]
+    lib.spear_w4ec_gemm.argtypes = [ctypes.POINTER(spear_plan), P, I64, I64, I64, P, P, P,
+                                    ctypes.POINTER(spear_ec), P, ctypes.c_int, P, ctypes.c_size_t, P]
+    lib.spear_get_device_status.argtypes = [P, ctypes.c_int, P]
+    lib.spear_status_string.argtypes = [ctypes.c_int]
+    lib.spear_status_string.restype = ctypes.c_char_p
+    lib.spear_version.restype = ctypes.c_int
+    for fn in ("spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_w4ec_gemm",
+               "spear_get_device_status"):
+        getattr(lib, fn).restype = ctypes.c_int
+    return lib
+
+
+_lib = _load()
+
+
+def _check(fn: str, status: int):
+    if status != SPEAR_OK:
+        raise SpearError(fn, status)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def spear_status_string(status: int) -> str:
+    return _lib.spear_status_string(int(status)).decode()
+
+
+def spear_version() -> int:
+    return int(_lib.spear_version())
+
+
+@dataclasses.dataclass
+class EC:
+    """One layer's error compensator: A bf16 [K,r], B bf16 [r,N], w_g bf16 [K], b_g float."""
+    A: torch.Tensor
+    B: torch.Tensor
+    w_g: torch.Tensor
+    b_g: float = 0.0
+
+    @property
+    def rank(self) -> int:
+        return int(self.A.shape[1])
+
+    def as_c(self) -> spear_ec:
+        for name in ("A", "B", "w_g"):
+            t = getattr(self, name)
+            _dev(t, name)
+            if t.dtype != torch.bfloat16:
+                raise ValueError(f"EC.{name} must be bf16")
+        return spear_ec(self.A.data_ptr(), self.B.data_ptr(), self.w_g.data_ptr(), float(self.b_g), self.rank)
+
+
+def spear_pack_w4(W: torch.Tensor, packed=None, scale=None, zero=None, stream=None):
+    """RTN per-channel int4 packing of W [N,K] (fp32 or bf16) -> (packed u8 [N,K/2], scale f16 [N], zero f16 [N])."""
+    _dev(W, "W")
+    N, K = W.shape
+    if W.dtype == torch.float32:
+        wd = SPEAR_FP32
+    elif W.dtype == torch.bfloat16:
+        wd = SPEAR_BF16
+    else:
+        raise ValueError("W must be fp32 or bf16")
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device) if packed is None else packed
+    scale = torch.empty(N, dtype=torch.float16, device=W.device) if scale is None else scale
+    zero = torch.empty(N, dtype=torch.float16, device=W.device) if zero is None else zero
+    _check("spear_pack_w4", _lib.spear_pack_w4(_p(W), wd, N, K, _p(packed), _p(scale), _p(zero), _stream(stream)))
+    return packed, scale, zero
+
+
+def spear_debug_unpack_w4(packed: torch.Tensor, zero: torch.Tensor, K: int, want_q=True, want_qz=True,
+                          stream=None):
+    """Test hook: (q u8 [N,K] or None, (q - z) bf16 [N,K] or None)."""
+    _dev(packed, "packed")
+    N = packed.shape[0]
+    q = torch.empty((N, K), dtype=torch.uint8, device=packed.device) if want_q else None
+    qz = torch.empty((N, K), dtype=torch.bfloat16, device=packed.device) if want_qz else None
+    _check("spear_debug_unpack_w4",
+           _lib.spear_debug_unpack_w4(_p(packed), _p(zero), N, K, _p(q), _p(qz), _stream(stream)))
+    return q, qz
+
+
+def spear_gemm_plan(M: int, N: int, K: int, rank: int = 0, device: int = -1) -> spear_plan:
+    plan = spear_plan()
+    _check("spear_gemm_plan", _lib.spear_gemm_plan(M, N, K, rank, device, ctypes.byref(plan)))
+    return plan
+
+
+def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace (the control words must start at zero)."""
+    return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8,
+                       device=device if device is not None else torch.cuda.current_device())
+
+
+def spear_w4ec_gemm(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
+                    ec: Optional[EC] = None, y: Optional[torch.Tensor] = None, y_dtype=torch.bfloat16,
+                    workspace: Optional[torch.Tensor] = None, plan: Optional[spear_plan] = None, stream=None):
+    """y = x dequant(Wq)^T + g(x) (x A) B.  Returns y [M,N] (bf16, or fp32 for checks)."""
+    _dev(x, "x")
+    if x.dtype != torch.bfloat16:
+        raise ValueError("x must be bf16")
+    M, K = x.shape
+    N = packed.shape[0]
+    rank = ec.rank if ec is not None else 0
+    if plan is None:
+        plan = spear_gemm_plan(M, N, K, rank, x.device.index)
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=x.device)
+    yd = SPEAR_FP32 if y.dtype == torch.float32 else SPEAR_BF16
+    if workspace is None:
+        workspace = alloc_workspace(plan.workspace_bytes, x.device)
+    ec_c = ctypes.byref(ec.as_c()) if ec is not None else None
+    _check("spear_w4ec_gemm",
+           _lib.spear_w4ec_gemm(ctypes.byref(plan), _p(x), M, N, K, _p(packed), _p(scale), _p(zero), ec_c,
+                                _p(y), yd, _p(workspace), workspace.numel(), _stream(stream)))
+    return y
+
+
+def spear_get_device_status(workspace: torch.Tensor, clear: bool = True, stream=None) -> int:
+    return int(_lib.spear_get_device_status(_p(workspace), int(clear), _stream(stream)))
+
+
+def loaded_library_path() -> str:
+    return LIB_PATH
