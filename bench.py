@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the secondary prefill measurement")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every valid decode tiling for the workload's batches and print a table")
     return ap.parse_args()
 
 
@@ -72,25 +74,29 @@ def layer_flops(M, N, K, r):
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples (every 100 ms, timestamped) for the whole run; summary() keeps the ones
+    that fall inside a given wall-clock window."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
+        self.lines = []
 
-    def __enter__(self):
+    def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+        time.sleep(0.5)  # let the first samples arrive
         return self
 
-    def __exit__(self, *exc):
-        self.lines = []
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -99,26 +105,31 @@ class ClockSampler:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            self.proc = None
 
-    def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
+    def samples(self):
+        import datetime
+        out = []
+        for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, mx = float(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+            active = [nm for nm, v in zip(self.REASONS, parts[6:10]) if v.lower().startswith("active")]
+            out.append((ts, sm, mx, active))
+        return out
+
+    def summary(self, t0, t1, where):
+        sel = [s for s in self.samples() if t0 <= s[0] <= t1]
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "window": where}
+        reasons = sorted({r for s in sel for r in s[3]})
+        return {"sm_mhz": statistics.median(s[1] for s in sel), "sm_max_mhz": max(s[2] for s in sel),
+                "reasons": reasons, "samples": len(sel), "window": where}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -241,18 +252,30 @@ def run_ours(args, rank, world, torch, dist):
     stream.synchronize()
 
     # Timed region: barrier + sync on both sides, K steps, max over ranks.
+    clk = ClockSampler(torch.cuda.current_device()).start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        t_main = time_graph(g_main)
+    w0 = time.time()
+    t_main = time_graph(g_main)
     torch.cuda.synchronize()
+    w1 = time.time()
     if world > 1:
         t = torch.tensor([t_main], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         t_main = float(t.item())
         dist.barrier()
-    clocks = clk.summary()
+    # The timed region is often shorter than the 100 ms sampling period: then the clocks are
+    # read during an untimed soak of the same graph right after it.
+    soak0 = time.time()
+    while time.time() - soak0 < 1.5:
+        time_graph(g_main)
+    soak1 = time.time()
+    time.sleep(0.3)
+    clk.stop()
+    clocks = clk.summary(w0, w1, "timed region")
+    if clocks["samples"] < 3:
+        clocks = clk.summary(soak0, soak1, "soak of the timed graph right after the timed region")
 
     step_bytes = sum(layer_bytes(M, N, K, r) for M in batches)
     step_flops = sum(layer_flops(M, N, K, r) for M in batches)
@@ -395,8 +418,69 @@ def prefill_summary(torch, spear):
     return res
 
 
+def sweep_plans(args):
+    """Time each valid (tile_n, split_k) decode plan in a chained CUDA graph of layer calls."""
+    import torch
+    import w4_gemm_error_channel_b200 as spear
+    from synthetic import config_layers
+    torch.cuda.set_device(0)
+    cfg, batches, kind = WORKLOADS[args.workload]
+    L = config_layers(cfg, M=max(batches))[0]
+    N, K, r = L.N, L.K, L.rank
+    per_set = layer_bytes(max(batches), N, K, r)
+    copies = max(2, int(np.ceil(2 * L2_BYTES / per_set)) + 1)
+    sets = make_device_layer(torch, spear, L, copies)
+    dev = torch.device("cuda")
+    stream = torch.cuda.Stream()
+    rows = []
+    for M in batches:
+        x = torch.from_numpy(L.x(M).view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        base = spear.spear_gemm_plan(M, N, K, r)
+        ws = spear.alloc_workspace(base.workspace_bytes)
+        for tile_n in (16, 32, 64, 128):
+            for split in (1, 2, 4, 8):
+                for use_ec in (True, False):
+                    plan = spear.spear_plan.from_buffer_copy(base)
+                    plan.tile_n, plan.split_k = tile_n, split
+                    n_calls = 64
+
+                    def call(i):
+                        p, sc, z, A, B, wg = sets[i % copies]
+                        ec = spear.EC(A, B, wg, L.b_g) if use_ec else None
+                        spear.spear_w4ec_gemm(x, p, sc, z, ec, y=y, workspace=ws, plan=plan, stream=stream)
+                    try:
+                        with torch.cuda.stream(stream):
+                            call(0)
+                        stream.synchronize()
+                    except spear.SpearError:
+                        continue
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.stream(stream):
+                        with torch.cuda.graph(g, stream=stream):
+                            for i in range(n_calls):
+                                call(i)
+                    best = 1e9
+                    for _ in range(5):
+                        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        with torch.cuda.stream(stream):
+                            e0.record(stream)
+                            g.replay()
+                            e1.record(stream)
+                        e1.synchronize()
+                        best = min(best, e0.elapsed_time(e1) * 1e3 / n_calls)
+                    del g
+                    rows.append({"M": M, "N": N, "K": K, "rank": r if use_ec else 0, "tile_n": tile_n,
+                                 "split_k": split, "us": best,
+                                 "GBps": layer_bytes(M, N, K, r if use_ec else 0) / best / 1e3})
+    print(json.dumps({"workload": args.workload, "sweep": rows}))
+
+
 def main():
     args = parse()
+    if args.sweep:
+        sweep_plans(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -58,7 +58,9 @@ def test_plan_is_consistent(M, N, K, r):
     st, p = _plan(M, N, K, r)
     assert st == OK
     assert p.kernel_id in (spear.SPEAR_KERNEL_SPLITK, spear.SPEAR_KERNEL_TC05)
-    assert N % p.tile_n == 0 and K % (p.split_k * 64) == 0
+    assert N % p.tile_n == 0
+    k_slice = ((K + p.split_k - 1) // p.split_k + 63) // 64 * 64
+    assert (p.split_k - 1) * k_slice < K          # no empty K slice
     assert p.workspace_bytes >= 128 * 1024
     if r:
         assert p.workspace_bytes >= 128 * 1024 + 4 * M * r
@@ -93,6 +95,7 @@ def test_gemm_host_checks_return_before_launch():
     assert _gemm(ws=0x6004) == MISALIGNED
     assert _gemm(ws_bytes=1024) == WS_SMALL
     assert _gemm(M=0) == OK               # empty batch: nothing to launch
+    assert _gemm(M=0, x=0, y=0) == OK     # ... and may come without activation/output buffers
     ec = spear.spear_ec(0x7000, 0x8000, 0x9000, 0.0, 16)
     assert _gemm(ec=ctypes.byref(ec), ws_bytes=1024) == WS_SMALL
     bad = spear.spear_ec(0x7000, 0, 0x9000, 0.0, 16)
@@ -108,7 +111,7 @@ def test_gemm_host_checks_return_before_launch():
 def test_gemm_rejects_bad_plans():
     st, p = _plan(4, 512, 512, 0)
     assert st == OK
-    for field, val in (("kernel_id", 9), ("split_k", 0), ("split_k", 3), ("tile_n", 48), ("tile_m", 12)):
+    for field, val in (("kernel_id", 9), ("split_k", 0), ("split_k", 9), ("tile_n", 48), ("tile_m", 12)):
         q = spear.spear_plan.from_buffer_copy(p)
         setattr(q, field, val)
         assert _gemm(plan=ctypes.byref(q)) == INVALID, field

@@ -1,7 +1,7 @@
 // api.cu -- the C ABI declared in include/spear.h: argument checks, planning, workspace layout
-// and kernel dispatch.  Host code only; the kernels live in pack.cu, splitk.cu and tc05.cu.
+// and kernel dispatch.  Host code only; the kernels live in pack.cu and decode.cu.
 #include <math.h>
-#include <mutex>
+#include <cmath>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -14,8 +14,6 @@ constexpr int MAX_DEVICES = 64;
 constexpr int DEFAULT_SMS = 148;  // B200, used when no device can be queried (host-only planning)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 int device_sms(int device) {
     static int cache[MAX_DEVICES] = {0};
@@ -32,21 +30,6 @@ int device_sms(int device) {
     return cache[device];
 }
 
-// One-time, per-device function attributes (dynamic shared memory above 48 KB).
-cudaError_t ensure_attributes() {
-    static std::once_flag flags[MAX_DEVICES];
-    static cudaError_t results[MAX_DEVICES];
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
-    std::call_once(flags[dev], [dev]() {
-        results[dev] = cudaFuncSetAttribute(ec_prepass_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)ec_prepass_max_smem_bytes());
-    });
-    return results[dev];
-}
-
 spear_status check_shape(int64_t M, int64_t N, int64_t K, int32_t rank) {
     if (M < 0 || N <= 0 || K <= 0 || rank < 0) return SPEAR_ERR_INVALID_ARG;
     if (N % 128 != 0 || K % 64 != 0) return SPEAR_ERR_UNSUPPORTED_SHAPE;
@@ -55,50 +38,59 @@ spear_status check_shape(int64_t M, int64_t N, int64_t K, int32_t rank) {
     return SPEAR_OK;
 }
 
-// Workspace layout for a given problem and plan.
-struct Layout {
-    size_t u_off = 0, ec_part_off = 0, part_off = 0, total = 0;
-    int64_t ec_k_per_cta = 0, ec_splits = 0;
-};
-
-Layout layout_for(int64_t M, int64_t N, int64_t K, int32_t rank, const spear_plan& p, int sms) {
-    Layout L;
-    size_t off = CTRL_BYTES;
-    if (rank > 0 && M > 0) {
-        L.ec_k_per_cta = ec_prepass_k_per_cta(M, K, sms);
-        L.ec_splits = ec_prepass_splits(K, L.ec_k_per_cta);
-        L.u_off = off;
-        off = align_up(off + sizeof(float) * (size_t)M * rank, 256);
-        L.ec_part_off = off;
-        off = align_up(off + sizeof(float) * (size_t)L.ec_splits * M * (rank + 1), 256);
-    }
-    if (p.split_k > 1) {
-        L.part_off = off;
-        off = align_up(off + sizeof(float) * (size_t)p.split_k * M * N, 256);
-    }
-    L.total = off;
-    return L;
-}
-
 int nb_for_tile_m(int tile_m) { return tile_m <= 8 ? 1 : (tile_m <= 16 ? 2 : 4); }
 
-spear_status plan_splitk(int64_t M, int64_t N, int64_t K, int sms, spear_plan* p) {
+// K codes per slice for S slices: a multiple of 64, so every lane's 32-code piece is whole.
+int64_t k_slice_for(int64_t K, int64_t S) { return ((K + S - 1) / S + 63) / 64 * 64; }
+int wpw_for(int64_t k_slice) { return (int)((k_slice + 511) / 512); }
+int ec_jr_for(int32_t rank, int64_t S) {
+    if (rank <= 0) return 0;
+    return (int)(((rank + S - 1) / S + 3) / 4 * 4);
+}
+// Workspace: only the zeroed prefix (control block + EC accumulators); split-K partial sums meet
+// in distributed shared memory.
+size_t workspace_bytes_for() { return ZEROED_BYTES; }
+
+int ec_splits_for(int64_t K) { return (int)((K + 63) / 64); }     // 64 rows of A per EC CTA
+
+// Decode plan.  Every weight byte of a CTA (16*g rows x K/S codes, 128 threads) is requested up
+// front; the S K slices of a row tile form a cluster (S in {1, 2, 4, 8}).  The cost model prefers
+// tilings that spread the weight bytes evenly over all SMs (many small CTAs stream best), then
+// the least re-reading of activations from L2, then fewer slices.
+spear_status plan_decode(int64_t M, int64_t N, int64_t K, int sms, spear_plan* p) {
     const int nb = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
     const int64_t tm = 8 * nb;
-    const int64_t mchunks = (M + tm - 1) / tm;
-    int g = 4;
-    if (nb <= 2 && (N / 64) * mchunks > 4 * (int64_t)sms && N % 128 == 0) g = 8;
-    const int64_t rt = 16 * g;
-    const int64_t tiles = (N / rt) * mchunks;
-    int64_t want = (2 * (int64_t)sms + tiles - 1) / tiles;
-    int64_t smax = K / 512;
-    if (smax < 1) smax = 1;
-    int64_t s = want < smax ? want : smax;
-    if (s < 1) s = 1;
-    while (s > 1 && (K % (s * 64) != 0 || (size_t)tiles > GEMM_TICKETS_MAX)) --s;
+    const int64_t ml = M < LAUNCH_TOKENS_MAX ? M : LAUNCH_TOKENS_MAX;
+    const int64_t mchunks = (ml + tm - 1) / tm;
+    const double wbytes = (double)N * K / 2;
+    const double hbm = 6.5e12, l2 = 20e12;
+    double best = 1e300;
+    int best_g = 1, best_s = 1;
+    const int gs[4] = {1, 2, 4, 8};
+    const int ss[4] = {1, 2, 4, 8};
+    for (int gi = 0; gi < 4; ++gi) {
+        const int g = gs[gi];
+        const int64_t rt = 16 * g;
+        if (N % rt != 0) continue;
+        const int64_t tiles = (N / rt) * mchunks;
+        for (int si = 0; si < 4; ++si) {
+            const int64_t S = ss[si];
+            const int64_t ksl = k_slice_for(K, S);
+            if ((S - 1) * ksl >= K) continue;               // no empty slices
+            if (!decode_config_supported(nb, g, wpw_for(ksl))) continue;
+            const double ctas = (double)tiles * S;
+            // Work per SM in whole CTAs (4 CTAs of 128 threads resident per SM).
+            const double rounds = std::ceil(ctas / (4.0 * sms));
+            const double balance = rounds * 4.0 * sms / ctas;   // >= 1; 1 = even
+            const double spread = ctas < sms ? (double)sms / ctas : 1.0;
+            const double xbytes = (double)(N / rt) * M * K * 2;
+            const double cost = wbytes / hbm * balance * spread + xbytes / l2 + (S > 1 ? 0.2e-6 : 0.0);
+            if (cost < best * 0.999) { best = cost; best_g = g; best_s = (int)S; }
+        }
+    }
     p->kernel_id = SPEAR_KERNEL_SPLITK;
-    p->tile_n = (int32_t)rt;
-    p->split_k = (int32_t)s;
+    p->tile_n = 16 * best_g;
+    p->split_k = best_s;
     p->tile_m = (int32_t)tm;
     p->flags = 0;
     p->reserved = 0;
@@ -106,16 +98,19 @@ spear_status plan_splitk(int64_t M, int64_t N, int64_t K, int sms, spear_plan* p
 }
 
 spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K) {
+    (void)M;
     if (p.kernel_id != SPEAR_KERNEL_SPLITK) return SPEAR_ERR_INVALID_ARG;
-    if (p.split_k < 1 || K % ((int64_t)p.split_k * 64) != 0) return SPEAR_ERR_INVALID_ARG;
+    if (!(p.split_k == 1 || p.split_k == 2 || p.split_k == 4 || p.split_k == 8)) return SPEAR_ERR_INVALID_ARG;
     const int nb = nb_for_tile_m(p.tile_m);
     if (p.tile_m != 8 * nb) return SPEAR_ERR_INVALID_ARG;
+    if (p.tile_n % 16 != 0 || p.tile_n <= 0) return SPEAR_ERR_INVALID_ARG;
     const int g = p.tile_n / 16;
-    if (p.tile_n % 16 != 0 || !(g == 1 || g == 2 || g == 4 || g == 8) || (g == 8 && nb > 2))
-        return SPEAR_ERR_INVALID_ARG;
+    const int64_t ksl = k_slice_for(K, p.split_k);
+    if ((p.split_k - 1) * ksl >= K) return SPEAR_ERR_INVALID_ARG;
+    if (!decode_config_supported(nb, g, wpw_for(ksl))) return SPEAR_ERR_INVALID_ARG;
     if (N % p.tile_n != 0) return SPEAR_ERR_INVALID_ARG;
-    const int64_t tiles = (N / p.tile_n) * ((M + p.tile_m - 1) / p.tile_m);
-    if (p.split_k > 1 && (size_t)tiles > GEMM_TICKETS_MAX) return SPEAR_ERR_INVALID_ARG;
+    // Consumer counters: at most GROUPS_MAX groups of GEMM CTAs per token chunk.
+    if ((N / p.tile_n) * p.split_k > (int64_t)GROUPS_MAX * CONSUMER_GROUP) return SPEAR_ERR_INVALID_ARG;
     return SPEAR_OK;
 }
 
@@ -166,9 +161,9 @@ spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int 
     if (st != SPEAR_OK) return st;
     const int sms = device_sms(device);
     spear_plan p = {};
-    st = plan_splitk(M > 0 ? M : 1, N, K, sms, &p);
+    st = plan_decode(M > 0 ? M : 1, N, K, sms, &p);
     if (st != SPEAR_OK) return st;
-    p.workspace_bytes = layout_for(M, N, K, rank, p, sms).total;
+    p.workspace_bytes = workspace_bytes_for();
     *out = p;
     return SPEAR_OK;
 }
@@ -176,7 +171,9 @@ spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int 
 spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, int64_t N, int64_t K,
                              const void* packed, const void* scale, const void* zero, const spear_ec* ec, void* y,
                              spear_dtype y_dtype, void* workspace, size_t workspace_bytes, void* stream) {
-    if (!x || !packed || !scale || !zero || !y || !workspace) return SPEAR_ERR_INVALID_ARG;
+    // An empty batch may come with NULL activation/output pointers (M = 0 launches nothing).
+    if (!packed || !scale || !zero || !workspace) return SPEAR_ERR_INVALID_ARG;
+    if (M != 0 && (!x || !y)) return SPEAR_ERR_INVALID_ARG;
     if (y_dtype != SPEAR_BF16 && y_dtype != SPEAR_FP32) return SPEAR_ERR_INVALID_ARG;
     const int32_t rank = ec ? ec->rank : 0;
     if (ec && (!ec->A || !ec->B || !ec->w_g)) return SPEAR_ERR_INVALID_ARG;
@@ -184,8 +181,8 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
     spear_status st = check_shape(M, N, K, rank);
     if (st != SPEAR_OK) return st;
     if (ec && rank == 0) return SPEAR_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(x) || !aligned16(packed) || !aligned16(scale) || !aligned16(zero) || !aligned16(y) ||
-        !aligned16(workspace))
+    if ((M != 0 && (!aligned16(x) || !aligned16(y))) || !aligned16(packed) || !aligned16(scale) ||
+        !aligned16(zero) || !aligned16(workspace))
         return SPEAR_ERR_MISALIGNED;
     if (ec && (!aligned16(ec->A) || !aligned16(ec->B) || !aligned16(ec->w_g))) return SPEAR_ERR_MISALIGNED;
     if (M == 0) return SPEAR_OK;
@@ -195,56 +192,54 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
     if (plan) {
         p = *plan;
     } else {
-        st = plan_splitk(M, N, K, sms, &p);
+        st = plan_decode(M, N, K, sms, &p);
         if (st != SPEAR_OK) return st;
     }
     st = validate_plan(p, M, N, K);
     if (st != SPEAR_OK) return st;
-    const Layout L = layout_for(M, N, K, rank, p, sms);
-    if (workspace_bytes < L.total) return SPEAR_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace_bytes < workspace_bytes_for()) return SPEAR_ERR_WORKSPACE_TOO_SMALL;
 
-    if (ensure_attributes() != cudaSuccess) return SPEAR_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
     unsigned char* ws = (unsigned char*)workspace;
-    unsigned* ec_tickets = (unsigned*)(ws + CTRL_HEADER_BYTES);
-    unsigned* gemm_tickets = ec_tickets + EC_TICKETS_MAX;
+    unsigned* ctrl = (unsigned*)ws;
+    const int nb = nb_for_tile_m(p.tile_m);
+    const int g = p.tile_n / 16;
 
-    float* u = nullptr;
-    if (ec) {
-        EcPrepassArgs ea;
-        ea.x = (const uint16_t*)x;
-        ea.A = (const uint16_t*)ec->A;
-        ea.wg = (const uint16_t*)ec->w_g;
-        ea.b_g = ec->b_g;
-        ea.M = M;
-        ea.K = K;
-        ea.rank = rank;
-        ea.k_per_cta = L.ec_k_per_cta;
-        ea.ec_part = (float*)(ws + L.ec_part_off);
-        ea.u = (float*)(ws + L.u_off);
-        ea.tickets = ec_tickets;
-        if (launch_ec_prepass(ea, s) != cudaSuccess) return SPEAR_ERR_CUDA;
-        u = ea.u;
-    }
-
-    SplitKArgs a;
-    a.x = (const uint16_t*)x;
+    DecodeArgs a;
     a.packed = (const uint8_t*)packed;
     a.scale = (const __half*)scale;
     a.zero = (const __half*)zero;
+    a.A = ec ? (const uint16_t*)ec->A : nullptr;
     a.B = ec ? (const uint16_t*)ec->B : nullptr;
-    a.u = u;
+    a.wg = ec ? (const uint16_t*)ec->w_g : nullptr;
+    a.b_g = ec ? ec->b_g : 0.0f;
     a.rank = rank;
-    a.y = y;
     a.y_fp32 = (y_dtype == SPEAR_FP32);
-    a.M = M;
     a.N = N;
     a.K = K;
-    a.k_slice = K / p.split_k;
-    a.part = p.split_k > 1 ? (float*)(ws + L.part_off) : nullptr;
-    a.tickets = gemm_tickets;
-    cudaError_t e = launch_splitk(a, nb_for_tile_m(p.tile_m), p.tile_n / 16, p.split_k, s, ec != nullptr);
-    return e == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
+    a.k_slice = k_slice_for(K, p.split_k);
+    a.split = p.split_k;
+    a.ec_jr = ec_jr_for(rank, p.split_k);
+    a.ec_splits = rank > 0 ? ec_splits_for(K) : 0;
+    a.row_tiles = (int)(N / p.tile_n);
+    a.tacc = (long long*)(ws + CTRL_BYTES);
+    a.err = ctrl;
+    a.arrivals = ctrl + CTRL_HEADER_WORDS;
+    a.consumed = a.arrivals + CHUNKS_MAX;
+    a.consumed1 = a.consumed + CHUNKS_MAX;
+    const size_t ysz = y_dtype == SPEAR_FP32 ? 4 : 2;
+    // Launches of at most LAUNCH_TOKENS_MAX tokens, in token order on one stream.
+    for (int64_t m0 = 0; m0 < M; m0 += LAUNCH_TOKENS_MAX) {
+        const int64_t ml = (M - m0) < LAUNCH_TOKENS_MAX ? (M - m0) : LAUNCH_TOKENS_MAX;
+        a.x = (const uint16_t*)x + m0 * K;
+        a.y = (unsigned char*)y + (size_t)m0 * N * ysz;
+        a.M = ml;
+        a.mchunks = (int)((ml + p.tile_m - 1) / p.tile_m);
+        const int e = a.ec_splits * a.mchunks;
+        a.ec_ctas = (e + p.split_k - 1) / p.split_k * p.split_k;
+        if (launch_decode(a, nb, g, wpw_for(a.k_slice), s) != cudaSuccess) return SPEAR_ERR_CUDA;
+    }
+    return SPEAR_OK;
 }
 
 spear_status spear_get_device_status(void* workspace, int clear, void* stream) {

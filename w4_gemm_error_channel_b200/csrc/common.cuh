@@ -81,7 +81,7 @@ SPEAR_DEVI void mma_bf16_16816(float c[4], const uint32_t a[4], uint32_t b0, uin
 SPEAR_DEVI uint4 ldg_stream_u4(const void* p) {
     // Weight stream: read once, keep it out of L1.
     uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+    asm volatile("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
 }

@@ -8,40 +8,52 @@
 
 namespace spear {
 
-// Workspace control block: the first CTRL_BYTES of every workspace.  Must start zeroed; every
-// call leaves the tickets zeroed again.  Layout: [0] device error word, then ticket arrays.
+// Zeroed part of every workspace: it must start zeroed and every call leaves it zeroed again
+// (unless a bounded wait timed out).
+//   control block, CTRL_BYTES, in 32-bit words:
+//     [0]                     device error word (bit 0: an arrival wait gave up; bit 1: an EC
+//                             partial sum was outside the fixed-point range)
+//     [64, +CHUNKS)           EC arrival counters, one per token chunk of a launch
+//     [.., +CHUNKS)           consumer counters (level 2: finished groups), one per token chunk
+//     [.., +CHUNKS*GROUPS)    consumer counters (level 1: CTAs of a group of 64 GEMM CTAs)
+//   EC accumulators, TACC_BYTES: int64 [tokens of a launch][r + 1] (t, then the gate
+//   pre-activation), fixed point with 32 fraction bits.
 constexpr size_t CTRL_BYTES = 128 * 1024;
-constexpr size_t CTRL_HEADER_BYTES = 256;
-constexpr size_t EC_TICKETS_MAX = 4096;                          // token chunks of 16 -> M <= 65536
-constexpr size_t GEMM_TICKETS_MAX = (CTRL_BYTES - CTRL_HEADER_BYTES) / 4 - EC_TICKETS_MAX;
+constexpr size_t CTRL_HEADER_WORDS = 64;
+constexpr size_t CHUNKS_MAX = 32;                          // token chunks per launch (>= 8 tokens each)
+constexpr int CONSUMER_GROUP = 64;                         // GEMM CTAs per level-1 consumer counter
+constexpr size_t GROUPS_MAX = 256;                         // level-1 counters per token chunk
+constexpr size_t TACC_BYTES = 1024 * 1024;
+constexpr size_t ZEROED_BYTES = CTRL_BYTES + TACC_BYTES;
+constexpr int64_t LAUNCH_TOKENS_MAX = 256;                 // tokens per decode launch
 constexpr int64_t M_MAX = 65536;
+static_assert(CTRL_HEADER_WORDS + 2 * CHUNKS_MAX + CHUNKS_MAX * GROUPS_MAX <= CTRL_BYTES / 4, "control block");
 
-struct EcPrepassArgs {
-    const uint16_t* x;      // bf16 [M, K]
-    const uint16_t* A;      // bf16 [K, r]
-    const uint16_t* wg;     // bf16 [K]
-    float b_g;
-    int64_t M, K;
-    int rank;
-    int64_t k_per_cta;
-    float* ec_part;         // [S_ec][M][r + 1]
-    float* u;               // [M][r]   u = g * t
-    unsigned* tickets;      // [ceil(M / 16)]
-};
-
-struct SplitKArgs {
+struct DecodeArgs {
     const uint16_t* x;      // bf16 [M, K]
     const uint8_t* packed;  // [N, K/2]
     const __half* scale;    // [N]
     const __half* zero;     // [N]
-    const uint16_t* B;      // bf16 [r, N] (unused when u == nullptr)
-    const float* u;         // [M][r] or nullptr (no EC)
+    const uint16_t* A;      // bf16 [K, r]   (EC; rank == 0 means no EC)
+    const uint16_t* B;      // bf16 [r, N]
+    const uint16_t* wg;     // bf16 [K]
+    float b_g;
     int rank;
     void* y;
     int y_fp32;
-    int64_t M, N, K, k_slice;
-    float* part;            // [S][M][N] when S > 1
-    unsigned* tickets;      // [(N / RT) * ceil(M / TM)]
+    int64_t M, N, K;
+    int64_t k_slice;        // GEMM K slice per CTA, a multiple of 64
+    int split;              // S: GEMM K slices = thread-block cluster size (1, 2, 4 or 8)
+    int ec_jr;              // EC columns added per K slice (multiple of 4)
+    int ec_splits;          // EC CTAs per token chunk (128 rows of A each)
+    int ec_ctas;            // EC CTAs in the grid (ec_splits * mchunks, padded to whole clusters)
+    int row_tiles;          // N / (16 G)
+    int mchunks;            // ceil(M / (8 NB))
+    long long* tacc;        // [M][r + 1] EC accumulators (zeroed part of the workspace)
+    unsigned* err;          // error word
+    unsigned* arrivals;     // [mchunks]
+    unsigned* consumed;     // [mchunks] level-2 consumer counters
+    unsigned* consumed1;    // [mchunks][GROUPS_MAX] level-1 consumer counters
 };
 
 cudaError_t launch_pack_w4(const void* W, bool w_is_bf16, int64_t N, int64_t K, void* packed, void* scale,
@@ -49,15 +61,10 @@ cudaError_t launch_pack_w4(const void* W, bool w_is_bf16, int64_t N, int64_t K, 
 cudaError_t launch_unpack_w4(const void* packed, const void* zero, int64_t N, int64_t K, void* q_out,
                              void* qz_out, cudaStream_t stream);
 
-int64_t ec_prepass_token_chunks(int64_t M);
-int64_t ec_prepass_k_per_cta(int64_t M, int64_t K, int num_sms);
-int64_t ec_prepass_splits(int64_t K, int64_t k_per_cta);
-size_t ec_prepass_smem_bytes(int rank);
-size_t ec_prepass_max_smem_bytes();
-const void* ec_prepass_kernel_ptr();
-cudaError_t launch_ec_prepass(const EcPrepassArgs& a, cudaStream_t stream);
-
-// nb in {1,2,4} (tokens per CTA = 8*nb), g in {1,2,4,8} (rows per CTA = 16*g; g=8 needs nb<=2).
-cudaError_t launch_splitk(const SplitKArgs& a, int nb, int g, int split, cudaStream_t stream, bool pdl);
+// nb: tokens per CTA = 8*nb (1, 2, 4); g: weight rows per CTA = 16*g; wpw: 128-wide K windows per
+// warp (K slice of a CTA <= 512*wpw).  decode_config_supported() lists the compiled combinations.
+bool decode_config_supported(int nb, int g, int wpw);
+size_t decode_dyn_smem_bytes(int nb, int g, int ec_jr, int rank);
+cudaError_t launch_decode(const DecodeArgs& a, int nb, int g, int wpw, cudaStream_t stream);
 
 }  // namespace spear
