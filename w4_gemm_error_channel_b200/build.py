@@ -29,6 +29,7 @@ def sources():
 
 def _newest_input():
     files = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
+        glob.glob(os.path.join(CSRC, "*.inc")) + \
         [os.path.join(INCLUDE, "spear.h"), os.path.abspath(__file__)]
     return max(os.path.getmtime(f) for f in files)
 

@@ -2,6 +2,7 @@
 // and kernel dispatch.  Host code only; the kernels live in pack.cu and decode.cu.
 #include <math.h>
 #include <cmath>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -57,7 +58,37 @@ int ec_splits_for(int64_t K) { return (int)((K + 63) / 64); }     // 64 rows of 
 // front; the S K slices of a row tile form a cluster (S in {1, 2, 4, 8}).  The cost model prefers
 // tilings that spread the weight bytes evenly over all SMs (many small CTAs stream best), then
 // the least re-reading of activations from L2, then fewer slices.
-spear_status plan_decode(int64_t M, int64_t N, int64_t K, int sms, spear_plan* p) {
+// Measured plans (plans/gen_table.py): the fastest tiling per swept shape on one B200.
+struct MeasuredPlan {
+    int64_t M, N, K;
+    int has_ec, tile_n, split_k;
+    double us;
+};
+const MeasuredPlan kMeasured[] = {
+#include "plan_table.inc"
+};
+
+bool lookup_measured(int64_t M, int64_t N, int64_t K, int has_ec, spear_plan* p) {
+    const int nb = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
+    const MeasuredPlan* best = nullptr;
+    for (const MeasuredPlan& e : kMeasured) {
+        const int enb = e.M <= 8 ? 1 : (e.M <= 16 ? 2 : 4);
+        if (e.N != N || e.K != K || e.has_ec != has_ec || enb != nb) continue;
+        // Same token-tile size; prefer the measured batch closest to M.
+        if (!best || std::llabs(e.M - M) < std::llabs(best->M - M)) best = &e;
+    }
+    if (!best) return false;
+    p->kernel_id = SPEAR_KERNEL_SPLITK;
+    p->tile_n = best->tile_n;
+    p->split_k = best->split_k;
+    p->tile_m = 8 * nb;
+    p->flags = 0;
+    p->reserved = 0;
+    return true;
+}
+
+spear_status plan_decode(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spear_plan* p) {
+    if (lookup_measured(M, N, K, rank > 0 ? 1 : 0, p)) return SPEAR_OK;
     const int nb = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
     const int64_t tm = 8 * nb;
     const int64_t ml = M < LAUNCH_TOKENS_MAX ? M : LAUNCH_TOKENS_MAX;
@@ -161,7 +192,7 @@ spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int 
     if (st != SPEAR_OK) return st;
     const int sms = device_sms(device);
     spear_plan p = {};
-    st = plan_decode(M > 0 ? M : 1, N, K, sms, &p);
+    st = plan_decode(M > 0 ? M : 1, N, K, rank, sms, &p);
     if (st != SPEAR_OK) return st;
     p.workspace_bytes = workspace_bytes_for();
     *out = p;
@@ -192,7 +223,7 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
     if (plan) {
         p = *plan;
     } else {
-        st = plan_decode(M, N, K, sms, &p);
+        st = plan_decode(M, N, K, rank, sms, &p);
         if (st != SPEAR_OK) return st;
     }
     st = validate_plan(p, M, N, K);
