@@ -1,0 +1,68 @@
+"""The tcgen05 (TMEM) prefill kernel against the CPU oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synthetic import config_layers, make_layer
+from gpu_helpers import check_close, host_f64, to_dev, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import w4_gemm_error_channel_b200 as spear
+else:
+    spear = None
+
+
+def tc_plan(M, N, K, tile_m):
+    p = spear.spear_gemm_plan(M, N, K, 0)
+    p.kernel_id = spear.SPEAR_KERNEL_TC05
+    p.tile_n, p.split_k, p.tile_m = 128, 1, tile_m
+    return p
+
+
+def run(L, M, tile_m, y_dtype=torch.bfloat16, rows=None):
+    W = to_dev(L.W)
+    packed, scale, zero = spear.spear_pack_w4(W)
+    x = to_dev_bf16(L.x(M))
+    ws = spear.alloc_workspace(spear.spear_gemm_plan(M, L.N, L.K, 0).workspace_bytes)
+    y = spear.spear_w4ec_gemm(x, packed, scale, zero, None, y_dtype=y_dtype, plan=tc_plan(M, L.N, L.K, tile_m),
+                              workspace=ws)
+    torch.cuda.synchronize()
+    assert spear.spear_get_device_status(ws) == 0
+    p, s, z = oracle.pack_w4(L.W)
+    xs = L.x(M) if rows is None else L.x(M)[rows]
+    ref = oracle.w4ec_gemm(xs, p, s, z)
+    got = host_f64(y) if rows is None else host_f64(y)[rows]
+    return got, ref
+
+
+@pytest.mark.parametrize("tile_m", [128, 256])
+@pytest.mark.parametrize("M", [1, 77, 128, 129, 300, 512])
+def test_tc05_small(M, tile_m):
+    L = make_layer("tc", 5 + M, M, 384, 448, 0, outlier_frac=0.02, outlier_scale=10.0)
+    got, ref = run(L, M, tile_m)
+    check_close(got, ref, True, f"tc05 M={M} tile_m={tile_m}")
+
+
+def test_tc05_fp32_output():
+    L = make_layer("tc", 9, 200, 256, 1024, 0)
+    got, ref = run(L, 200, 128, y_dtype=torch.float32)
+    check_close(got, ref, False, "tc05 fp32")
+
+
+@pytest.mark.parametrize("tile_m", [128, 256])
+def test_tc05_prefill_shape_sampled(tile_m):
+    L = config_layers(3)[0]
+    rows = np.array([0, 1, 255, 256, 1031, 2047])
+    got, ref = run(L, 2048, tile_m, rows=rows)
+    check_close(got, ref, True, f"tc05 prefill tile_m={tile_m}")
+
+
+@pytest.mark.parametrize("li", [0, 1, 2, 3])
+def test_tc05_sweep_layer_without_ec(li):
+    L = config_layers(4, M=4096, layers=(2,))[li]     # layer 2 carries no compensator
+    rows = np.array([0, 100, 2049, 4095])
+    got, ref = run(L, 4096, 256, rows=rows)
+    check_close(got, ref, True, f"tc05 sweep L2.{li}")

@@ -128,8 +128,27 @@ spear_status plan_decode(int64_t M, int64_t N, int64_t K, int32_t rank, int sms,
     return SPEAR_OK;
 }
 
-spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K) {
+// Prefill (tcgen05) plan: 128 weight rows x tile_m tokens per CTA, no K split.
+spear_status plan_tc05(int64_t M, spear_plan* p) {
+    p->kernel_id = SPEAR_KERNEL_TC05;
+    p->tile_n = 128;
+    p->split_k = 1;
+    p->tile_m = M >= 2048 ? 256 : 128;
+    p->flags = 0;
+    p->reserved = 0;
+    return SPEAR_OK;
+}
+
+// Token count from which the tensor-core kernel replaces the weight-streaming kernel.
+constexpr int64_t TC05_MIN_M = 128;
+
+spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K, int32_t rank) {
     (void)M;
+    if (p.kernel_id == SPEAR_KERNEL_TC05) {
+        if (rank > 0) return SPEAR_ERR_INVALID_ARG;          // the compensator runs on the other kernel
+        if (p.tile_n != 128 || p.split_k != 1 || !(p.tile_m == 128 || p.tile_m == 256)) return SPEAR_ERR_INVALID_ARG;
+        return SPEAR_OK;
+    }
     if (p.kernel_id != SPEAR_KERNEL_SPLITK) return SPEAR_ERR_INVALID_ARG;
     if (!(p.split_k == 1 || p.split_k == 2 || p.split_k == 4 || p.split_k == 8)) return SPEAR_ERR_INVALID_ARG;
     const int nb = nb_for_tile_m(p.tile_m);
@@ -192,7 +211,8 @@ spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int 
     if (st != SPEAR_OK) return st;
     const int sms = device_sms(device);
     spear_plan p = {};
-    st = plan_decode(M > 0 ? M : 1, N, K, rank, sms, &p);
+    if (rank == 0 && M >= TC05_MIN_M) st = plan_tc05(M, &p);
+    else st = plan_decode(M > 0 ? M : 1, N, K, rank, sms, &p);
     if (st != SPEAR_OK) return st;
     p.workspace_bytes = workspace_bytes_for();
     *out = p;
@@ -223,16 +243,31 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
     if (plan) {
         p = *plan;
     } else {
-        st = plan_decode(M, N, K, rank, sms, &p);
+        if (rank == 0 && M >= TC05_MIN_M) st = plan_tc05(M, &p);
+        else st = plan_decode(M, N, K, rank, sms, &p);
         if (st != SPEAR_OK) return st;
     }
-    st = validate_plan(p, M, N, K);
+    st = validate_plan(p, M, N, K, rank);
     if (st != SPEAR_OK) return st;
     if (workspace_bytes < workspace_bytes_for()) return SPEAR_ERR_WORKSPACE_TOO_SMALL;
 
     cudaStream_t s = (cudaStream_t)stream;
     unsigned char* ws = (unsigned char*)workspace;
     unsigned* ctrl = (unsigned*)ws;
+    if (p.kernel_id == SPEAR_KERNEL_TC05) {
+        TcArgs t;
+        t.x = (const uint16_t*)x;
+        t.packed = (const uint8_t*)packed;
+        t.scale = (const __half*)scale;
+        t.zero = (const __half*)zero;
+        t.y = y;
+        t.y_fp32 = (y_dtype == SPEAR_FP32);
+        t.M = M;
+        t.N = N;
+        t.K = K;
+        t.err = ctrl;
+        return launch_tc05(t, p.tile_m, s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
+    }
     const int nb = nb_for_tile_m(p.tile_m);
     const int g = p.tile_n / 16;
 

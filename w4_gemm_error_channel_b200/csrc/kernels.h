@@ -56,6 +56,21 @@ struct DecodeArgs {
     unsigned* consumed1;    // [mchunks][GROUPS_MAX] level-1 consumer counters
 };
 
+// Prefill (tcgen05) kernel arguments.
+struct TcArgs {
+    const uint16_t* x;      // bf16 [M, K]
+    const uint8_t* packed;  // [N, K/2]
+    const __half* scale;    // [N]
+    const __half* zero;     // [N]
+    void* y;
+    int y_fp32;
+    int64_t M, N, K;
+    unsigned* err;          // error word (bit 2: an mbarrier wait gave up)
+};
+
+// bn: tokens per tile (128 or 256).
+cudaError_t launch_tc05(const TcArgs& a, int bn, cudaStream_t stream);
+
 cudaError_t launch_pack_w4(const void* W, bool w_is_bf16, int64_t N, int64_t K, void* packed, void* scale,
                            void* zero, cudaStream_t stream);
 cudaError_t launch_unpack_w4(const void* packed, const void* zero, int64_t N, int64_t K, void* q_out,

@@ -1,0 +1,329 @@
+// tc05.cu -- the prefill kernel: TMA + tcgen05 (TMEM accumulators) W4 GEMM for sm_100a.
+//
+// SPEAR (Post-Quantization Error-Adaptive Recovery), technical summary section 2.2A: prefill is
+// compute-bound, so the low-bit GEMM must run on the tensor cores.  There is no tcgen05 kind that
+// multiplies int4 by bf16 without changing x, so the int4 codes are turned into the exact bf16
+// integers (q - z) in shared memory and the MMA is kind::f16 (bf16 x bf16 -> fp32 in TMEM).  The
+// per-channel scale s[n] factors out of the K sum and is applied in the epilogue:
+//
+//   D[n, m] = sum_k (q[n,k] - z[n]) x[m,k]        (tcgen05.mma, fp32 accumulator in TMEM)
+//   y[m, n] = s[n] D[n, m] (+ the EC term)         (epilogue: tcgen05.ld -> registers -> y)
+//
+// One CTA computes a 128 (weight rows) x BN (tokens) tile with 6 warps:
+//   warp 0      TMA producer: per 64-wide K stage, the bf16 x tile (128-byte swizzle) and the
+//               packed int4 tile (128 rows x 32 bytes) into a STAGES-deep shared-memory ring;
+//   warp 1      allocates the TMEM accumulator and issues tcgen05.mma (one thread), committing
+//               each stage back to the producer through an mbarrier;
+//   warps 2-5   convert each packed tile to bf16 (q - z) in the canonical K-major 128-byte-swizzle
+//               layout the MMA reads (one weight row per thread), then run the epilogue.
+// Every mbarrier wait is bounded: on timeout the kernel records an error bit and stops.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace spear {
+
+constexpr int TC_THREADS = 192;
+constexpr int TC_BM = 128;               // weight rows per tile (MMA M)
+constexpr int TC_BK = 64;                // K codes per stage
+constexpr uint32_t WAIT_LIMIT = 1u << 24;
+
+// ---------------------------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------------------------
+SPEAR_DEVI uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+SPEAR_DEVI void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+SPEAR_DEVI void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+SPEAR_DEVI void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Bounded wait for the phase with the given parity.  Returns false after WAIT_LIMIT polls.
+SPEAR_DEVI bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_u32(bar);
+    for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
+        uint32_t done;
+        asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                     : "=r"(done) : "r"(a), "r"(parity) : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+SPEAR_DEVI void tma_load_2d(void* dst, const CUtensorMap* map, int32_t c0, int32_t c1, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar)) : "memory");
+}
+
+SPEAR_DEVI void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+SPEAR_DEVI void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+SPEAR_DEVI void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 bytes apart.
+SPEAR_DEVI uint64_t smem_desc_k_sw128(const void* base) {
+    const uint64_t addr = smem_u32(base);
+    uint64_t d = 0;
+    d |= (addr >> 4) & 0x3FFFull;            // start address (16-byte units)
+    d |= 1ull << 16;                         // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;        // stride byte offset: 8 rows x 128 bytes
+    d |= 1ull << 46;                         // descriptor version (sm_100)
+    d |= 2ull << 61;                         // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: kind::f16 with bf16 A and B (both K-major), fp32 accumulator.
+constexpr uint32_t idesc_bf16_f32(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+SPEAR_DEVI void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+SPEAR_DEVI void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+
+SPEAR_DEVI void tmem_ld16(uint32_t taddr, float v[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------------------------
+template <int BN, int STAGES>
+struct TcSmem {
+    static constexpr int X_BYTES = BN * TC_BK * 2;        // bf16 x tile, 128-byte swizzle
+    static constexpr int A_BYTES = TC_BM * TC_BK * 2;     // converted bf16 weight tile
+    static constexpr int P_BYTES = TC_BM * TC_BK / 2;     // packed int4 tile
+    static constexpr int X_OFF = 0;
+    static constexpr int A_OFF = X_OFF + STAGES * X_BYTES;
+    static constexpr int P_OFF = A_OFF + STAGES * A_BYTES;
+    static constexpr int BAR_OFF = P_OFF + STAGES * P_BYTES;
+    static constexpr int TOTAL = BAR_OFF + 3 * STAGES * 8 + 8 + 16 + 1024;   // + alignment slack
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+               TcArgs a) {
+    using L = TcSmem<BN, STAGES>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);       // TMA landed
+    uint64_t* cvt = full + STAGES;                                         // converted tile ready
+    uint64_t* empty = cvt + STAGES;                                        // MMA done with the stage
+    uint64_t* acc_full = empty + STAGES;                                   // accumulator complete
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    __shared__ unsigned s_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n0 = (int64_t)blockIdx.x * TC_BM;
+    const int64_t m0 = (int64_t)blockIdx.y * BN;
+    const int ksteps = (int)(a.K / TC_BK);
+
+    if (threadIdx.x == 0) {
+        s_abort = 0u;
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&cvt[s], 128);        // every converter thread arrives
+            mbar_init(&empty[s], 1);        // tcgen05.commit
+        }
+        mbar_init(acc_full, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        // TMEM accumulator: 128 lanes x BN fp32 columns.
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"((uint32_t)BN) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            // The x tile may be written by the previous kernel in the stream.
+            pdl_wait_primary();
+            for (int kt = 0; kt < ksteps; ++kt) {
+                const int s = kt % STAGES;
+                if (kt >= STAGES && !mbar_wait(&empty[s], ((kt / STAGES) - 1) & 1)) {
+                    atomicOr(a.err, 4u); s_abort = 1u; break;
+                }
+                mbar_arrive_expect_tx(&full[s], L::X_BYTES + L::P_BYTES);
+                tma_load_2d(smem + L::X_OFF + s * L::X_BYTES, &tmap_x, kt * TC_BK, (int32_t)m0, &full[s]);
+                tma_load_2d(smem + L::P_OFF + s * L::P_BYTES, &tmap_w, kt * (TC_BK / 2), (int32_t)n0, &full[s]);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, BN);
+            for (int kt = 0; kt < ksteps; ++kt) {
+                const int s = kt % STAGES;
+                if (!mbar_wait(&cvt[s], (kt / STAGES) & 1)) { atomicOr(a.err, 4u); s_abort = 1u; break; }
+                tc_fence_after();
+                const uint64_t ad = smem_desc_k_sw128(smem + L::A_OFF + s * L::A_BYTES);
+                const uint64_t bd = smem_desc_k_sw128(smem + L::X_OFF + s * L::X_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < TC_BK / 16; ++kk)   // 16 bf16 = 32 bytes = 2 descriptor units
+                    mma_bf16_ss(tmem_d, ad + 2 * kk, bd + 2 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&empty[s]);
+            }
+            mma_commit(acc_full);
+        }
+    } else {
+        // ---------------- converters, then epilogue ----------------
+        // Weight row of this thread: warp w may only read TMEM lanes 32*(w % 4) .. +31, and the
+        // accumulator row n lives in lane n, so warps 2, 3, 4, 5 take rows 64, 96, 0, 32 (+lane).
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t z = (uint32_t)__half2float(a.zero[n0 + row]);
+        const uint32_t zb = zero_bias_bf16x2(z);
+        for (int kt = 0; kt < ksteps; ++kt) {
+            const int s = kt % STAGES;
+            if (!mbar_wait(&full[s], (kt / STAGES) & 1)) { atomicOr(a.err, 4u); s_abort = 1u; break; }
+            const uint4* prow = reinterpret_cast<const uint4*>(smem + L::P_OFF + s * L::P_BYTES + row * 32);
+            unsigned char* arow = smem + L::A_OFF + s * L::A_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 w = prow[h];
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {              // 8 codes -> one 16-byte chunk
+                    uint32_t o[4];
+                    cvt_w4_pairs_natural(ws[q], zb, o);
+                    const int c = h * 4 + q;               // logical 16-byte chunk (k = 8c .. 8c+7)
+                    *reinterpret_cast<uint4*>(arow + ((c ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+            fence_proxy_async_smem();                      // generic-proxy writes -> tensor core
+            mbar_arrive(&cvt[s]);
+        }
+
+        // Epilogue: y[m, n0 + row] = s[n] * D[row, m].
+        const bool ok = mbar_wait(acc_full, 0);
+        if (!ok) { atomicOr(a.err, 4u); s_abort = 1u; }
+        tc_fence_after();
+        const float sc = __half2float(a.scale[n0 + row]);
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const int64_t n = n0 + row;
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+            float v[16];
+            tmem_ld16(tmem_d + lane_base + (uint32_t)c0, v);
+            if (!ok) continue;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int64_t m = m0 + c0 + i;
+                if (m < a.M) {
+                    const float yv = sc * v[i];
+                    if (a.y_fp32)
+                        reinterpret_cast<float*>(a.y)[m * a.N + n] = yv;
+                    else
+                        reinterpret_cast<__nv_bfloat16*>(a.y)[m * a.N + n] = __float2bfloat16_rn(yv);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    pdl_launch_dependents();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"((uint32_t)BN) : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D tensor map over a row-major [rows][cols] array of `elem` bytes per element.
+static bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem, uint64_t cols,
+                        uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * (uint64_t)elem};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES>
+static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
+    using L = TcSmem<BN, STAGES>;
+    CUtensorMap mx, mw;
+    if (!make_map_2d(&mx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.K, (uint64_t)a.M, TC_BK, BN,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!make_map_2d(&mw, a.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(a.K / 2), (uint64_t)a.N, TC_BK / 2,
+                     TC_BM, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    static bool opted[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !opted[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(w4_tc05_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             L::TOTAL);
+        if (e != cudaSuccess) return e;
+        opted[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.N / TC_BM), (unsigned)((a.M + BN - 1) / BN));
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = L::TOTAL;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, w4_tc05_kernel<BN, STAGES>, mx, mw, a);
+}
+
+cudaError_t launch_tc05(const TcArgs& a, int bn, cudaStream_t stream) {
+    if (bn == 128) return launch_tc_t<128, 4>(a, stream);
+    if (bn == 256) return launch_tc_t<256, 3>(a, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace spear
