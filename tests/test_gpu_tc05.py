@@ -66,3 +66,59 @@ def test_tc05_sweep_layer_without_ec(li):
     rows = np.array([0, 100, 2049, 4095])
     got, ref = run(L, 4096, 256, rows=rows)
     check_close(got, ref, True, f"tc05 sweep L2.{li}")
+
+
+def run_ec(L, M, tile_m, rows=None, b_g=None, y_dtype=torch.bfloat16):
+    W = to_dev(L.W)
+    packed, scale, zero = spear.spear_pack_w4(W)
+    x = to_dev_bf16(L.x(M))
+    bg = L.b_g if b_g is None else b_g
+    ec = spear.EC(to_dev_bf16(L.A_bits), to_dev_bf16(L.B_bits), to_dev_bf16(L.wg_bits), bg)
+    plan = spear.spear_gemm_plan(M, L.N, L.K, L.rank)
+    plan.kernel_id, plan.tile_n, plan.split_k, plan.tile_m = spear.SPEAR_KERNEL_TC05, 128, 1, tile_m
+    ws = spear.alloc_workspace(plan.workspace_bytes + (M * L.rank * 2 + 256))
+    y = spear.spear_w4ec_gemm(x, packed, scale, zero, ec, y_dtype=y_dtype, plan=plan, workspace=ws)
+    torch.cuda.synchronize()
+    assert spear.spear_get_device_status(ws) == 0
+    p, s, z = oracle.pack_w4(L.W)
+    xs = L.x(M) if rows is None else L.x(M)[rows]
+    ref = oracle.w4ec_gemm(xs, p, s, z, L.A_bits, L.B_bits, L.wg_bits, bg)
+    got = host_f64(y) if rows is None else host_f64(y)[rows]
+    return got, ref, y, ws
+
+
+@pytest.mark.parametrize("tile_m", [128, 256])
+@pytest.mark.parametrize("r", [16, 32, 48, 64, 128])
+@pytest.mark.parametrize("M", [128, 300])
+def test_tc05_ec_small(M, r, tile_m):
+    L = make_layer("tcec", 11 + r + M, M, 256, 512, r, outlier_frac=0.02, outlier_scale=10.0, b_g=0.3)
+    got, ref, _, _ = run_ec(L, M, tile_m)
+    check_close(got, ref, True, f"tc05 EC M={M} r={r} tile_m={tile_m}")
+
+
+def test_tc05_ec_fp32_and_gate_off():
+    L = make_layer("tcec", 21, 200, 384, 640, 64, b_g=-1.0)
+    got, ref, _, _ = run_ec(L, 200, 128, y_dtype=torch.float32)
+    check_close(got, ref, False, "tc05 EC fp32")
+    # b_g = -inf: g = 0 exactly, so the compensated layer equals the plain one bit for bit.
+    _, _, y_off, _ = run_ec(L, 200, 128, b_g=float("-inf"))
+    plain, _ = run(L, 200, 128)
+    assert np.array_equal(host_f64(y_off), plain)
+
+
+@pytest.mark.parametrize("tile_m", [128, 256])
+def test_tc05_ec_prefill_sampled(tile_m):
+    L = config_layers(3)[0]
+    rows = np.array([0, 1, 255, 256, 1031, 2047])
+    got, ref, _, ws = run_ec(L, 2048, tile_m, rows=rows)
+    check_close(got, ref, True, f"tc05 EC prefill tile_m={tile_m}")
+    zeroed = ws[: (128 + 1024) * 1024].cpu()
+    assert int(zeroed.count_nonzero()) == 0, "EC flags not re-armed"
+
+
+@pytest.mark.parametrize("li", [0, 3])
+def test_tc05_ec_sweep_layer(li):
+    L = config_layers(4, M=4096, layers=(0,))[li]     # layer 0 carries a rank-32 compensator
+    rows = np.array([0, 100, 2049, 4095])
+    got, ref, _, _ = run_ec(L, 4096, 256, rows=rows)
+    check_close(got, ref, True, f"tc05 EC sweep L0.{li}")

@@ -48,9 +48,13 @@ int ec_jr_for(int32_t rank, int64_t S) {
     if (rank <= 0) return 0;
     return (int)(((rank + S - 1) / S + 3) / 4 * 4);
 }
-// Workspace: only the zeroed prefix (control block + EC accumulators); split-K partial sums meet
-// in distributed shared memory.
-size_t workspace_bytes_for() { return ZEROED_BYTES; }
+// Workspace: the zeroed prefix (control block + EC accumulators); split-K partial sums meet in
+// distributed shared memory.  The prefill kernel with a compensator also keeps u (bf16 [M][r]).
+size_t workspace_bytes_for(const spear_plan& p, int64_t M, int32_t rank) {
+    size_t b = ZEROED_BYTES;
+    if (p.kernel_id == SPEAR_KERNEL_TC05 && rank > 0) b += ((size_t)M * rank * 2 + 255) / 256 * 256;
+    return b;
+}
 
 int ec_splits_for(int64_t K) { return (int)((K + 63) / 64); }     // 64 rows of A per EC CTA
 
@@ -139,13 +143,17 @@ spear_status plan_tc05(int64_t M, spear_plan* p) {
     return SPEAR_OK;
 }
 
-// Token count from which the tensor-core kernel replaces the weight-streaming kernel.
+// Token count from which the tensor-core kernel replaces the weight-streaming kernel, and the
+// largest compensator rank it takes (one 128-row EC tile per token block).
 constexpr int64_t TC05_MIN_M = 128;
+constexpr int32_t TC05_MAX_RANK = 128;
+bool use_tc05(int64_t M, int32_t rank) { return M >= TC05_MIN_M && rank <= TC05_MAX_RANK; }
 
 spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K, int32_t rank) {
     (void)M;
     if (p.kernel_id == SPEAR_KERNEL_TC05) {
-        if (rank > 0) return SPEAR_ERR_INVALID_ARG;          // the compensator runs on the other kernel
+        if (rank > TC05_MAX_RANK) return SPEAR_ERR_INVALID_ARG;
+        if ((M + p.tile_m - 1) / p.tile_m > (int64_t)TC_BLOCKS_MAX) return SPEAR_ERR_INVALID_ARG;
         if (p.tile_n != 128 || p.split_k != 1 || !(p.tile_m == 128 || p.tile_m == 256)) return SPEAR_ERR_INVALID_ARG;
         return SPEAR_OK;
     }
@@ -211,10 +219,10 @@ spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int 
     if (st != SPEAR_OK) return st;
     const int sms = device_sms(device);
     spear_plan p = {};
-    if (rank == 0 && M >= TC05_MIN_M) st = plan_tc05(M, &p);
+    if (use_tc05(M, rank)) st = plan_tc05(M, &p);
     else st = plan_decode(M > 0 ? M : 1, N, K, rank, sms, &p);
     if (st != SPEAR_OK) return st;
-    p.workspace_bytes = workspace_bytes_for();
+    p.workspace_bytes = workspace_bytes_for(p, M, rank);
     *out = p;
     return SPEAR_OK;
 }
@@ -243,13 +251,13 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
     if (plan) {
         p = *plan;
     } else {
-        if (rank == 0 && M >= TC05_MIN_M) st = plan_tc05(M, &p);
+        if (use_tc05(M, rank)) st = plan_tc05(M, &p);
         else st = plan_decode(M, N, K, rank, sms, &p);
         if (st != SPEAR_OK) return st;
     }
     st = validate_plan(p, M, N, K, rank);
     if (st != SPEAR_OK) return st;
-    if (workspace_bytes < workspace_bytes_for()) return SPEAR_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace_bytes < workspace_bytes_for(p, M, rank)) return SPEAR_ERR_WORKSPACE_TOO_SMALL;
 
     cudaStream_t s = (cudaStream_t)stream;
     unsigned char* ws = (unsigned char*)workspace;
@@ -260,12 +268,20 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         t.packed = (const uint8_t*)packed;
         t.scale = (const __half*)scale;
         t.zero = (const __half*)zero;
+        t.A = ec ? (const uint16_t*)ec->A : nullptr;
+        t.B = ec ? (const uint16_t*)ec->B : nullptr;
+        t.wg = ec ? (const uint16_t*)ec->w_g : nullptr;
+        t.b_g = ec ? ec->b_g : 0.0f;
+        t.rank = rank;
+        t.u = rank > 0 ? (__nv_bfloat16*)(ws + ZEROED_BYTES) : nullptr;
         t.y = y;
         t.y_fp32 = (y_dtype == SPEAR_FP32);
         t.M = M;
         t.N = N;
         t.K = K;
         t.err = ctrl;
+        t.ec_ready = ctrl + TC_FLAGS_WORD;
+        t.ec_consumed = t.ec_ready + TC_BLOCKS_MAX;
         return launch_tc05(t, p.tile_m, s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
     }
     const int nb = nb_for_tile_m(p.tile_m);

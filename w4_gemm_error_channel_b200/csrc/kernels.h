@@ -16,6 +16,8 @@ namespace spear {
 //     [64, +CHUNKS)           EC arrival counters, one per token chunk of a launch
 //     [.., +CHUNKS)           consumer counters (level 2: finished groups), one per token chunk
 //     [.., +CHUNKS*GROUPS)    consumer counters (level 1: CTAs of a group of 64 GEMM CTAs)
+//     [.., +TC_BLOCKS)        prefill kernel: u-ready flags, one per token block
+//     [.., +TC_BLOCKS)        prefill kernel: flag consumer counters
 //   EC accumulators, TACC_BYTES: int64 [tokens of a launch][r + 1] (t, then the gate
 //   pre-activation), fixed point with 32 fraction bits.
 constexpr size_t CTRL_BYTES = 128 * 1024;
@@ -26,8 +28,10 @@ constexpr size_t GROUPS_MAX = 256;                         // level-1 counters p
 constexpr size_t TACC_BYTES = 1024 * 1024;
 constexpr size_t ZEROED_BYTES = CTRL_BYTES + TACC_BYTES;
 constexpr int64_t LAUNCH_TOKENS_MAX = 256;                 // tokens per decode launch
+constexpr size_t TC_BLOCKS_MAX = 512;                      // token blocks of the prefill kernel (M <= 65536)
 constexpr int64_t M_MAX = 65536;
-static_assert(CTRL_HEADER_WORDS + 2 * CHUNKS_MAX + CHUNKS_MAX * GROUPS_MAX <= CTRL_BYTES / 4, "control block");
+constexpr size_t TC_FLAGS_WORD = CTRL_HEADER_WORDS + 2 * CHUNKS_MAX + CHUNKS_MAX * GROUPS_MAX;
+static_assert(TC_FLAGS_WORD + 2 * TC_BLOCKS_MAX <= CTRL_BYTES / 4, "control block");
 
 struct DecodeArgs {
     const uint16_t* x;      // bf16 [M, K]
@@ -62,10 +66,18 @@ struct TcArgs {
     const uint8_t* packed;  // [N, K/2]
     const __half* scale;    // [N]
     const __half* zero;     // [N]
+    const uint16_t* A;      // bf16 [K, r]  (EC; rank == 0 means none)
+    const uint16_t* B;      // bf16 [r, N]
+    const uint16_t* wg;     // bf16 [K]
+    float b_g;
+    int rank;               // 0 or 16..128
+    __nv_bfloat16* u;       // [M][r] bf16 u = g t (workspace, written by the EC tiles)
     void* y;
     int y_fp32;
     int64_t M, N, K;
-    unsigned* err;          // error word (bit 2: an mbarrier wait gave up)
+    unsigned* err;          // error word (bit 2: an mbarrier wait gave up; bit 3: an EC-ready wait gave up)
+    unsigned* ec_ready;     // [token blocks] u of the block is ready
+    unsigned* ec_consumed;  // [token blocks] main tiles that have seen the flag
 };
 
 // bn: tokens per tile (128 or 256).

@@ -105,42 +105,76 @@ SPEAR_DEVI void tmem_ld16(uint32_t taddr, float v[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Shared-memory matrix descriptor: MN-major, 128-byte swizzle.  The MN extent is split in groups
+// of 64 elements `lbo_bytes` apart; K rows are 128 bytes apart, 8-row groups 1024 bytes apart.
+SPEAR_DEVI uint64_t smem_desc_mn_sw128(const void* base, uint32_t lbo_bytes) {
+    const uint64_t addr = smem_u32(base);
+    uint64_t d = 0;
+    d |= (addr >> 4) & 0x3FFFull;
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= 1ull << 46;
+    d |= 2ull << 61;
+    return d;
+}
+constexpr uint32_t IDESC_A_MN = 1u << 15;   // A operand MN-major
+
+SPEAR_DEVI unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+SPEAR_DEVI void named_bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }   // warps 2-5
+
 // ---------------------------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------------------------
 template <int BN, int STAGES>
 struct TcSmem {
-    static constexpr int X_BYTES = BN * TC_BK * 2;        // bf16 x tile, 128-byte swizzle
-    static constexpr int A_BYTES = TC_BM * TC_BK * 2;     // converted bf16 weight tile
+    static constexpr int X_BYTES = BN * TC_BK * 2;        // bf16 x tile (or u chunk), 128-byte swizzle
+    static constexpr int A_BYTES = TC_BM * TC_BK * 2;     // bf16 A-operand tile (converted W, A or B chunk)
     static constexpr int P_BYTES = TC_BM * TC_BK / 2;     // packed int4 tile
     static constexpr int X_OFF = 0;
     static constexpr int A_OFF = X_OFF + STAGES * X_BYTES;
     static constexpr int P_OFF = A_OFF + STAGES * A_BYTES;
-    static constexpr int BAR_OFF = P_OFF + STAGES * P_BYTES;
+    static constexpr int G_OFF = P_OFF + STAGES * P_BYTES;               // gate values, BN floats
+    static constexpr int BAR_OFF = G_OFF + BN * 4;
     static constexpr int TOTAL = BAR_OFF + 3 * STAGES * 8 + 8 + 16 + 1024;   // + alignment slack
 };
 
+// Tiles: the first `ec_tiles` blocks are EC tiles (one per token block; compute u), the rest are
+// main tiles (weight tile nb, token block mb), token-block major.
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-               TcArgs a) {
+               const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+               const __grid_constant__ CUtensorMap tmap_u, TcArgs a) {
     using L = TcSmem<BN, STAGES>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);       // TMA landed
-    uint64_t* cvt = full + STAGES;                                         // converted tile ready
+    uint64_t* cvt = full + STAGES;                                         // stage ready for the MMA
     uint64_t* empty = cvt + STAGES;                                        // MMA done with the stage
-    uint64_t* acc_full = empty + STAGES;                                   // accumulator complete
+    uint64_t* acc_full = empty + STAGES;                                   // accumulators complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
-    __shared__ unsigned s_abort;
+    float* s_gate = reinterpret_cast<float*>(smem + L::G_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n0 = (int64_t)blockIdx.x * TC_BM;
-    const int64_t m0 = (int64_t)blockIdx.y * BN;
+    const bool has_ec = a.rank > 0;
+    const int mblocks = (int)((a.M + BN - 1) / BN);
+    const int ec_tiles = has_ec ? mblocks : 0;
+    const bool is_ec = (int)blockIdx.x < ec_tiles;
+    const int t = is_ec ? (int)blockIdx.x : (int)blockIdx.x - ec_tiles;
+    const int ntiles = (int)(a.N / TC_BM);
+    const int mb = is_ec ? t : t / ntiles;
+    const int64_t n0 = is_ec ? 0 : (int64_t)(t % ntiles) * TC_BM;
+    const int64_t m0 = (int64_t)mb * BN;
     const int ksteps = (int)(a.K / TC_BK);
+    const int ec_chunks = (!is_ec && has_ec) ? (a.rank + 63) / 64 : 0;   // EC MMA steps of 64 columns
+    const int rboxes = (a.rank + 63) / 64;                                 // 64-wide boxes of A per stage
+    const uint32_t ncols = has_ec ? 2 * BN : BN;                           // D (and E) in TMEM
 
     if (threadIdx.x == 0) {
-        s_abort = 0u;
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&cvt[s], 128);        // every converter thread arrives
@@ -150,96 +184,199 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
-        // TMEM accumulator: 128 lanes x BN fp32 columns.
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(tmem_slot)), "r"((uint32_t)BN) : "memory");
+                     ::"r"(smem_u32(tmem_slot)), "r"(ncols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_d = *tmem_slot;
+    const uint32_t tmem_e = tmem_d + BN;
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
-            // The x tile may be written by the previous kernel in the stream.
-            pdl_wait_primary();
-            for (int kt = 0; kt < ksteps; ++kt) {
+            pdl_wait_primary();            // x may be written by the previous kernel in the stream
+            bool ok = true;
+            for (int kt = 0; kt < ksteps && ok; ++kt) {
                 const int s = kt % STAGES;
-                if (kt >= STAGES && !mbar_wait(&empty[s], ((kt / STAGES) - 1) & 1)) {
-                    atomicOr(a.err, 4u); s_abort = 1u; break;
+                if (kt >= STAGES && !mbar_wait(&empty[s], ((kt / STAGES) - 1) & 1)) { atomicOr(a.err, 4u); ok = false; break; }
+                unsigned char* xs = smem + L::X_OFF + s * L::X_BYTES;
+                unsigned char* as = smem + L::A_OFF + s * L::A_BYTES;
+                if (is_ec) {
+                    // A[k, j] for k in this stage, j in 64-wide boxes: MN-major A-operand tiles.
+                    mbar_arrive_expect_tx(&full[s], L::X_BYTES + rboxes * (TC_BK * 64 * 2));
+                    tma_load_2d(xs, &tmap_x, kt * TC_BK, (int32_t)m0, &full[s]);
+                    for (int bx = 0; bx < rboxes; ++bx)
+                        tma_load_2d(as + bx * (TC_BK * 64 * 2), &tmap_a, bx * 64, kt * TC_BK, &full[s]);
+                } else {
+                    mbar_arrive_expect_tx(&full[s], L::X_BYTES + L::P_BYTES);
+                    tma_load_2d(xs, &tmap_x, kt * TC_BK, (int32_t)m0, &full[s]);
+                    tma_load_2d(smem + L::P_OFF + s * L::P_BYTES, &tmap_w, kt * (TC_BK / 2), (int32_t)n0, &full[s]);
                 }
-                mbar_arrive_expect_tx(&full[s], L::X_BYTES + L::P_BYTES);
-                tma_load_2d(smem + L::X_OFF + s * L::X_BYTES, &tmap_x, kt * TC_BK, (int32_t)m0, &full[s]);
-                tma_load_2d(smem + L::P_OFF + s * L::P_BYTES, &tmap_w, kt * (TC_BK / 2), (int32_t)n0, &full[s]);
+            }
+            if (ok && ec_chunks > 0) {
+                // u of this token block is written by its EC tile: wait (bounded) for the flag.
+                unsigned it = 0;
+                while (ld_acquire_gpu(&a.ec_ready[mb]) == 0u) {
+                    if (++it > WAIT_LIMIT) { atomicOr(a.err, 8u); ok = false; break; }
+                    if (it > 64) __nanosleep(128);
+                }
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                for (int c = 0; c < ec_chunks && ok; ++c) {
+                    const int v = ksteps + c, s = v % STAGES;
+                    if (v >= STAGES && !mbar_wait(&empty[s], ((v / STAGES) - 1) & 1)) { atomicOr(a.err, 4u); ok = false; break; }
+                    unsigned char* xs = smem + L::X_OFF + s * L::X_BYTES;
+                    unsigned char* as = smem + L::A_OFF + s * L::A_BYTES;
+                    mbar_arrive_expect_tx(&full[s], L::X_BYTES + 2 * (64 * 64 * 2));
+                    tma_load_2d(xs, &tmap_u, c * 64, (int32_t)m0, &full[s]);                 // u[m, 64c ..]
+                    tma_load_2d(as, &tmap_b, (int32_t)n0, c * 64, &full[s]);                 // B[64c .., n0 .. +64]
+                    tma_load_2d(as + 64 * 64 * 2, &tmap_b, (int32_t)n0 + 64, c * 64, &full[s]);
+                }
+                // Every main tile of this token block has seen the flag: the last one re-arms it.
+                if (atomicAdd(&a.ec_consumed[mb], 1u) == (unsigned)ntiles - 1) {
+                    a.ec_consumed[mb] = 0u;
+                    a.ec_ready[mb] = 0u;
+                }
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, BN);
+            bool ok = true;
             for (int kt = 0; kt < ksteps; ++kt) {
                 const int s = kt % STAGES;
-                if (!mbar_wait(&cvt[s], (kt / STAGES) & 1)) { atomicOr(a.err, 4u); s_abort = 1u; break; }
+                if (!mbar_wait(&cvt[s], (kt / STAGES) & 1)) { atomicOr(a.err, 4u); ok = false; break; }
                 tc_fence_after();
-                const uint64_t ad = smem_desc_k_sw128(smem + L::A_OFF + s * L::A_BYTES);
+                const uint64_t bd = smem_desc_k_sw128(smem + L::X_OFF + s * L::X_BYTES);
+                if (is_ec) {
+                    const uint64_t ad = smem_desc_mn_sw128(smem + L::A_OFF + s * L::A_BYTES, TC_BK * 64 * 2);
+#pragma unroll
+                    for (int kk = 0; kk < TC_BK / 16; ++kk)   // 16 K rows = 2 groups of 1024 bytes
+                        mma_bf16_ss(tmem_d, ad + 128 * kk, bd + 2 * kk, idesc | IDESC_A_MN, (kt > 0 || kk > 0) ? 1u : 0u);
+                } else {
+                    const uint64_t ad = smem_desc_k_sw128(smem + L::A_OFF + s * L::A_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < TC_BK / 16; ++kk)   // 16 bf16 = 32 bytes = 2 descriptor units
+                        mma_bf16_ss(tmem_d, ad + 2 * kk, bd + 2 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&empty[s]);
+            }
+            for (int c = 0; c < ec_chunks && ok; ++c) {
+                // E[n, m] += sum_j B[j, n] u[m, j], 64 columns j per step (B slice MN-major).
+                const int v = ksteps + c, s = v % STAGES;
+                if (!mbar_wait(&cvt[s], (v / STAGES) & 1)) { atomicOr(a.err, 4u); ok = false; break; }
+                tc_fence_after();
+                const uint64_t ad = smem_desc_mn_sw128(smem + L::A_OFF + s * L::A_BYTES, 64 * 64 * 2);
                 const uint64_t bd = smem_desc_k_sw128(smem + L::X_OFF + s * L::X_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < TC_BK / 16; ++kk)   // 16 bf16 = 32 bytes = 2 descriptor units
-                    mma_bf16_ss(tmem_d, ad + 2 * kk, bd + 2 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tmem_e, ad + 128 * kk, bd + 2 * kk, idesc | IDESC_A_MN, (c > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&empty[s]);
             }
             mma_commit(acc_full);
         }
     } else {
-        // ---------------- converters, then epilogue ----------------
+        // ---------------- converters / gate, then epilogue ----------------
         // Weight row of this thread: warp w may only read TMEM lanes 32*(w % 4) .. +31, and the
         // accumulator row n lives in lane n, so warps 2, 3, 4, 5 take rows 64, 96, 0, 32 (+lane).
         const int row = (warp & 3) * 32 + lane;
-        const uint32_t z = (uint32_t)__half2float(a.zero[n0 + row]);
-        const uint32_t zb = zero_bias_bf16x2(z);
-        for (int kt = 0; kt < ksteps; ++kt) {
+        const uint32_t zb = is_ec ? 0u : zero_bias_bf16x2((uint32_t)__half2float(a.zero[n0 + row]));
+        constexpr int TPT = BN / 128;                      // gate: tokens per thread
+        float pg[TPT];
+#pragma unroll
+        for (int i = 0; i < TPT; ++i) pg[i] = 0.0f;
+        bool ok = true;
+        for (int kt = 0; kt < ksteps + ec_chunks; ++kt) {
             const int s = kt % STAGES;
-            if (!mbar_wait(&full[s], (kt / STAGES) & 1)) { atomicOr(a.err, 4u); s_abort = 1u; break; }
-            const uint4* prow = reinterpret_cast<const uint4*>(smem + L::P_OFF + s * L::P_BYTES + row * 32);
-            unsigned char* arow = smem + L::A_OFF + s * L::A_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+            if (!mbar_wait(&full[s], (kt / STAGES) & 1)) { atomicOr(a.err, 4u); ok = false; break; }
+            if (is_ec) {
+                // Gate pre-activation: x[m, k] w_g[k] over this stage, tokens row + 128 i.
+                const unsigned char* xs = smem + L::X_OFF + s * L::X_BYTES;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint4 w = prow[h];
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                for (int c = 0; c < 8; ++c) {
+                    float wv[8];
+                    const uint4 wr = ldg_u4(a.wg + (int64_t)kt * TC_BK + 8 * c);
+                    const uint32_t ww[4] = {wr.x, wr.y, wr.z, wr.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {              // 8 codes -> one 16-byte chunk
-                    uint32_t o[4];
-                    cvt_w4_pairs_natural(ws[q], zb, o);
-                    const int c = h * 4 + q;               // logical 16-byte chunk (k = 8c .. 8c+7)
-                    *reinterpret_cast<uint4*>(arow + ((c ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    for (int e = 0; e < 4; ++e) { wv[2 * e] = __uint_as_float(ww[e] << 16); wv[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u); }
+#pragma unroll
+                    for (int i = 0; i < TPT; ++i) {
+                        const int m = row + 128 * i;
+                        const uint4 xr = *reinterpret_cast<const uint4*>(xs + (m >> 3) * 1024 + (m & 7) * 128 + ((c ^ (m & 7)) << 4));
+                        const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            pg[i] = fmaf(__uint_as_float(xw[e] << 16), wv[2 * e], pg[i]);
+                            pg[i] = fmaf(__uint_as_float(xw[e] & 0xFFFF0000u), wv[2 * e + 1], pg[i]);
+                        }
+                    }
                 }
+            } else if (kt < ksteps) {
+                const uint4* prow = reinterpret_cast<const uint4*>(smem + L::P_OFF + s * L::P_BYTES + row * 32);
+                unsigned char* arow = smem + L::A_OFF + s * L::A_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint4 w = prow[h];
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {              // 8 codes -> one 16-byte chunk
+                        uint32_t o[4];
+                        cvt_w4_pairs_natural(ws[q], zb, o);
+                        const int c = h * 4 + q;               // logical 16-byte chunk (k = 8c .. 8c+7)
+                        *reinterpret_cast<uint4*>(arow + ((c ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                }
+                fence_proxy_async_smem();                      // generic-proxy writes -> tensor core
             }
-            fence_proxy_async_smem();                      // generic-proxy writes -> tensor core
             mbar_arrive(&cvt[s]);
         }
 
-        // Epilogue: y[m, n0 + row] = s[n] * D[row, m].
-        const bool ok = mbar_wait(acc_full, 0);
-        if (!ok) { atomicOr(a.err, 4u); s_abort = 1u; }
+        const bool acc_ok = ok && mbar_wait(acc_full, 0);
+        if (!acc_ok) atomicOr(a.err, 4u);
         tc_fence_after();
-        const float sc = __half2float(a.scale[n0 + row]);
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const int64_t n = n0 + row;
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-            float v[16];
-            tmem_ld16(tmem_d + lane_base + (uint32_t)c0, v);
-            if (!ok) continue;
+        if (is_ec) {
+            // g[m] = sigmoid(p[m] + b_g); u[m, j] = g[m] t[j, m] for j = row < r, as bf16.
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int64_t m = m0 + c0 + i;
-                if (m < a.M) {
-                    const float yv = sc * v[i];
-                    if (a.y_fp32)
-                        reinterpret_cast<float*>(a.y)[m * a.N + n] = yv;
-                    else
-                        reinterpret_cast<__nv_bfloat16*>(a.y)[m * a.N + n] = __float2bfloat16_rn(yv);
+            for (int i = 0; i < TPT; ++i) s_gate[row + 128 * i] = 1.0f / (1.0f + expf(-(pg[i] + a.b_g)));
+            named_bar_epi();
+            const int j = row;
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                float v[16];
+                tmem_ld16(tmem_d + lane_base + (uint32_t)c0, v);
+                if (!acc_ok || j >= a.rank) continue;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int64_t m = m0 + c0 + i;
+                    if (m < a.M) a.u[m * a.rank + j] = __float2bfloat16_rn(s_gate[c0 + i] * v[i]);
+                }
+            }
+            asm volatile("fence.proxy.async.global;" ::: "memory");   // u is read by other CTAs' TMA
+            __threadfence();
+            named_bar_epi();
+            if (row == 0 && acc_ok) asm volatile("st.release.gpu.global.u32 [%0], 1;" ::"l"(&a.ec_ready[mb]) : "memory");
+        } else {
+            // y[m, n] = s[n] D[n, m] (+ E[n, m]).
+            const float sc = __half2float(a.scale[n0 + row]);
+            const int64_t n = n0 + row;
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                float v[16], e[16];
+                tmem_ld16(tmem_d + lane_base + (uint32_t)c0, v);
+                if (has_ec) tmem_ld16(tmem_e + lane_base + (uint32_t)c0, e);
+                if (!acc_ok) continue;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int64_t m = m0 + c0 + i;
+                    if (m < a.M) {
+                        const float yv = has_ec ? fmaf(sc, v[i], e[i]) : sc * v[i];
+                        if (a.y_fp32)
+                            reinterpret_cast<float*>(a.y)[m * a.N + n] = yv;
+                        else
+                            reinterpret_cast<__nv_bfloat16*>(a.y)[m * a.N + n] = __float2bfloat16_rn(yv);
+                    }
                 }
             }
         }
@@ -250,7 +387,7 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     pdl_launch_dependents();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"((uint32_t)BN) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"(ncols) : "memory");
     }
 }
 
@@ -291,13 +428,26 @@ static bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
 template <int BN, int STAGES>
 static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
     using L = TcSmem<BN, STAGES>;
-    CUtensorMap mx, mw;
+    CUtensorMap mx, mw, ma, mb, mu;
     if (!make_map_2d(&mx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.K, (uint64_t)a.M, TC_BK, BN,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     if (!make_map_2d(&mw, a.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(a.K / 2), (uint64_t)a.N, TC_BK / 2,
                      TC_BM, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
+    const bool has_ec = a.rank > 0;
+    if (has_ec) {
+        // A [K, r] read as 64 (j) x 64 (k) boxes; B [r, N] as 64 (n) x 64 (j); u [M, r] as 64 (j) x BN (m).
+        if (!make_map_2d(&ma, a.A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.rank, (uint64_t)a.K, 64, TC_BK,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map_2d(&mb, a.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.N, (uint64_t)a.rank, 64, 64,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map_2d(&mu, a.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.rank, (uint64_t)a.M, 64, BN,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    } else {
+        ma = mx; mb = mx; mu = mx;      // unused
+    }
     static bool opted[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -307,8 +457,10 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         opted[dev] = true;
     }
+    const unsigned mblocks = (unsigned)((a.M + BN - 1) / BN);
+    const unsigned tiles = (unsigned)(a.N / TC_BM) * mblocks + (has_ec ? mblocks : 0u);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(a.N / TC_BM), (unsigned)((a.M + BN - 1) / BN));
+    cfg.gridDim = dim3(tiles);
     cfg.blockDim = dim3(TC_THREADS);
     cfg.dynamicSmemBytes = L::TOTAL;
     cfg.stream = stream;
@@ -317,7 +469,7 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, w4_tc05_kernel<BN, STAGES>, mx, mw, a);
+    return cudaLaunchKernelEx(&cfg, w4_tc05_kernel<BN, STAGES>, mx, mw, ma, mb, mu, a);
 }
 
 cudaError_t launch_tc05(const TcArgs& a, int bn, cudaStream_t stream) {
