@@ -12,11 +12,20 @@
 // One CTA computes a 128 (weight rows) x BN (tokens) tile with 6 warps:
 //   warp 0      TMA producer: per 64-wide K stage, the bf16 x tile (128-byte swizzle) and the
 //               packed int4 tile (128 rows x 32 bytes) into a STAGES-deep shared-memory ring;
-//   warp 1      allocates the TMEM accumulator and issues tcgen05.mma (one thread), committing
-//               each stage back to the producer through an mbarrier;
-//   warps 2-5   convert each packed tile to bf16 (q - z) in the canonical K-major 128-byte-swizzle
-//               layout the MMA reads (one weight row per thread), then run the epilogue.
-// Every mbarrier wait is bounded: on timeout the kernel records an error bit and stops.
+//   warp 1      allocates TMEM and issues tcgen05.mma (one thread), A operand from TMEM, B (x)
+//               from shared memory, committing each stage back to the producer;
+//   warps 2-5   convert each packed tile to bf16 (q - z) and store it to TMEM with tcgen05.st
+//               (one weight row = one TMEM lane per thread), then run the epilogue.
+// Keeping the converted weights out of shared memory leaves its bandwidth to the TMA stream and
+// the x operand.
+//
+// The compensator: the first ceil(M / 128) blocks are EC tiles.  Each computes, for 128 tokens,
+// t[j, m] = sum_k A[k, j] x[m, k] with tcgen05 (A read MN-major straight from its [K, r] layout by
+// TMA) and the gate pre-activation on its converter warps, then stores u = g t (bf16) and raises
+// its ready flag.  A main tile, after its K loop, waits (bounded) for the flags of its tokens, loads
+// the u tile and the B slice (MN-major, from [r, N]) by TMA and accumulates E[n, m] = sum_j
+// B[j, n] u[m, j] into TMEM; the epilogue writes y = s[n] D + E.
+// Every mbarrier and flag wait is bounded: on timeout the kernel records an error bit and stops.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -88,6 +97,23 @@ SPEAR_DEVI void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, u
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
+// A operand from TMEM (128 lanes = rows, 32-bit columns holding bf16 pairs k = 2c, 2c + 1).
+SPEAR_DEVI void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+SPEAR_DEVI void tmem_st32(uint32_t taddr, const uint32_t v[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+          "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+          "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
 SPEAR_DEVI void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                  ::"r"(smem_u32(bar)) : "memory");
@@ -132,23 +158,30 @@ SPEAR_DEVI void named_bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory");
 template <int BN, int STAGES>
 struct TcSmem {
     static constexpr int X_BYTES = BN * TC_BK * 2;        // bf16 x tile (or u chunk), 128-byte swizzle
-    static constexpr int A_BYTES = TC_BM * TC_BK * 2;     // bf16 A-operand tile (converted W, A or B chunk)
+    static constexpr int A_BYTES = TC_BM * TC_BK * 2;     // bf16 MN-major tile (A or B slice)
     static constexpr int P_BYTES = TC_BM * TC_BK / 2;     // packed int4 tile
     static constexpr int X_OFF = 0;
     static constexpr int A_OFF = X_OFF + STAGES * X_BYTES;
     static constexpr int P_OFF = A_OFF + STAGES * A_BYTES;
-    static constexpr int G_OFF = P_OFF + STAGES * P_BYTES;               // gate values, BN floats
-    static constexpr int BAR_OFF = G_OFF + BN * 4;
-    static constexpr int TOTAL = BAR_OFF + 3 * STAGES * 8 + 8 + 16 + 1024;   // + alignment slack
+    static constexpr int WG_OFF = P_OFF + STAGES * P_BYTES;              // w_g slice per stage (EC tiles)
+    static constexpr int G_OFF = WG_OFF + STAGES * TC_BK * 2;            // gate values, 128 floats
+    static constexpr int BAR_OFF = G_OFF + 128 * 4;
+    static constexpr int TOTAL = BAR_OFF + 3 * STAGES * 8 + 16 + 16 + 1024;   // + alignment slack
+    // TMEM columns: D [0, BN); converted weight stages [BN, BN + 32 STAGES); E [BN, 2 BN) reuses
+    // the stage columns once the main K loop has retired.
+    static constexpr int NEED = BN + (STAGES * 32 > BN ? STAGES * 32 : BN);
+    static constexpr uint32_t TMEM_COLS = NEED <= 32 ? 32 : NEED <= 64 ? 64 : NEED <= 128 ? 128 : NEED <= 256 ? 256 : 512;
 };
+constexpr int TC_EB = 128;               // tokens per EC tile
 
-// Tiles: the first `ec_tiles` blocks are EC tiles (one per token block; compute u), the rest are
-// main tiles (weight tile nb, token block mb), token-block major.
+// Tiles: the first `ec_tiles` blocks are EC tiles (one per 128 tokens; compute u), the rest are
+// main tiles (weight tile nb, token block mb of BN tokens), token-block major.
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-               const __grid_constant__ CUtensorMap tmap_u, TcArgs a) {
+               const __grid_constant__ CUtensorMap tmap_u, const __grid_constant__ CUtensorMap tmap_g,
+               const __grid_constant__ CUtensorMap tmap_x128, TcArgs a) {
     using L = TcSmem<BN, STAGES>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -156,23 +189,25 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     uint64_t* cvt = full + STAGES;                                         // stage ready for the MMA
     uint64_t* empty = cvt + STAGES;                                        // MMA done with the stage
     uint64_t* acc_full = empty + STAGES;                                   // accumulators complete
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    uint64_t* main_done = acc_full + 1;                                    // main K loop retired
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(main_done + 1);
     float* s_gate = reinterpret_cast<float*>(smem + L::G_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool has_ec = a.rank > 0;
-    const int mblocks = (int)((a.M + BN - 1) / BN);
-    const int ec_tiles = has_ec ? mblocks : 0;
+    const int eblocks = (int)((a.M + TC_EB - 1) / TC_EB);
+    const int ec_tiles = has_ec ? eblocks : 0;
     const bool is_ec = (int)blockIdx.x < ec_tiles;
     const int t = is_ec ? (int)blockIdx.x : (int)blockIdx.x - ec_tiles;
     const int ntiles = (int)(a.N / TC_BM);
-    const int mb = is_ec ? t : t / ntiles;
+    const int mb = is_ec ? t : t / ntiles;                                 // EC: 128-token block; main: BN block
     const int64_t n0 = is_ec ? 0 : (int64_t)(t % ntiles) * TC_BM;
-    const int64_t m0 = (int64_t)mb * BN;
+    const int64_t m0 = (int64_t)mb * (is_ec ? TC_EB : BN);
     const int ksteps = (int)(a.K / TC_BK);
     const int ec_chunks = (!is_ec && has_ec) ? (a.rank + 63) / 64 : 0;   // EC MMA steps of 64 columns
     const int rboxes = (a.rank + 63) / 64;                                 // 64-wide boxes of A per stage
-    const uint32_t ncols = has_ec ? 2 * BN : BN;                           // D (and E) in TMEM
+    const int e_lo = (int)(m0 / TC_EB);                                    // EC blocks this main tile needs
+    const int e_hi = min(eblocks, (int)((m0 + BN + TC_EB - 1) / TC_EB));
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -181,18 +216,20 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             mbar_init(&empty[s], 1);        // tcgen05.commit
         }
         mbar_init(acc_full, 1);
+        mbar_init(main_done, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(tmem_slot)), "r"(ncols) : "memory");
+                     ::"r"(smem_u32(tmem_slot)), "r"(L::TMEM_COLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_d = *tmem_slot;
-    const uint32_t tmem_e = tmem_d + BN;
+    const uint32_t tmem_a = tmem_d + BN;       // converted weight stages (main K loop)
+    const uint32_t tmem_e = tmem_d + BN;       // EC accumulator (after the main K loop)
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -203,13 +240,14 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 const int s = kt % STAGES;
                 if (kt >= STAGES && !mbar_wait(&empty[s], ((kt / STAGES) - 1) & 1)) { atomicOr(a.err, 4u); ok = false; break; }
                 unsigned char* xs = smem + L::X_OFF + s * L::X_BYTES;
-                unsigned char* as = smem + L::A_OFF + s * L::A_BYTES;
                 if (is_ec) {
-                    // A[k, j] for k in this stage, j in 64-wide boxes: MN-major A-operand tiles.
-                    mbar_arrive_expect_tx(&full[s], L::X_BYTES + rboxes * (TC_BK * 64 * 2));
-                    tma_load_2d(xs, &tmap_x, kt * TC_BK, (int32_t)m0, &full[s]);
+                    // x (128 tokens), A[k, j] in 64-wide MN-major boxes, and the w_g slice.
+                    unsigned char* as = smem + L::A_OFF + s * L::A_BYTES;
+                    mbar_arrive_expect_tx(&full[s], TC_EB * TC_BK * 2 + rboxes * (TC_BK * 64 * 2) + TC_BK * 2);
+                    tma_load_2d(xs, &tmap_x128, kt * TC_BK, (int32_t)m0, &full[s]);
                     for (int bx = 0; bx < rboxes; ++bx)
                         tma_load_2d(as + bx * (TC_BK * 64 * 2), &tmap_a, bx * 64, kt * TC_BK, &full[s]);
+                    tma_load_2d(smem + L::WG_OFF + s * TC_BK * 2, &tmap_g, kt * TC_BK, 0, &full[s]);
                 } else {
                     mbar_arrive_expect_tx(&full[s], L::X_BYTES + L::P_BYTES);
                     tma_load_2d(xs, &tmap_x, kt * TC_BK, (int32_t)m0, &full[s]);
@@ -217,11 +255,13 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 }
             }
             if (ok && ec_chunks > 0) {
-                // u of this token block is written by its EC tile: wait (bounded) for the flag.
-                unsigned it = 0;
-                while (ld_acquire_gpu(&a.ec_ready[mb]) == 0u) {
-                    if (++it > WAIT_LIMIT) { atomicOr(a.err, 8u); ok = false; break; }
-                    if (it > 64) __nanosleep(128);
+                // u of these tokens is written by their EC tiles: wait (bounded) for the flags.
+                for (int e = e_lo; e < e_hi && ok; ++e) {
+                    unsigned it = 0;
+                    while (ld_acquire_gpu(&a.ec_ready[e]) == 0u) {
+                        if (++it > WAIT_LIMIT) { atomicOr(a.err, 8u); ok = false; break; }
+                        if (it > 64) __nanosleep(128);
+                    }
                 }
                 asm volatile("fence.proxy.async.global;" ::: "memory");
                 for (int c = 0; c < ec_chunks && ok; ++c) {
@@ -234,17 +274,19 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                     tma_load_2d(as, &tmap_b, (int32_t)n0, c * 64, &full[s]);                 // B[64c .., n0 .. +64]
                     tma_load_2d(as + 64 * 64 * 2, &tmap_b, (int32_t)n0 + 64, c * 64, &full[s]);
                 }
-                // Every main tile of this token block has seen the flag: the last one re-arms it.
-                if (atomicAdd(&a.ec_consumed[mb], 1u) == (unsigned)ntiles - 1) {
-                    a.ec_consumed[mb] = 0u;
-                    a.ec_ready[mb] = 0u;
+                // Every main tile of these tokens has seen the flags: the last one re-arms each.
+                if (ok) {
+                    for (int e = e_lo; e < e_hi; ++e)
+                        if (atomicAdd(&a.ec_consumed[e], 1u) == (unsigned)ntiles - 1) {
+                            a.ec_consumed[e] = 0u;
+                            a.ec_ready[e] = 0u;
+                        }
                 }
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, BN);
             bool ok = true;
             for (int kt = 0; kt < ksteps; ++kt) {
                 const int s = kt % STAGES;
@@ -252,18 +294,26 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 tc_fence_after();
                 const uint64_t bd = smem_desc_k_sw128(smem + L::X_OFF + s * L::X_BYTES);
                 if (is_ec) {
+                    constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, TC_EB) | IDESC_A_MN;
                     const uint64_t ad = smem_desc_mn_sw128(smem + L::A_OFF + s * L::A_BYTES, TC_BK * 64 * 2);
 #pragma unroll
                     for (int kk = 0; kk < TC_BK / 16; ++kk)   // 16 K rows = 2 groups of 1024 bytes
-                        mma_bf16_ss(tmem_d, ad + 128 * kk, bd + 2 * kk, idesc | IDESC_A_MN, (kt > 0 || kk > 0) ? 1u : 0u);
+                        mma_bf16_ss(tmem_d, ad + 128 * kk, bd + 2 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
                 } else {
-                    const uint64_t ad = smem_desc_k_sw128(smem + L::A_OFF + s * L::A_BYTES);
+                    constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, BN);
 #pragma unroll
-                    for (int kk = 0; kk < TC_BK / 16; ++kk)   // 16 bf16 = 32 bytes = 2 descriptor units
-                        mma_bf16_ss(tmem_d, ad + 2 * kk, bd + 2 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < TC_BK / 16; ++kk)   // 16 bf16 = 8 TMEM columns = 2 descriptor units
+                        mma_bf16_ts(tmem_d, tmem_a + s * 32 + 8 * kk, bd + 2 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&empty[s]);
             }
+            if (ok && ec_chunks > 0) {
+                // The EC accumulator reuses the weight-stage columns: let the main loop retire first.
+                mma_commit(main_done);
+                if (!mbar_wait(main_done, 0)) { atomicOr(a.err, 4u); ok = false; }
+                tc_fence_after();
+            }
+            constexpr uint32_t idesc_ec = idesc_bf16_f32(TC_BM, BN) | IDESC_A_MN;
             for (int c = 0; c < ec_chunks && ok; ++c) {
                 // E[n, m] += sum_j B[j, n] u[m, j], 64 columns j per step (B slice MN-major).
                 const int v = ksteps + c, s = v % STAGES;
@@ -273,63 +323,54 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 const uint64_t bd = smem_desc_k_sw128(smem + L::X_OFF + s * L::X_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tmem_e, ad + 128 * kk, bd + 2 * kk, idesc | IDESC_A_MN, (c > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ss(tmem_e, ad + 128 * kk, bd + 2 * kk, idesc_ec, (c > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&empty[s]);
             }
             mma_commit(acc_full);
         }
     } else {
         // ---------------- converters / gate, then epilogue ----------------
-        // Weight row of this thread: warp w may only read TMEM lanes 32*(w % 4) .. +31, and the
-        // accumulator row n lives in lane n, so warps 2, 3, 4, 5 take rows 64, 96, 0, 32 (+lane).
+        // Weight row of this thread: warp w may only access TMEM lanes 32*(w % 4) .. +31, and the
+        // accumulator and weight-operand row n live in lane n, so warps 2, 3, 4, 5 take rows
+        // 64, 96, 0, 32 (+lane).
         const int row = (warp & 3) * 32 + lane;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t zb = is_ec ? 0u : zero_bias_bf16x2((uint32_t)__half2float(a.zero[n0 + row]));
-        constexpr int TPT = BN / 128;                      // gate: tokens per thread
-        float pg[TPT];
-#pragma unroll
-        for (int i = 0; i < TPT; ++i) pg[i] = 0.0f;
+        float pg = 0.0f;                                   // EC tiles: gate pre-activation of token `row`
         bool ok = true;
         for (int kt = 0; kt < ksteps + ec_chunks; ++kt) {
             const int s = kt % STAGES;
             if (!mbar_wait(&full[s], (kt / STAGES) & 1)) { atomicOr(a.err, 4u); ok = false; break; }
             if (is_ec) {
-                // Gate pre-activation: x[m, k] w_g[k] over this stage, tokens row + 128 i.
-                const unsigned char* xs = smem + L::X_OFF + s * L::X_BYTES;
+                // Gate pre-activation: x[m, k] w_g[k] over this stage for token m = row.
+                const unsigned char* xr = smem + L::X_OFF + s * L::X_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+                const uint4* wgs = reinterpret_cast<const uint4*>(smem + L::WG_OFF + s * TC_BK * 2);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    float wv[8];
-                    const uint4 wr = ldg_u4(a.wg + (int64_t)kt * TC_BK + 8 * c);
-                    const uint32_t ww[4] = {wr.x, wr.y, wr.z, wr.w};
+                    const uint4 wr = wgs[c];
+                    const uint4 xv = *reinterpret_cast<const uint4*>(xr + ((c ^ (row & 7)) << 4));
+                    const uint32_t ww[4] = {wr.x, wr.y, wr.z, wr.w}, xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) { wv[2 * e] = __uint_as_float(ww[e] << 16); wv[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u); }
-#pragma unroll
-                    for (int i = 0; i < TPT; ++i) {
-                        const int m = row + 128 * i;
-                        const uint4 xr = *reinterpret_cast<const uint4*>(xs + (m >> 3) * 1024 + (m & 7) * 128 + ((c ^ (m & 7)) << 4));
-                        const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            pg[i] = fmaf(__uint_as_float(xw[e] << 16), wv[2 * e], pg[i]);
-                            pg[i] = fmaf(__uint_as_float(xw[e] & 0xFFFF0000u), wv[2 * e + 1], pg[i]);
-                        }
+                    for (int e = 0; e < 4; ++e) {
+                        pg = fmaf(__uint_as_float(xw[e] << 16), __uint_as_float(ww[e] << 16), pg);
+                        pg = fmaf(__uint_as_float(xw[e] & 0xFFFF0000u), __uint_as_float(ww[e] & 0xFFFF0000u), pg);
                     }
                 }
             } else if (kt < ksteps) {
+                // 64 codes of weight row `row` -> 32 TMEM columns of bf16 pairs (q - z), natural order.
                 const uint4* prow = reinterpret_cast<const uint4*>(smem + L::P_OFF + s * L::P_BYTES + row * 32);
-                unsigned char* arow = smem + L::A_OFF + s * L::A_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+                uint32_t o[32];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const uint4 w = prow[h];
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {              // 8 codes -> one 16-byte chunk
-                        uint32_t o[4];
-                        cvt_w4_pairs_natural(ws[q], zb, o);
-                        const int c = h * 4 + q;               // logical 16-byte chunk (k = 8c .. 8c+7)
-                        *reinterpret_cast<uint4*>(arow + ((c ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                    }
+                    cvt_w4_pairs_natural(w.x, zb, o + 16 * h);
+                    cvt_w4_pairs_natural(w.y, zb, o + 16 * h + 4);
+                    cvt_w4_pairs_natural(w.z, zb, o + 16 * h + 8);
+                    cvt_w4_pairs_natural(w.w, zb, o + 16 * h + 12);
                 }
-                fence_proxy_async_smem();                      // generic-proxy writes -> tensor core
+                tmem_st32(tmem_a + lane_base + s * 32, o);
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tc_fence_before();
             }
             mbar_arrive(&cvt[s]);
         }
@@ -337,14 +378,12 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         const bool acc_ok = ok && mbar_wait(acc_full, 0);
         if (!acc_ok) atomicOr(a.err, 4u);
         tc_fence_after();
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         if (is_ec) {
             // g[m] = sigmoid(p[m] + b_g); u[m, j] = g[m] t[j, m] for j = row < r, as bf16.
-#pragma unroll
-            for (int i = 0; i < TPT; ++i) s_gate[row + 128 * i] = 1.0f / (1.0f + expf(-(pg[i] + a.b_g)));
+            s_gate[row] = 1.0f / (1.0f + expf(-(pg + a.b_g)));
             named_bar_epi();
             const int j = row;
-            for (int c0 = 0; c0 < BN; c0 += 16) {
+            for (int c0 = 0; c0 < TC_EB; c0 += 16) {
                 float v[16];
                 tmem_ld16(tmem_d + lane_base + (uint32_t)c0, v);
                 if (!acc_ok || j >= a.rank) continue;
@@ -387,7 +426,7 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     pdl_launch_dependents();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"(ncols) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"(L::TMEM_COLS) : "memory");
     }
 }
 
@@ -428,12 +467,15 @@ static bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
 template <int BN, int STAGES>
 static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
     using L = TcSmem<BN, STAGES>;
-    CUtensorMap mx, mw, ma, mb, mu;
+    CUtensorMap mx, mw, ma, mb, mu, mg, mx128;
     if (!make_map_2d(&mx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.K, (uint64_t)a.M, TC_BK, BN,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     if (!make_map_2d(&mw, a.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(a.K / 2), (uint64_t)a.N, TC_BK / 2,
                      TC_BM, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    if (!make_map_2d(&mx128, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.K, (uint64_t)a.M, TC_BK, TC_EB,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     const bool has_ec = a.rank > 0;
     if (has_ec) {
@@ -443,10 +485,12 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
             !make_map_2d(&mb, a.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.N, (uint64_t)a.rank, 64, 64,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map_2d(&mu, a.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.rank, (uint64_t)a.M, 64, BN,
-                         CU_TENSOR_MAP_SWIZZLE_128B))
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map_2d(&mg, a.wg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.K, 1, TC_BK, 1,
+                         CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     } else {
-        ma = mx; mb = mx; mu = mx;      // unused
+        ma = mx; mb = mx; mu = mx; mg = mx;      // unused
     }
     static bool opted[64] = {false};
     int dev = 0;
@@ -458,7 +502,8 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
         opted[dev] = true;
     }
     const unsigned mblocks = (unsigned)((a.M + BN - 1) / BN);
-    const unsigned tiles = (unsigned)(a.N / TC_BM) * mblocks + (has_ec ? mblocks : 0u);
+    const unsigned eblocks = (unsigned)((a.M + TC_EB - 1) / TC_EB);
+    const unsigned tiles = (unsigned)(a.N / TC_BM) * mblocks + (has_ec ? eblocks : 0u);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles);
     cfg.blockDim = dim3(TC_THREADS);
@@ -469,7 +514,7 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, w4_tc05_kernel<BN, STAGES>, mx, mw, ma, mb, mu, a);
+    return cudaLaunchKernelEx(&cfg, w4_tc05_kernel<BN, STAGES>, mx, mw, ma, mb, mu, mg, mx128, a);
 }
 
 cudaError_t launch_tc05(const TcArgs& a, int bn, cudaStream_t stream) {
