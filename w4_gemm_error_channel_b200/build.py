@@ -1,6 +1,6 @@
 """Build the sm_100a C-ABI library ``libspear.so`` in-tree with nvcc.
 
-    python -m w4_gemm_error_channel_b200.build [--force] [--verbose-ptxas]
+    python w4_gemm_error_channel_b200/build.py [--force] [--verbose-ptxas]
 
 The library links the CUDA runtime statically and takes the driver entry points
 it needs at run time, so it loads on hosts without a GPU (argument checks and
