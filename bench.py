@@ -132,6 +132,21 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sel), "window": where}
 
 
+# ----------------------------------------------------------------------------- replicas
+
+def max_over_ranks(dist, seconds: float, device) -> float:
+    """The slowest rank's time: every rank gets the max (all-reduce MAX)."""
+    import torch
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput of `world` independent replicas timed by the slowest one."""
+    return units_per_rank * world / max_seconds
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 
 def oracle_sample(widx, seconds, M_list):
@@ -261,9 +276,7 @@ def run_ours(args, rank, world, torch, dist):
     torch.cuda.synchronize()
     w1 = time.time()
     if world > 1:
-        t = torch.tensor([t_main], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_main = float(t.item())
+        t_main = max_over_ranks(dist, t_main, dev)
         dist.barrier()
     # The timed region is often shorter than the 100 ms sampling period: then the clocks are
     # read during an untimed soak of the same graph right after it.
@@ -326,9 +339,7 @@ def run_ours(args, rank, world, torch, dist):
     e1.synchronize()
     t_e2e = e0.elapsed_time(e1) / 1e3
     if world > 1:
-        t = torch.tensor([t_e2e], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_e2e = float(t.item())
+        t_e2e = max_over_ranks(dist, t_e2e, dev)
 
     import json as _json
     peaks = {}
@@ -340,18 +351,18 @@ def run_ours(args, rank, world, torch, dist):
     peak_src = "measured" if peaks else "fallback"
 
     if kind == "decode":
-        metric_val = step_bytes * args.steps * world / t_main / 1e9
+        metric_val = replica_throughput(step_bytes * args.steps, world, t_main) / 1e9
         unit = "GB/s"
-        e2e_val = step_bytes * e2e_steps * world / t_e2e / 1e9
+        e2e_val = replica_throughput(step_bytes * e2e_steps, world, t_e2e) / 1e9
         Mr = max(b for b in batches if b <= 16) if any(b <= 16 for b in batches) else max(batches)
         rl = {"bound": "hbm", "achieved": per_m[Mr]["GBps"], "peak": hbm_peak, "unit": "GB/s",
               "frac": per_m[Mr]["GBps"] / hbm_peak, "traffic": None,
               "kernel": f"spear_w4ec_gemm M={Mr} (splitk_w4_kernel with the EC pre-pass overlapped)",
               "peak_source": f"{peak_src} hbm_gbs (copy)", "algorithmic_bytes": layer_bytes(Mr, N, K, r)}
     else:
-        metric_val = step_flops * args.steps * world / t_main / 1e12
+        metric_val = replica_throughput(step_flops * args.steps, world, t_main) / 1e12
         unit = "TFLOP/s"
-        e2e_val = step_flops * e2e_steps * world / t_e2e / 1e12
+        e2e_val = replica_throughput(step_flops * e2e_steps, world, t_e2e) / 1e12
         M0 = batches[0]
         ach = per_m[M0]["TFLOPs"]
         rl = {"bound": "tensor", "achieved": ach, "peak": tc_peak, "unit": "TFLOP/s", "frac": ach / tc_peak,
