@@ -157,6 +157,33 @@ SPEAR_API spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, in
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * spear_w4ec_gemm_noalloc -- the same layer as spear_w4ec_gemm for decode-sized batches, without a
+ * workspace.  The SPEAR pages have no counterpart to this call; it exists for callers that cannot
+ * allocate device memory: code whose device memory belongs to another allocator or framework
+ * that hands out no scratch buffers, and latency-critical paths where an allocation could block
+ * or fail at an unpredictable moment.
+ *
+ * The layer's scratch (an error word, per-token-chunk counters and the compensator's int64
+ * accumulators) lives in one library-owned device array of 256 KiB.  Every GPU that loads the
+ * library holds that array until the process exits.  Nothing is allocated, by this call or by
+ * anything it calls.
+ *
+ *   Arguments as for spear_w4ec_gemm, minus the workspace.  plan may be NULL; a given plan must
+ *   select SPEAR_KERNEL_SPLITK.
+ *   Limits: 1 <= M <= 64 (larger M returns SPEAR_ERR_UNSUPPORTED_SHAPE), rank 0 or 16..256.
+ *   The first call on a device looks up that device's scratch address (once per device, with the
+ *   device current); make that first call before any stream capture.  Every call first clears the
+ *   part of the scratch it uses, then launches the fused decode kernel.
+ *   All calls share the one array and it keeps the last call's contents: calls that can overlap
+ *   on the GPU (different streams, or different host threads) race and must be serialised by the
+ *   caller.  Errors from bounded in-kernel waits are not reported by this call; run the same
+ *   problem through spear_w4ec_gemm and spear_get_device_status to diagnose one.
+ */
+SPEAR_API spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const void* x, int64_t M, int64_t N,
+                                               int64_t K, const void* packed, const void* scale, const void* zero,
+                                               const spear_ec* ec, void* y, spear_dtype y_dtype, void* stream);
+
+/*
  * spear_get_device_status -- read (and optionally clear) the error word that
  * bounded in-kernel waits set when they give up.  Synchronises `stream`.
  * Returns SPEAR_OK, SPEAR_ERR_TIMEOUT, or SPEAR_ERR_CUDA.

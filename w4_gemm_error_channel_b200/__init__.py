@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "SPEAR_OK", 1: "SPEAR_ERR_INVALID_ARG", 2: "SPEAR_ERR_UNSUPPO
                 3: "SPEAR_ERR_MISALIGNED", 4: "SPEAR_ERR_WORKSPACE_TOO_SMALL", 5: "SPEAR_ERR_CUDA",
                 6: "SPEAR_ERR_TIMEOUT"}
 EXPORTED = ["spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_w4ec_gemm",
-            "spear_get_device_status", "spear_status_string", "spear_version"]
+            "spear_w4ec_gemm_noalloc", "spear_get_device_status", "spear_status_string", "spear_version"]
 
 
 class SpearError(RuntimeError):
@@ -52,7 +52,7 @@ class spear_ec(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m w4_gemm_error_channel_b200.build` "
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python w4_gemm_error_channel_b200/build.py` "
                           "(there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I64 = ctypes.c_void_p, ctypes.c_int64
@@ -61,12 +61,14 @@ def _load():
     lib.spear_gemm_plan.argtypes = [I64, I64, I64, ctypes.c_int32, ctypes.c_int, ctypes.POINTER(spear_plan)]
     lib.spear_w4ec_gemm.argtypes = [ctypes.POINTER(spear_plan), P, I64, I64, I64, P, P, P,
                                     ctypes.POINTER(spear_ec), P, ctypes.c_int, P, ctypes.c_size_t, P]
+    lib.spear_w4ec_gemm_noalloc.argtypes = [ctypes.POINTER(spear_plan), P, I64, I64, I64, P, P, P,
+                                            ctypes.POINTER(spear_ec), P, ctypes.c_int, P]
     lib.spear_get_device_status.argtypes = [P, ctypes.c_int, P]
     lib.spear_status_string.argtypes = [ctypes.c_int]
     lib.spear_status_string.restype = ctypes.c_char_p
     lib.spear_version.restype = ctypes.c_int
     for fn in ("spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_w4ec_gemm",
-               "spear_get_device_status"):
+               "spear_w4ec_gemm_noalloc", "spear_get_device_status"):
         getattr(lib, fn).restype = ctypes.c_int
     return lib
 
@@ -187,6 +189,29 @@ def spear_w4ec_gemm(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, 
     _check("spear_w4ec_gemm",
            _lib.spear_w4ec_gemm(ctypes.byref(plan), _p(x), M, N, K, _p(packed), _p(scale), _p(zero), ec_c,
                                 _p(y), yd, _p(workspace), workspace.numel(), _stream(stream)))
+    return y
+
+
+def spear_w4ec_gemm_noalloc(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
+                            ec: Optional[EC] = None, y: Optional[torch.Tensor] = None, y_dtype=torch.bfloat16,
+                            plan: Optional[spear_plan] = None, stream=None):
+    """The layer for up to 64 tokens with the library's own device scratch (no workspace).
+
+    For callers that cannot allocate device memory; calls sharing the scratch must not overlap.
+    """
+    _dev(x, "x")
+    if x.dtype != torch.bfloat16:
+        raise ValueError("x must be bf16")
+    M, K = x.shape
+    N = packed.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=x.device)
+    yd = SPEAR_FP32 if y.dtype == torch.float32 else SPEAR_BF16
+    ec_c = ctypes.byref(ec.as_c()) if ec is not None else None
+    plan_c = ctypes.byref(plan) if plan is not None else None
+    _check("spear_w4ec_gemm_noalloc",
+           _lib.spear_w4ec_gemm_noalloc(plan_c, _p(x), M, N, K, _p(packed), _p(scale), _p(zero), ec_c, _p(y), yd,
+                                        _stream(stream)))
     return y
 
 
