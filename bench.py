@@ -55,7 +55,26 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--sweep", action="store_true",
                     help="time every valid decode tiling for the workload's batches and print a table")
+    ap.add_argument("--once", type=int, default=0, metavar="M",
+                    help="run 5 layer calls of the workload with M tokens and exit (for profilers)")
+    ap.add_argument("--no-ec", action="store_true", help="with --once: the plain W4 layer")
     return ap.parse_args()
+
+
+def measured_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the kernel's
+    source has changed since those counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    entry = json.load(open(path)).get(kernel)
+    if not entry:
+        return None
+    src = os.path.join(ROOT, entry["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != entry["source_sha256_16"]:
+        return None
+    return {"bytes_per_launch": entry["dram_bytes_per_launch"], "workload": entry["workload"]}
 
 
 def layer_bytes(M, N, K, r):
@@ -355,9 +374,11 @@ def run_ours(args, rank, world, torch, dist):
         unit = "GB/s"
         e2e_val = replica_throughput(step_bytes * e2e_steps, world, t_e2e) / 1e9
         Mr = max(b for b in batches if b <= 16) if any(b <= 16 for b in batches) else max(batches)
+        tr = measured_traffic("w4ec_decode_kernel") if (plans[Mr].kernel_id == spear.SPEAR_KERNEL_SPLITK and
+                                                        args.workload == "decode-qo" and Mr == 16) else None
         rl = {"bound": "hbm", "achieved": per_m[Mr]["GBps"], "peak": hbm_peak, "unit": "GB/s",
-              "frac": per_m[Mr]["GBps"] / hbm_peak, "traffic": None,
-              "kernel": f"spear_w4ec_gemm M={Mr} (splitk_w4_kernel with the EC pre-pass overlapped)",
+              "frac": per_m[Mr]["GBps"] / hbm_peak, "traffic": tr["bytes_per_launch"] if tr else None,
+              "kernel": f"spear_w4ec_gemm M={Mr} (w4ec_decode_kernel: EC fused into the weight-streaming kernel)",
               "peak_source": f"{peak_src} hbm_gbs (copy)", "algorithmic_bytes": layer_bytes(Mr, N, K, r)}
     else:
         metric_val = replica_throughput(step_flops * args.steps, world, t_main) / 1e12
@@ -365,8 +386,9 @@ def run_ours(args, rank, world, torch, dist):
         e2e_val = replica_throughput(step_flops * e2e_steps, world, t_e2e) / 1e12
         M0 = batches[0]
         ach = per_m[M0]["TFLOPs"]
+        tr = measured_traffic("w4_tc05_kernel") if args.workload == "prefill" else None
         rl = {"bound": "tensor", "achieved": ach, "peak": tc_peak, "unit": "TFLOP/s", "frac": ach / tc_peak,
-              "traffic": None, "kernel": f"spear_w4ec_gemm M={M0}",
+              "traffic": tr["bytes_per_launch"] if tr else None, "kernel": f"spear_w4ec_gemm M={M0} (w4_tc05_kernel)",
               "peak_source": f"{peak_src} bf16_tflops (burst)", "algorithmic_flops": layer_flops(M0, N, K, r)}
 
     out = {
@@ -487,8 +509,34 @@ def sweep_plans(args):
     print(json.dumps({"workload": args.workload, "sweep": rows}))
 
 
+def run_once(args):
+    """Five untimed calls of one layer of the workload (the launches a profiler captures)."""
+    import torch
+    import w4_gemm_error_channel_b200 as spear
+    from synthetic import config_layers
+    torch.cuda.set_device(0)
+    cfg, batches, kind = WORKLOADS[args.workload]
+    M = args.once
+    L = config_layers(cfg, M=M)[0]
+    packed, scale, zero = spear.spear_pack_w4(torch.from_numpy(L.W).cuda())
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    ec = None if args.no_ec else spear.EC(bf(L.A_bits), bf(L.B_bits), bf(L.wg_bits), L.b_g)
+    x = bf(L.x(M))
+    plan = spear.spear_gemm_plan(M, L.N, L.K, 0 if args.no_ec else L.rank)
+    ws = spear.alloc_workspace(plan.workspace_bytes)
+    y = torch.empty((M, L.N), dtype=torch.bfloat16, device="cuda")
+    for _ in range(5):
+        spear.spear_w4ec_gemm(x, packed, scale, zero, ec, y=y, workspace=ws, plan=plan)
+    torch.cuda.synchronize()
+    print(json.dumps({"once": args.workload, "M": M, "ec": not args.no_ec, "plan": repr(plan),
+                      "device_status": spear.spear_get_device_status(ws)}))
+
+
 def main():
     args = parse()
+    if args.once:
+        run_once(args)
+        return
     if args.sweep:
         sweep_plans(args)
         return
