@@ -49,7 +49,7 @@ extern "C" {
 typedef enum {
     SPEAR_OK = 0,
     SPEAR_ERR_INVALID_ARG = 1,        /* NULL pointer, bad enum, negative size, ... */
-    SPEAR_ERR_UNSUPPORTED_SHAPE = 2,  /* N % 128, K % 64, rank outside 16..256 or not % 16 */
+    SPEAR_ERR_UNSUPPORTED_SHAPE = 2,  /* N % 128, K % 64, rank outside 16..256 or not % 16, K > 65536 with EC */
     SPEAR_ERR_MISALIGNED = 3,         /* a device pointer is not 16-byte aligned */
     SPEAR_ERR_WORKSPACE_TOO_SMALL = 4,
     SPEAR_ERR_CUDA = 5,               /* CUDA runtime / launch failure */
@@ -146,9 +146,9 @@ SPEAR_API spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t 
  *              first use.  Every call leaves its control words zeroed again.
  *              Calls that share a workspace must be ordered on one stream.
  *
- * Requires N % 128 == 0, K % 64 == 0, M >= 0 (M = 0 launches nothing).  The
- * accumulation is fp32 throughout (the EC factors u = g t enter the prefill
- * tensor cores as a bf16 hi/lo pair).  The output is deterministic for a given
+ * Requires N % 128 == 0, K % 64 == 0 (and K <= 65536 with a compensator),
+ * M >= 0 (M = 0 launches nothing).  The accumulation is fp32 throughout (the
+ * EC factors u = g t enter the prefill tensor cores as a bf16 hi/lo pair).  The output is deterministic for a given
  * plan: no atomics take part in any floating-point sum.
  */
 SPEAR_API spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, int64_t N, int64_t K,

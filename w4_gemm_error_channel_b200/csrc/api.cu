@@ -36,6 +36,7 @@ spear_status check_shape(int64_t M, int64_t N, int64_t K, int32_t rank) {
     if (N % 128 != 0 || K % 64 != 0) return SPEAR_ERR_UNSUPPORTED_SHAPE;
     if (M > M_MAX) return SPEAR_ERR_UNSUPPORTED_SHAPE;
     if (rank != 0 && (rank < 16 || rank > 256 || rank % 16 != 0)) return SPEAR_ERR_UNSUPPORTED_SHAPE;
+    if (rank != 0 && K > EC_K_MAX) return SPEAR_ERR_UNSUPPORTED_SHAPE;
     return SPEAR_OK;
 }
 
@@ -55,8 +56,6 @@ size_t workspace_bytes_for(const spear_plan& p, int64_t M, int32_t rank) {
     if (p.kernel_id == SPEAR_KERNEL_TC05 && rank > 0) b += ((size_t)M * rank * 2 + 255) / 256 * 256;
     return b;
 }
-
-int ec_splits_for(int64_t K) { return (int)((K + 63) / 64); }     // 64 rows of A per EC CTA
 
 // Decode plan.  Every weight byte of a CTA (16*g rows x K/S codes, 128 threads) is requested up
 // front; the S K slices of a row tile form a cluster (S in {1, 2, 4, 8}).  The cost model prefers
@@ -302,7 +301,7 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
     a.k_slice = k_slice_for(K, p.split_k);
     a.split = p.split_k;
     a.ec_jr = ec_jr_for(rank, p.split_k);
-    a.ec_splits = rank > 0 ? ec_splits_for(K) : 0;
+    a.ec_splits = decode_ec_ctas_per_chunk(K, rank);
     a.row_tiles = (int)(N / p.tile_n);
     a.tacc = (long long*)(ws + CTRL_BYTES);
     a.err = ctrl;

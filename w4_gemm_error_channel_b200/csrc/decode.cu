@@ -8,11 +8,12 @@
 //   u[m,j] = g[m] t[m,j],  t = x A,  g = sigmoid(x w_g + b_g).
 //
 // One grid, two kinds of CTA (128 threads each):
-//   * EC CTAs (the lowest block indices, so they are dispatched first) each take 128 rows of A
-//     (warp w: 32 rows; lane l: column pairs l, l+32, ...; the gate column by a warp reduction),
-//     compute partial sums of t and of the gate pre-activation, add them into the token chunk's
-//     int64 fixed-point accumulators (2^-32 resolution; integer addition is exact, so the sum
-//     does not depend on arrival order) and count themselves in the chunk's arrival counter;
+//   * EC CTAs (the lowest block indices, so they are dispatched first) each take one 16-column
+//     group of A (or the gate vector) over 512 rows and compute, on the tensor cores, the partial
+//     sums of t (or of the gate pre-activation) for their token chunk.  They add them into the
+//     chunk's int64 fixed-point accumulators (2^-32 resolution; integer addition is exact, so the
+//     sum does not depend on arrival order).  The low 8 bits of every word count the K slices
+//     added so far, so the word itself says when it is complete: no separate flag is published;
 //   * GEMM CTAs own 16*G weight rows, a K slice of at most 512*WPW codes and 8*NB tokens.  Every
 //     weight byte of the CTA is requested from HBM first (registers), then the kernel waits for
 //     its predecessor in the stream (programmatic dependent launch) before reading x.  Lane
@@ -21,16 +22,16 @@
 //     registers and feed mma.sync m16n8k16 with the weights as the M=16 operand and the tokens as
 //     N=8.  Inside each MMA the K order is permuted to pairs (k, k+4), and x is loaded with the
 //     same permutation, which leaves the dot product unchanged;
-//   * the four warps meet in shared memory in a fixed order.  Each GEMM CTA then waits, with a
-//     bounded spin, until all EC CTAs of its token chunk have arrived, forms g = sigmoid(p + b_g)
-//     and u = g t for its share (r/S columns) of the EC term from the accumulators, scales by
-//     s[n] and adds u B (the B slice was prefetched with cp.async at the start).  The S K slices
-//     of a row tile form one thread-block cluster and meet in distributed shared memory: after a
-//     cluster barrier, rank q sums its share of the tile over ranks 0..S-1 in rank order and
-//     rounds once to bf16.
-// No floating-point atomics: results are deterministic for a given plan.  Counters and
-// accumulators re-arm themselves, so the zeroed part of the workspace is zero again after every
-// call.
+//   * the four warps meet in shared memory in a fixed order and each unit (4 rows of one token)
+//     gets its main term s[n] * acc.  Each GEMM CTA then reads the accumulator words of its share
+//     (r/S columns) of the EC term until they are complete (a bounded wait), forms
+//     u = sigmoid(p + b_g) t and adds u B (the B slice was prefetched with cp.async at the
+//     start).  The S K slices of a row tile form one thread-block cluster: every rank pushes each
+//     unit to the rank that owns it in distributed shared memory, and after one cluster barrier
+//     the owner sums the unit over ranks 0..S-1 in rank order and rounds once to bf16.
+// No floating-point atomics: results are deterministic for a given plan.  The last GEMM CTA of a
+// token chunk to read the accumulators clears them, so the zeroed part of the workspace is zero
+// again after every call.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -55,30 +56,45 @@ SPEAR_DEVI unsigned ld_acquire_u32(const unsigned* p) {
     return v;
 }
 
-SPEAR_DEVI void bf16x8_to_f32(const uint4 v, float f[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
+// ---------------------------------------------------------------------------------------------
+// EC role: one EC CTA computes, on the tensor cores, the partial sums over 512 rows of A (a "K
+// slice") of one 16-column group of t = x A, or of the gate pre-activation p = x w_g.  Tokens
+// are the M=16 operand of mma.sync m16n8k16 and columns of A are N.  The 16 columns of group P
+// form two n8 tiles, "even" (columns 16P + 2i) and "odd" (16P + 2i + 1), so that one 32-bit load
+// of A (two adjacent columns of one row) feeds both tiles; the gate group is one n8 tile whose
+// column 0 is w_g.  Warp w takes rows 128 w .. 128 w + 127 of the slice, with its fragments of A
+// in registers (requested before the wait on the previous kernel); the warps meet in shared
+// memory and the CTA adds its sums into the int64 fixed-point accumulators, so each accumulator
+// receives one addition per K slice.
+// ---------------------------------------------------------------------------------------------
+constexpr int EC_KR = 512;                   // rows of A per EC CTA
+constexpr int EC_KK = EC_KR / DK_WARPS / 16; // k16 steps per warp
+constexpr int EC_RS = 20;                    // padded row of the cross-warp buffer (16 columns)
+constexpr float FIX_ONE = 4294967296.0f;     // 2^32: fixed-point resolution 2^-32
+// Each accumulator word holds (sum << 8) + (number of K slices added so far): every addition adds
+// its fixed-point value shifted left by 8 plus one, so a reader knows from the word alone when
+// all slices are in.  That leaves 55 bits for the signed sum: |t| and |p| stay below 2^23.
+constexpr int FIX_COUNT_BITS = 8;
+constexpr unsigned long long FIX_COUNT_MASK = (1ull << FIX_COUNT_BITS) - 1;
+constexpr float FIX_TOTAL = 8388608.0f;      // 2^23
 
-// ---------------------------------------------------------------------------------------------
-// EC role: partial t = x A and p = x w_g over 128 rows of A for one token chunk.
-// Warp w takes rows kbeg + 16 w .. + 15.  Lane l accumulates column pairs (2p, 2p + 1),
-// p = l, l + 32, ..., so a warp reads whole rows of A; the gate column is a per-lane product
-// (lane l < 16 <-> row l of the warp) reduced across the warp.  The warps meet in
-// shared memory, and the CTA's sums go into the int64 fixed-point accumulators.
-// ---------------------------------------------------------------------------------------------
-constexpr int EC_ROWS = 64;                  // rows of A per EC CTA (16 per warp)
-constexpr int EC_WROWS = EC_ROWS / DK_WARPS;
-constexpr double FIX_SCALE = 4294967296.0;   // 2^32
-constexpr float FIX_LIMIT = 67108864.0f;     // 2^26: |CTA partial| bound, so 32 slices fit in int64
+// K slices of the compensator, each adding once into every accumulator word.
+__host__ __device__ inline int ec_slices(int64_t K) { return (int)((K + EC_KR - 1) / EC_KR); }
+
+// EC CTAs per token chunk: one per (K slice, column group), the gate group included.
+int decode_ec_ctas_per_chunk(int64_t K, int rank) {
+    return rank > 0 ? (int)((K + EC_KR - 1) / EC_KR) * (rank / 16 + 1) : 0;
+}
 
 // Signed fixed-point values added as two's-complement 64-bit integers (exact, order-free).
 SPEAR_DEVI void red_add_s64(long long* p, long long v) {
     asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"((unsigned long long)v) : "memory");
+}
+
+SPEAR_DEVI long long ld_relaxed_s64(const long long* p) {
+    long long v;
+    asm volatile("ld.relaxed.gpu.global.s64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
 }
 
 SPEAR_DEVI uint32_t ldg_u32(const void* p) {
@@ -89,117 +105,131 @@ SPEAR_DEVI uint32_t ldg_u32(const void* p) {
 
 template <int TM>
 SPEAR_DEVI void ec_role(const DecodeArgs& a, int s, int chunk, unsigned char* dyn) {
+    constexpr int MT = (TM + 15) / 16;       // m16 token tiles
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = a.rank, NP = r / 2, NC = (NP + 31) / 32, RS = r + 4;
-    uint16_t* xs = reinterpret_cast<uint16_t*>(dyn);                            // [TM][EC_ROWS]
-    float* red_ec = reinterpret_cast<float*>(dyn + (size_t)TM * EC_ROWS * 2);    // [DK_WARPS][8][RS]
-    const int64_t kc0 = (int64_t)s * EC_ROWS;
-    const int64_t kw = kc0 + EC_WROWS * warp;            // this warp's first row
+    const int g = lane >> 2, q = lane & 3;
+    const int r = a.rank, NG = r / 16;
+    const int P = s % (NG + 1), slice = s / (NG + 1);
+    const bool gate = P == NG;
+    const int64_t kw = (int64_t)slice * EC_KR + 16 * EC_KK * warp;   // this warp's first row
     const int64_t m0 = (int64_t)chunk * TM;
     const int tm = (int)imin64(TM, a.M - m0);
 
-    // Prefetch (before the wait) the first 64 columns of this warp's rows and its gate weight.
-    uint32_t a0[EC_WROWS];
+    // Raw words of A (or w_g): rows kw + 16 kk + 2q + {0, 1, 8, 9}, two adjacent columns each.
+    // Every load is issued here, unconditionally (a step past the end of A re-reads its first
+    // rows and is zeroed below), so that all of them are in flight before the wait.
+    uint32_t wv[EC_KK][4];
 #pragma unroll
-    for (int i = 0; i < EC_WROWS; ++i)
-        a0[i] = (kw + i < a.K && lane < NP) ? ldg_u32(a.A + (kw + i) * r + 2 * lane) : 0u;
-    const float wgv = (lane < EC_WROWS && kw + lane < a.K) ? bf16_bits_to_f32(a.wg[kw + lane]) : 0.0f;
+    for (int kk = 0; kk < EC_KK; ++kk) {
+        const int64_t row = (kw + 16 * kk < a.K ? kw + 16 * kk : 0) + 2 * q;
+        if (!gate) {
+            const uint16_t* p = a.A + row * r + 16 * P + 2 * g;
+            wv[kk][0] = ldg_u32(p);
+            wv[kk][1] = ldg_u32(p + r);
+            wv[kk][2] = ldg_u32(p + 8 * r);
+            wv[kk][3] = ldg_u32(p + 9 * r);
+        } else {
+            wv[kk][0] = ldg_u32(a.wg + row);
+            wv[kk][1] = ldg_u32(a.wg + row + 8);
+            wv[kk][2] = wv[kk][3] = 0u;
+        }
+    }
 
     // x may be the previous kernel's output; the previous call may still use the workspace.
     pdl_wait_primary();
+    // Keep every use of the words below the wait, so that the x loads are not held up behind them.
+#pragma unroll
+    for (int kk = 0; kk < EC_KK; ++kk)
+        asm volatile("" : "+r"(wv[kk][0]), "+r"(wv[kk][1]), "+r"(wv[kk][2]), "+r"(wv[kk][3]));
 
-    for (int i = threadIdx.x; i < TM * (EC_ROWS / 8); i += DK_THREADS) {
-        const int m = i / (EC_ROWS / 8), k8 = i % (EC_ROWS / 8);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (m < tm && kc0 + 8 * k8 < a.K) v = ldg_u4(a.x + (m0 + m) * a.K + kc0 + 8 * k8);
-        *reinterpret_cast<uint4*>(xs + m * EC_ROWS + 8 * k8) = v;
+    // x fragments of all token tiles: every load in flight before the first use.
+    uint32_t xa[MT][EC_KK][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int t0 = 16 * mt + g, t1 = t0 + 8;
+#pragma unroll
+        for (int kk = 0; kk < EC_KK; ++kk) {
+            const int64_t k = kw + 16 * kk + 2 * q;
+            const bool in = kw + 16 * kk < a.K;
+            xa[mt][kk][0] = (in && t0 < tm) ? ldg_u32(a.x + (m0 + t0) * a.K + k) : 0u;
+            xa[mt][kk][1] = (in && t1 < tm) ? ldg_u32(a.x + (m0 + t1) * a.K + k) : 0u;
+            xa[mt][kk][2] = (in && t0 < tm) ? ldg_u32(a.x + (m0 + t0) * a.K + k + 8) : 0u;
+            xa[mt][kk][3] = (in && t1 < tm) ? ldg_u32(a.x + (m0 + t1) * a.K + k + 8) : 0u;
+        }
+    }
+
+    // B fragments: [kk][0..1] the even tile, [kk][2..3] the odd tile; the gate tile has w_g in
+    // column 0 (lanes g == 0).  K is a multiple of 64, so a k16 step lies wholly inside or outside.
+    uint32_t b[EC_KK][4];
+#pragma unroll
+    for (int kk = 0; kk < EC_KK; ++kk) {
+        const bool in = kw + 16 * kk < a.K;
+        if (!gate) {
+            b[kk][0] = in ? prmt(wv[kk][0], wv[kk][1], 0x5410u) : 0u;
+            b[kk][1] = in ? prmt(wv[kk][2], wv[kk][3], 0x5410u) : 0u;
+            b[kk][2] = in ? prmt(wv[kk][0], wv[kk][1], 0x7632u) : 0u;
+            b[kk][3] = in ? prmt(wv[kk][2], wv[kk][3], 0x7632u) : 0u;
+        } else {
+            b[kk][0] = (in && g == 0) ? wv[kk][0] : 0u;
+            b[kk][1] = (in && g == 0) ? wv[kk][1] : 0u;
+            b[kk][2] = b[kk][3] = 0u;
+        }
+    }
+
+    // Lane (g, q) ends with columns 4q + {0, 1, 2, 3} of the group for tokens 16 mt + g and + 8.
+    float* red_ec = reinterpret_cast<float*>(dyn);      // [DK_WARPS][TM][EC_RS]
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int t0 = 16 * mt + g, t1 = t0 + 8;
+        float de[4] = {0.f, 0.f, 0.f, 0.f}, dod[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < EC_KK; ++kk) {
+            mma_bf16_16816(de, xa[mt][kk], b[kk][0], b[kk][1]);
+            if (!gate) mma_bf16_16816(dod, xa[mt][kk], b[kk][2], b[kk][3]);
+        }
+        if (t0 < TM)
+            *reinterpret_cast<float4*>(red_ec + (warp * TM + t0) * EC_RS + 4 * q) = make_float4(de[0], dod[0], de[1], dod[1]);
+        if (t1 < TM)
+            *reinterpret_cast<float4*>(red_ec + (warp * TM + t1) * EC_RS + 4 * q) = make_float4(de[2], dod[2], de[3], dod[3]);
     }
     __syncthreads();
 
-    // Column pairs p of this lane against the warp's 32 rows, for tokens ms .. ms+7.
-    auto columns = [&](const uint32_t (&av)[EC_WROWS], int p, int ms) {
-        float acc[8][2];
+    // Cross-warp sums (fixed order), then exact integer accumulation across K slices.  Each slice
+    // is held to its share of the 2^23 bound on |t| and |p|.
+    const float lim = FIX_TOTAL / (float)ec_slices(a.K);
+    long long* tc = a.tacc + (int64_t)chunk * TM * (r + 1);
+    const int ncol = gate ? 1 : 16;
+    for (int o = threadIdx.x; o < tm * ncol; o += DK_THREADS) {
+        const int m = o / ncol, c = o % ncol;
+        float v = red_ec[m * EC_RS + c];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) acc[m][0] = acc[m][1] = 0.0f;
-#pragma unroll
-        for (int i = 0; i < EC_WROWS; ++i) {
-            const float lo = __uint_as_float(av[i] << 16), hi = __uint_as_float(av[i] & 0xFFFF0000u);
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const float xv = bf16_bits_to_f32(xs[(ms + m) * EC_ROWS + EC_WROWS * warp + i]);
-                acc[m][0] = fmaf(xv, lo, acc[m][0]);
-                acc[m][1] = fmaf(xv, hi, acc[m][1]);
-            }
+        for (int w = 1; w < DK_WARPS; ++w) v += red_ec[(w * TM + m) * EC_RS + c];
+        if (!(fabsf(v) < lim)) {
+            atomicOr(a.err, 2u);
+            v = 0.0f;
         }
-        if (p < NP) {
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                red_ec[(warp * 8 + m) * RS + 2 * p] = acc[m][0];
-                red_ec[(warp * 8 + m) * RS + 2 * p + 1] = acc[m][1];
-            }
-        }
-    };
-
-    for (int ms = 0; ms < tm; ms += 8) {
-        columns(a0, lane, ms);
-        for (int c = 1; c < NC; ++c) {
-            const int p = lane + 32 * c;
-            uint32_t av[EC_WROWS];
-#pragma unroll
-            for (int i = 0; i < EC_WROWS; ++i) av[i] = (kw + i < a.K && p < NP) ? ldg_u32(a.A + (kw + i) * r + 2 * p) : 0u;
-            columns(av, p, ms);
-        }
-        // Gate pre-activation: lane l < 16 holds row kw + l (wgv = 0 on the other lanes).
-        float gp[8];
-        const int gl = lane < EC_WROWS ? lane : 0;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) gp[m] = bf16_bits_to_f32(xs[(ms + m) * EC_ROWS + EC_WROWS * warp + gl]) * wgv;
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) gp[m] += __shfl_xor_sync(0xFFFFFFFFu, gp[m], o);
-        if (lane == 0) {
-#pragma unroll
-            for (int m = 0; m < 8; ++m) red_ec[(warp * 8 + m) * RS + r] = gp[m];
-        }
-        __syncthreads();
-        // Cross-warp sums (fixed order), then exact integer accumulation across CTAs.
-        for (int o = threadIdx.x; o < 8 * (r + 1); o += DK_THREADS) {
-            const int m = o / (r + 1), j = o % (r + 1);
-            if (ms + m >= tm) continue;
-            float v = red_ec[m * RS + j];
-#pragma unroll
-            for (int w = 1; w < DK_WARPS; ++w) v += red_ec[(w * 8 + m) * RS + j];
-            if (!(fabsf(v) < FIX_LIMIT)) {
-                atomicOr(a.err, 2u);
-                v = 0.0f;
-            }
-            red_add_s64(a.tacc + (chunk * TM + ms + m) * (int64_t)(r + 1) + j, __double2ll_rn((double)v * FIX_SCALE));
-        }
-        __syncthreads();
+        const unsigned long long fx = (unsigned long long)__float2ll_rn(v * FIX_ONE);
+        red_add_s64(tc + (int64_t)m * (r + 1) + (gate ? r : 16 * P + c), (long long)((fx << FIX_COUNT_BITS) | 1ull));
     }
-    __syncthreads();
     pdl_launch_dependents();
-    if (threadIdx.x == 0) {
-        // The barrier above orders every thread's accumulator additions before this fence; the
-        // release add then publishes the arrival.
-        __threadfence();
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&a.arrivals[chunk]) : "memory");
-    }
 }
 
 // ---------------------------------------------------------------------------------------------
 // Cluster helpers (distributed shared memory).
 // ---------------------------------------------------------------------------------------------
+// Split form of the cluster barrier: the arrive at kernel start and the wait before the first
+// remote store make sure every CTA of the cluster is running before its shared memory is written.
+SPEAR_DEVI void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
+SPEAR_DEVI void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 SPEAR_DEVI void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-SPEAR_DEVI float4 ld_dsmem_f4(const float* local, unsigned rank) {
+// Store to the same shared-memory offset in cluster rank `rank`.
+SPEAR_DEVI void st_dsmem_f4(float4* local, unsigned rank, float4 v) {
     uint32_t la = (uint32_t)__cvta_generic_to_shared(local), ra;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(la), "r"(rank));
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(ra) : "memory");
-    return v;
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(ra), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -209,8 +239,11 @@ template <int NB, int G, int WPW>
 SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsigned char* dyn) {
     constexpr int RT = 16 * G;        // weight rows per CTA
     constexpr int TM = 8 * NB;        // tokens per CTA
-    __shared__ float red[DK_WARPS][RT][TM + 1];
-    __shared__ __align__(16) float ps[TM * RT];      // this K slice's finished partial, [token][row]
+    constexpr int RT4 = RT / 4;
+    constexpr int RS = RT + 4;        // padded row: the fragment stores below are conflict-free
+    __shared__ __align__(16) float red[DK_WARPS][TM][RS];
+    // K slices pushed here by the cluster's ranks: [rank][this CTA's share of the tile].
+    __shared__ __align__(16) float4 recv[TM * RT4];
     __shared__ float s_scale[RT];
     __shared__ unsigned s_flag;
     uint16_t* Bs = reinterpret_cast<uint16_t*>(dyn);                           // [ec_jr][RT] bf16
@@ -227,6 +260,8 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
     const bool has_ec = a.rank > 0;
     const int j0 = ks * a.ec_jr;
     const int nj = has_ec ? max(0, min(a.rank, j0 + a.ec_jr) - j0) : 0;
+
+    if (S > 1) cluster_arrive_relaxed();
 
     // ---- Prologue: only inputs that no earlier kernel in the stream can be writing. ----
     if (nj > 0) {
@@ -313,50 +348,187 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
     for (int i = 0; i < G; ++i)
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-            red[warp][16 * i + g][8 * b + 2 * t] = acc[i][b][0];
-            red[warp][16 * i + g][8 * b + 2 * t + 1] = acc[i][b][1];
-            red[warp][16 * i + g + 8][8 * b + 2 * t] = acc[i][b][2];
-            red[warp][16 * i + g + 8][8 * b + 2 * t + 1] = acc[i][b][3];
+            red[warp][8 * b + 2 * t][16 * i + g] = acc[i][b][0];
+            red[warp][8 * b + 2 * t + 1][16 * i + g] = acc[i][b][1];
+            red[warp][8 * b + 2 * t][16 * i + g + 8] = acc[i][b][2];
+            red[warp][8 * b + 2 * t + 1][16 * i + g + 8] = acc[i][b][3];
         }
     pdl_launch_dependents();
     const int tm = (int)imin64(TM, a.M - m0);
+    __syncthreads();
+
+    // Output units: 4 rows of one token, e4 = token * RT4 + row / 4.  The main term of each unit,
+    // s[n] * (sum over warps), is formed here, before the wait for the compensator.
+    auto main_part = [&](int e4) {
+        const int r4 = e4 % RT4, mm = min(e4 / RT4, TM - 1);
+        float4 acc = *reinterpret_cast<const float4*>(&red[0][mm][4 * r4]);
+#pragma unroll
+        for (int w = 1; w < DK_WARPS; ++w) {
+            const float4 p = *reinterpret_cast<const float4*>(&red[w][mm][4 * r4]);
+            acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
+        }
+        acc.x *= s_scale[4 * r4]; acc.y *= s_scale[4 * r4 + 1];
+        acc.z *= s_scale[4 * r4 + 2]; acc.w *= s_scale[4 * r4 + 3];
+        return acc;
+    };
+    const int units = tm * RT4;
+    // With few units and an EC term, TPU lanes (a power of two, at most a warp) share one unit's
+    // EC columns and meet by shuffles in a fixed order; otherwise thread i takes units i, i + 128, ...
+    const bool spread = nj > 0 && 2 * units <= DK_THREADS;
+    int tpu = 1;
+    if (spread)
+        while (2 * tpu * units <= DK_THREADS && tpu < 32) tpu *= 2;
+    const int se4 = threadIdx.x / tpu, sub = threadIdx.x % tpu;
+    constexpr int UPT = (TM * RT4 + DK_THREADS - 1) / DK_THREADS;
+    float4 v[UPT];
+    if (spread) {
+        v[0] = (se4 < units && sub == 0) ? main_part(se4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+#pragma unroll
+        for (int q = 0; q < UPT; ++q) v[q] = main_part(threadIdx.x + q * DK_THREADS);
+    }
 
     if (has_ec) {
-        // Every EC CTA of this token chunk has added its partial sums (bounded wait).
-        if (threadIdx.x == 0) {
-            unsigned it = 0, ok = 1;
-            while (ld_acquire_u32(&a.arrivals[chunk]) < (unsigned)a.ec_splits) {
-                if (++it > SPIN_LIMIT) { atomicOr(a.err, 1u); ok = 0; break; }
-                if (it > 256) __nanosleep(64);
-            }
-            s_flag = ok;
-        }
-        __syncthreads();
-        // g = sigmoid(p + b_g) and u = g t for this CTA's EC columns, from the exact accumulators.
+        // u = sigmoid(p + b_g) t for this CTA's EC columns.  Element c = mm * nj + jj; thread i
+        // takes c = i, i + 128, ... (stepping without dividing) and reads the words of t[mm, j0 + jj]
+        // and p[mm] until both hold every K slice (a bounded wait); each element recomputes its
+        // token's gate, so one pass and one barrier suffice.
         const long long* tc = a.tacc + (int64_t)chunk * TM * (a.rank + 1);
-        for (int c = threadIdx.x; c < tm * (nj + 1); c += DK_THREADS) {
-            const int mm = c / (nj + 1), jj = c % (nj + 1);
-            const int col = jj < nj ? j0 + jj : a.rank;
-            const long long v = s_flag ? __ldcg(tc + (int64_t)mm * (a.rank + 1) + col) : 0ll;
-            us[mm * (a.ec_jr + 1) + jj] = (float)((double)v * (1.0 / FIX_SCALE));
+        const int ujr = a.ec_jr + 1, total = tm * nj;
+        const unsigned long long want = (unsigned long long)ec_slices(a.K) & FIX_COUNT_MASK;
+        if (nj > 0) {
+            const int dmm = DK_THREADS / nj, djj = DK_THREADS % nj;
+            int mm = threadIdx.x / nj, jj = threadIdx.x % nj;
+            constexpr int UB = 8;         // elements per thread per pass, loads issued together
+            for (int base = 0; base < total; base += UB * DK_THREADS) {   // uniform trip count
+                const long long* tp[UB];
+                const long long* pp[UB];
+                int um[UB], uj[UB];
+                bool valid[UB];
+#pragma unroll
+                for (int u = 0; u < UB; ++u) {
+                    valid[u] = base + (int)threadIdx.x + u * DK_THREADS < total;
+                    um[u] = mm;
+                    uj[u] = jj;
+                    tp[u] = tc + (int64_t)(valid[u] ? mm : 0) * (a.rank + 1) + j0 + (valid[u] ? jj : 0);
+                    pp[u] = tc + (int64_t)(valid[u] ? mm : 0) * (a.rank + 1) + a.rank;
+                    mm += dmm;
+                    jj += djj;
+                    if (jj >= nj) { jj -= nj; ++mm; }
+                }
+                long long tv[UB], pv[UB];
+                unsigned it = 0;
+                for (;;) {
+                    bool done = true;
+#pragma unroll
+                    for (int u = 0; u < UB; ++u) {
+                        tv[u] = valid[u] ? ld_relaxed_s64(tp[u]) : 0ll;
+                        pv[u] = valid[u] ? ld_relaxed_s64(pp[u]) : 0ll;
+                    }
+#pragma unroll
+                    for (int u = 0; u < UB; ++u)
+                        done = done && (!valid[u] || (((unsigned long long)tv[u] & FIX_COUNT_MASK) == want &&
+                                                      ((unsigned long long)pv[u] & FIX_COUNT_MASK) == want));
+                    if (__syncthreads_and(done)) break;
+                    if (++it > SPIN_LIMIT) {          // give up: flag it and add nothing
+                        if (threadIdx.x == 0) atomicOr(a.err, 1u);
+#pragma unroll
+                        for (int u = 0; u < UB; ++u) tv[u] = pv[u] = 0ll;
+                        break;
+                    }
+                    if (it > 16) __nanosleep(64);
+                }
+#pragma unroll
+                for (int u = 0; u < UB; ++u) {
+                    if (valid[u]) {
+                        const float t_ = __ll2float_rn(tv[u] >> FIX_COUNT_BITS) * (1.0f / FIX_ONE);
+                        const float p_ = __ll2float_rn(pv[u] >> FIX_COUNT_BITS) * (1.0f / FIX_ONE);
+                        us[um[u] * ujr + uj[u]] = __fdividef(t_, 1.0f + __expf(-(p_ + a.b_g)));
+                    }
+                }
+            }
+            asm volatile("cp.async.wait_all;" ::: "memory");
         }
         __syncthreads();
-        for (int mm = threadIdx.x; mm < tm; mm += DK_THREADS) {
-            const float p = us[mm * (a.ec_jr + 1) + nj] + a.b_g;
-            us[mm * (a.ec_jr + 1) + nj] = 1.0f / (1.0f + expf(-p));
+
+        // This slice's EC columns: sum_j u[m, j] B[j, n] added to each unit.
+        if (spread) {
+            if (se4 < units) {
+                const int r4 = se4 % RT4, mu = se4 / RT4;
+                const float* ur = us + mu * ujr;
+                const uint16_t* br = Bs + 4 * r4;
+#pragma unroll 8
+                for (int jj = sub; jj < nj; jj += tpu) {
+                    const float uq = ur[jj];
+                    const uint2 bb = *reinterpret_cast<const uint2*>(br + jj * RT);
+                    v[0].x = fmaf(uq, __uint_as_float(bb.x << 16), v[0].x);
+                    v[0].y = fmaf(uq, __uint_as_float(bb.x & 0xFFFF0000u), v[0].y);
+                    v[0].z = fmaf(uq, __uint_as_float(bb.y << 16), v[0].z);
+                    v[0].w = fmaf(uq, __uint_as_float(bb.y & 0xFFFF0000u), v[0].w);
+                }
+            }
+            for (int o = 1; o < tpu; o *= 2) {
+                v[0].x += __shfl_down_sync(0xFFFFFFFFu, v[0].x, o);
+                v[0].y += __shfl_down_sync(0xFFFFFFFFu, v[0].y, o);
+                v[0].z += __shfl_down_sync(0xFFFFFFFFu, v[0].z, o);
+                v[0].w += __shfl_down_sync(0xFFFFFFFFu, v[0].w, o);
+            }
+        } else {
+#pragma unroll 4
+            for (int jj = 0; jj < nj; ++jj) {
+#pragma unroll
+                for (int q = 0; q < UPT; ++q) {
+                    const int e4 = threadIdx.x + q * DK_THREADS;
+                    const int r4 = e4 % RT4, mu = min(e4 / RT4, TM - 1);
+                    const float uq = us[mu * ujr + jj];
+                    const uint2 bb = *reinterpret_cast<const uint2*>(Bs + jj * RT + 4 * r4);
+                    v[q].x = fmaf(uq, __uint_as_float(bb.x << 16), v[q].x);
+                    v[q].y = fmaf(uq, __uint_as_float(bb.x & 0xFFFF0000u), v[q].y);
+                    v[q].z = fmaf(uq, __uint_as_float(bb.y << 16), v[q].z);
+                    v[q].w = fmaf(uq, __uint_as_float(bb.y & 0xFFFF0000u), v[q].w);
+                }
+            }
         }
-        __syncthreads();
-        for (int c = threadIdx.x; c < tm * nj; c += DK_THREADS) {
-            const int mm = c / nj, jj = c % nj;
-            us[mm * (a.ec_jr + 1) + jj] *= us[mm * (a.ec_jr + 1) + nj];
-        }
-        if (nj > 0) asm volatile("cp.async.wait_all;" ::: "memory");
     }
-    __syncthreads();
-    if (has_ec) {
-        // Every GEMM CTA of the chunk has read the accumulators: the last one clears them and the
-        // arrival counter for the next call.  Two counter levels (groups of CONSUMER_GROUP CTAs,
-        // then groups) keep same-address atomics few.
+
+    auto store4 = [&](int64_t m, int r4, float4 o) {
+        if (a.y_fp32) {
+            reinterpret_cast<float4*>(reinterpret_cast<float*>(a.y) + m * a.N + n0)[r4] = o;
+        } else {
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y), hi = __floats2bfloat162_rn(o.z, o.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+            pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+            reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.y) + m * a.N + n0)[r4] = pk;
+        }
+    };
+    // The S K slices of a row tile (one cluster) meet in distributed shared memory: unit e4 of the
+    // tile belongs to rank e4 / per, and every rank pushes its value of the unit to that owner.
+    const int per = TM * RT4 / S;
+    auto emit = [&](int e4, float4 o) {
+        if (S == 1) {
+            store4(m0 + e4 / RT4, e4 % RT4, o);
+        } else {
+            const int owner = e4 / per;
+            st_dsmem_f4(&recv[ks * per + (e4 - owner * per)], (unsigned)owner, o);
+        }
+    };
+    if (S > 1) cluster_wait();
+    if (spread) {
+        if (se4 < units && sub == 0) emit(se4, v[0]);
+    } else {
+#pragma unroll
+        for (int q = 0; q < UPT; ++q) {
+            const int e4 = threadIdx.x + q * DK_THREADS;
+            if (e4 < units) emit(e4, v[q]);
+        }
+    }
+
+    // Every GEMM CTA of the chunk has read the accumulators (before the barrier above): the last
+    // one clears them and the arrival counter for the next call.  Two counter levels (groups of
+    // CONSUMER_GROUP CTAs, then groups) keep same-address atomics few; this is off the path to y.
+    auto retire_accumulators = [&]() {
+        if (!has_ec) return;
         if (threadIdx.x == 0) {
             const int per_chunk = a.row_tiles * S;
             const int idx = tile * S + ks;                 // this CTA's index within the chunk
@@ -380,61 +552,27 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
                 a.arrivals[chunk] = 0u;
             }
         }
+    };
+    if (S == 1) {
+        retire_accumulators();
+        return;
     }
 
-    // Per element: s[n] * (sum over warps) + this slice's EC columns.
-    for (int e = threadIdx.x; e < RT * TM; e += DK_THREADS) {
-        const int rr = e % RT, mm = e / RT;
-        float v = 0.0f;
-        if (mm < tm) {
-            v = red[0][rr][mm];
-#pragma unroll
-            for (int w = 1; w < DK_WARPS; ++w) v += red[w][rr][mm];
-            v *= s_scale[rr];
-            for (int jj = 0; jj < nj; ++jj)
-                v = fmaf(us[mm * (a.ec_jr + 1) + jj], bf16_bits_to_f32(Bs[jj * RT + rr]), v);
-        }
-        if (S == 1) {
-            if (mm < tm) {
-                const int64_t n = n0 + rr, m = m0 + mm;
-                if (a.y_fp32)
-                    reinterpret_cast<float*>(a.y)[m * a.N + n] = v;
-                else
-                    reinterpret_cast<__nv_bfloat16*>(a.y)[m * a.N + n] = __float2bfloat16_rn(v);
-            }
-        } else {
-            ps[mm * RT + rr] = v;
-        }
-    }
-    if (S == 1) return;
-
-    // The S K slices of this row tile (one cluster) meet in distributed shared memory: rank ks sums
-    // its share of the tile over ranks 0..S-1 in rank order, then rounds once.
+    // After the barrier every push has landed; the owner sums its units over ranks 0..S-1 in rank
+    // order and rounds once.  No rank touches another's shared memory after the barrier.
     cluster_sync_all();
-    constexpr int RT4 = RT / 4;
-    const int total4 = tm * RT4;
-    const int per = (total4 + S - 1) / S;
-    const int e_beg = ks * per, e_end = min(total4, e_beg + per);
-    for (int e = e_beg + threadIdx.x; e < e_end; e += DK_THREADS) {
-        const int r4 = e % RT4, mm = e / RT4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q = 0; q < S; ++q) {
-            const float4 p = ld_dsmem_f4(ps + mm * RT + 4 * r4, (unsigned)q);
-            v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
+    for (int l = threadIdx.x; l < per; l += DK_THREADS) {
+        const int e4 = ks * per + l;
+        const int r4 = e4 % RT4, mm = e4 / RT4;
+        if (mm >= tm) continue;
+        float4 o = recv[l];
+        for (int q = 1; q < S; ++q) {
+            const float4 p = recv[q * per + l];
+            o.x += p.x; o.y += p.y; o.z += p.z; o.w += p.w;
         }
-        const int64_t m = m0 + mm;
-        if (a.y_fp32) {
-            reinterpret_cast<float4*>(reinterpret_cast<float*>(a.y) + m * a.N + n0)[r4] = v;
-        } else {
-            const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-            pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-            reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.y) + m * a.N + n0)[r4] = pk;
-        }
+        store4(m0 + mm, r4, o);
     }
-    // Keep this CTA's shared memory alive until every rank has read it.
-    cluster_sync_all();
+    retire_accumulators();
 }
 
 template <int NB, int G, int WPW>
@@ -458,7 +596,7 @@ __global__ void __launch_bounds__(DK_THREADS, 4) w4ec_decode_kernel(DecodeArgs a
 size_t decode_dyn_smem_bytes(int nb, int g, int ec_jr, int rank) {
     if (rank <= 0) return 0;
     const size_t gemm = (size_t)ec_jr * 16 * g * 2 + (size_t)8 * nb * (ec_jr + 1) * 4;
-    const size_t ec = (size_t)8 * nb * EC_ROWS * 2 + (size_t)DK_WARPS * 8 * (rank + 4) * 4;
+    const size_t ec = (size_t)DK_WARPS * 8 * nb * EC_RS * 4;
     return gemm > ec ? gemm : ec;
 }
 

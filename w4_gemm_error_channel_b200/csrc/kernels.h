@@ -49,7 +49,7 @@ struct DecodeArgs {
     int64_t k_slice;        // GEMM K slice per CTA, a multiple of 64
     int split;              // S: GEMM K slices = thread-block cluster size (1, 2, 4 or 8)
     int ec_jr;              // EC columns added per K slice (multiple of 4)
-    int ec_splits;          // EC CTAs per token chunk (128 rows of A each)
+    int ec_splits;          // EC CTAs per token chunk (decode_ec_ctas_per_chunk)
     int ec_ctas;            // EC CTAs in the grid (ec_splits * mchunks, padded to whole clusters)
     int row_tiles;          // N / (16 G)
     int mchunks;            // ceil(M / (8 NB))
@@ -91,6 +91,9 @@ cudaError_t launch_unpack_w4(const void* packed, const void* zero, int64_t N, in
 // nb: tokens per CTA = 8*nb (1, 2, 4); g: weight rows per CTA = 16*g; wpw: 128-wide K windows per
 // warp (K slice of a CTA <= 512*wpw).  decode_config_supported() lists the compiled combinations.
 bool decode_config_supported(int nb, int g, int wpw);
+// Largest K with a compensator: the decode kernel counts K slices of 512 rows in 8 bits.
+constexpr int64_t EC_K_MAX = 65536;
+int decode_ec_ctas_per_chunk(int64_t K, int rank);
 size_t decode_dyn_smem_bytes(int nb, int g, int ec_jr, int rank);
 cudaError_t launch_decode(const DecodeArgs& a, int nb, int g, int wpw, cudaStream_t stream);
 

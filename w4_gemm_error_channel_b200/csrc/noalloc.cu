@@ -67,7 +67,7 @@ extern "C" spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const vo
     if (M <= 0 || N <= 0 || K <= 0) return SPEAR_ERR_INVALID_ARG;
     if (M > NOALLOC_M_MAX) return SPEAR_ERR_UNSUPPORTED_SHAPE;       // the scratch is sized for 64 tokens
     if (N % 128 != 0 || K % 64 != 0) return SPEAR_ERR_UNSUPPORTED_SHAPE;
-    if (ec && (rank < 16 || rank > 256 || rank % 16 != 0)) return SPEAR_ERR_UNSUPPORTED_SHAPE;
+    if (ec && (rank < 16 || rank > 256 || rank % 16 != 0 || K > EC_K_MAX)) return SPEAR_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(x) || !aligned16(packed) || !aligned16(scale) || !aligned16(zero) || !aligned16(y))
         return SPEAR_ERR_MISALIGNED;
     if (ec && (!aligned16(ec->A) || !aligned16(ec->B) || !aligned16(ec->w_g))) return SPEAR_ERR_MISALIGNED;
@@ -115,7 +115,7 @@ extern "C" spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const vo
     a.k_slice = ksl;
     a.split = p.split_k;
     a.ec_jr = rank > 0 ? (int)(((rank + p.split_k - 1) / p.split_k + 3) / 4 * 4) : 0;
-    a.ec_splits = rank > 0 ? (int)((K + 63) / 64) : 0;
+    a.ec_splits = decode_ec_ctas_per_chunk(K, rank);
     a.row_tiles = (int)(N / p.tile_n);
     a.mchunks = (int)((M + p.tile_m - 1) / p.tile_m);
     a.ec_ctas = (a.ec_splits * a.mchunks + p.split_k - 1) / p.split_k * p.split_k;
