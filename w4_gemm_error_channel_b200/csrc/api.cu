@@ -64,9 +64,11 @@ size_t workspace_bytes_for(const spear_plan& p, int64_t M, int32_t rank) {
 // Measured plans (plans/gen_table.py): the fastest tiling per swept shape on one B200.
 struct MeasuredPlan {
     int64_t M, N, K;
-    int has_ec, tile_n, split_k;
+    int has_ec, kernel_id, tile_n, split_k;
     double us;
 };
+spear_status plan_tc05(int64_t M, spear_plan* p);
+
 const MeasuredPlan kMeasured[] = {
 #include "plan_table.inc"
 };
@@ -81,6 +83,7 @@ bool lookup_measured(int64_t M, int64_t N, int64_t K, int has_ec, spear_plan* p)
         if (!best || std::llabs(e.M - M) < std::llabs(best->M - M)) best = &e;
     }
     if (!best) return false;
+    if (best->kernel_id == SPEAR_KERNEL_TC05) return plan_tc05(M, p) == SPEAR_OK;
     p->kernel_id = SPEAR_KERNEL_SPLITK;
     p->tile_n = best->tile_n;
     p->split_k = best->split_k;
