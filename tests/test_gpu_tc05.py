@@ -38,7 +38,7 @@ def run(L, M, tile_m, y_dtype=torch.bfloat16, rows=None):
     return got, ref
 
 
-@pytest.mark.parametrize("tile_m", [128, 256])
+@pytest.mark.parametrize("tile_m", [128, 160, 192, 256])
 @pytest.mark.parametrize("M", [1, 77, 128, 129, 300, 512])
 def test_tc05_small(M, tile_m):
     L = make_layer("tc", 5 + M, M, 384, 448, 0, outlier_frac=0.02, outlier_scale=10.0)
@@ -52,7 +52,7 @@ def test_tc05_fp32_output():
     check_close(got, ref, False, "tc05 fp32")
 
 
-@pytest.mark.parametrize("tile_m", [128, 256])
+@pytest.mark.parametrize("tile_m", [128, 160, 192, 256])
 def test_tc05_prefill_shape_sampled(tile_m):
     L = config_layers(3)[0]
     rows = np.array([0, 1, 255, 256, 1031, 2047])
@@ -87,13 +87,15 @@ def run_ec(L, M, tile_m, rows=None, b_g=None, y_dtype=torch.bfloat16):
     return got, ref, y, ws
 
 
-@pytest.mark.parametrize("tile_m", [128, 256])
+@pytest.mark.parametrize("tile_m", [128, 160, 192, 256])
 @pytest.mark.parametrize("r", [16, 32, 48, 64, 128])
 @pytest.mark.parametrize("M", [128, 300])
 def test_tc05_ec_small(M, r, tile_m):
     L = make_layer("tcec", 11 + r + M, M, 256, 512, r, outlier_frac=0.02, outlier_scale=10.0, b_g=0.3)
-    got, ref, _, _ = run_ec(L, M, tile_m)
+    got, ref, _, ws = run_ec(L, M, tile_m)
     check_close(got, ref, True, f"tc05 EC M={M} r={r} tile_m={tile_m}")
+    # Token tiles of 160 or 192 share 128-token EC blocks; every flag must still be re-armed.
+    assert int(ws[: (128 + 1024) * 1024].count_nonzero().item()) == 0, "EC flags not re-armed"
 
 
 def test_tc05_ec_fp32_and_gate_off():
@@ -106,7 +108,7 @@ def test_tc05_ec_fp32_and_gate_off():
     assert np.array_equal(host_f64(y_off), plain)
 
 
-@pytest.mark.parametrize("tile_m", [128, 256])
+@pytest.mark.parametrize("tile_m", [128, 160, 192, 256])
 def test_tc05_ec_prefill_sampled(tile_m):
     L = config_layers(3)[0]
     rows = np.array([0, 1, 255, 256, 1031, 2047])

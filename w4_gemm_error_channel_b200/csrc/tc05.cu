@@ -234,25 +234,31 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
-            pdl_wait_primary();            // x may be written by the previous kernel in the stream
-            bool ok = true;
-            for (int kt = 0; kt < ksteps && ok; ++kt) {
-                const int s = kt % STAGES;
-                if (kt >= STAGES && !mbar_wait(&empty[s], ((kt / STAGES) - 1) & 1)) { atomicOr(a.err, 4u); ok = false; break; }
-                unsigned char* xs = smem + L::X_OFF + s * L::X_BYTES;
+            // Weight-side operands (packed W, or A and w_g) of a stage; x only after the wait.
+            auto load_weights = [&](int kt, int s) {
                 if (is_ec) {
-                    // x (128 tokens), A[k, j] in 64-wide MN-major boxes, and the w_g slice.
                     unsigned char* as = smem + L::A_OFF + s * L::A_BYTES;
                     mbar_arrive_expect_tx(&full[s], TC_EB * TC_BK * 2 + rboxes * (TC_BK * 64 * 2) + TC_BK * 2);
-                    tma_load_2d(xs, &tmap_x128, kt * TC_BK, (int32_t)m0, &full[s]);
                     for (int bx = 0; bx < rboxes; ++bx)
                         tma_load_2d(as + bx * (TC_BK * 64 * 2), &tmap_a, bx * 64, kt * TC_BK, &full[s]);
                     tma_load_2d(smem + L::WG_OFF + s * TC_BK * 2, &tmap_g, kt * TC_BK, 0, &full[s]);
                 } else {
                     mbar_arrive_expect_tx(&full[s], L::X_BYTES + L::P_BYTES);
-                    tma_load_2d(xs, &tmap_x, kt * TC_BK, (int32_t)m0, &full[s]);
                     tma_load_2d(smem + L::P_OFF + s * L::P_BYTES, &tmap_w, kt * (TC_BK / 2), (int32_t)n0, &full[s]);
                 }
+            };
+            const int pre = ksteps < STAGES ? ksteps : STAGES;
+            for (int kt = 0; kt < pre; ++kt) load_weights(kt, kt);
+            pdl_wait_primary();            // x may be written by the previous kernel in the stream
+            bool ok = true;
+            for (int kt = 0; kt < ksteps && ok; ++kt) {
+                const int s = kt % STAGES;
+                if (kt >= STAGES) {
+                    if (!mbar_wait(&empty[s], ((kt / STAGES) - 1) & 1)) { atomicOr(a.err, 4u); ok = false; break; }
+                    load_weights(kt, s);
+                }
+                unsigned char* xs = smem + L::X_OFF + s * L::X_BYTES;
+                tma_load_2d(xs, is_ec ? &tmap_x128 : &tmap_x, kt * TC_BK, (int32_t)m0, &full[s]);
             }
             if (ok && ec_chunks > 0) {
                 // u of these tokens is written by their EC tiles: wait (bounded) for the flags.
@@ -275,12 +281,17 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                     tma_load_2d(as + 64 * 64 * 2, &tmap_b, (int32_t)n0 + 64, c * 64, &full[s]);
                 }
                 // Every main tile of these tokens has seen the flags: the last one re-arms each.
+                // EC block e is read by every weight tile of each token block that overlaps it.
                 if (ok) {
-                    for (int e = e_lo; e < e_hi; ++e)
-                        if (atomicAdd(&a.ec_consumed[e], 1u) == (unsigned)ntiles - 1) {
+                    for (int e = e_lo; e < e_hi; ++e) {
+                        const int64_t t_lo = (int64_t)e * TC_EB;
+                        const int64_t t_hi = ((int64_t)(e + 1) * TC_EB < a.M ? (int64_t)(e + 1) * TC_EB : a.M) - 1;
+                        const unsigned readers = (unsigned)ntiles * (unsigned)(t_hi / BN - t_lo / BN + 1);
+                        if (atomicAdd(&a.ec_consumed[e], 1u) == readers - 1) {
                             a.ec_consumed[e] = 0u;
                             a.ec_ready[e] = 0u;
                         }
+                    }
                 }
             }
         }
@@ -519,6 +530,8 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_tc05(const TcArgs& a, int bn, cudaStream_t stream) {
     if (bn == 128) return launch_tc_t<128, 4>(a, stream);
+    if (bn == 160) return launch_tc_t<160, 4>(a, stream);
+    if (bn == 192) return launch_tc_t<192, 3>(a, stream);
     if (bn == 256) return launch_tc_t<256, 3>(a, stream);
     return cudaErrorInvalidValue;
 }
