@@ -115,6 +115,11 @@ def test_gemm_rejects_bad_plans():
         q = spear.spear_plan.from_buffer_copy(p)
         setattr(q, field, val)
         assert _gemm(plan=ctypes.byref(q)) == INVALID, field
+    # tcgen05 plans: 256 weight rows only with 128-token tiles; token widths 128, 160, 192, 256.
+    for tile_n, tile_m in ((256, 256), (256, 160), (64, 128), (128, 144)):
+        q = spear.spear_plan.from_buffer_copy(p)
+        q.kernel_id, q.split_k, q.tile_n, q.tile_m = 2, 1, tile_n, tile_m
+        assert _gemm(plan=ctypes.byref(q)) == INVALID, (tile_n, tile_m)
 
 
 def test_pack_and_unpack_host_checks():

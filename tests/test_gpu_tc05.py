@@ -15,20 +15,20 @@ else:
     spear = None
 
 
-def tc_plan(M, N, K, tile_m):
+def tc_plan(M, N, K, tile_m, wrows=128):
     p = spear.spear_gemm_plan(M, N, K, 0)
     p.kernel_id = spear.SPEAR_KERNEL_TC05
-    p.tile_n, p.split_k, p.tile_m = 128, 1, tile_m
+    p.tile_n, p.split_k, p.tile_m = wrows, 1, tile_m
     return p
 
 
-def run(L, M, tile_m, y_dtype=torch.bfloat16, rows=None):
+def run(L, M, tile_m, y_dtype=torch.bfloat16, rows=None, wrows=128):
     W = to_dev(L.W)
     packed, scale, zero = spear.spear_pack_w4(W)
     x = to_dev_bf16(L.x(M))
     ws = spear.alloc_workspace(spear.spear_gemm_plan(M, L.N, L.K, 0).workspace_bytes)
-    y = spear.spear_w4ec_gemm(x, packed, scale, zero, None, y_dtype=y_dtype, plan=tc_plan(M, L.N, L.K, tile_m),
-                              workspace=ws)
+    y = spear.spear_w4ec_gemm(x, packed, scale, zero, None, y_dtype=y_dtype,
+                              plan=tc_plan(M, L.N, L.K, tile_m, wrows), workspace=ws)
     torch.cuda.synchronize()
     assert spear.spear_get_device_status(ws) == 0
     p, s, z = oracle.pack_w4(L.W)
@@ -68,14 +68,14 @@ def test_tc05_sweep_layer_without_ec(li):
     check_close(got, ref, True, f"tc05 sweep L2.{li}")
 
 
-def run_ec(L, M, tile_m, rows=None, b_g=None, y_dtype=torch.bfloat16):
+def run_ec(L, M, tile_m, rows=None, b_g=None, y_dtype=torch.bfloat16, wrows=128):
     W = to_dev(L.W)
     packed, scale, zero = spear.spear_pack_w4(W)
     x = to_dev_bf16(L.x(M))
     bg = L.b_g if b_g is None else b_g
     ec = spear.EC(to_dev_bf16(L.A_bits), to_dev_bf16(L.B_bits), to_dev_bf16(L.wg_bits), bg)
     plan = spear.spear_gemm_plan(M, L.N, L.K, L.rank)
-    plan.kernel_id, plan.tile_n, plan.split_k, plan.tile_m = spear.SPEAR_KERNEL_TC05, 128, 1, tile_m
+    plan.kernel_id, plan.tile_n, plan.split_k, plan.tile_m = spear.SPEAR_KERNEL_TC05, wrows, 1, tile_m
     ws = spear.alloc_workspace(plan.workspace_bytes + (M * L.rank * 2 + 256))
     y = spear.spear_w4ec_gemm(x, packed, scale, zero, ec, y_dtype=y_dtype, plan=plan, workspace=ws)
     torch.cuda.synchronize()
@@ -124,3 +124,29 @@ def test_tc05_ec_sweep_layer(li):
     rows = np.array([0, 100, 2049, 4095])
     got, ref, _, _ = run_ec(L, 4096, 256, rows=rows)
     check_close(got, ref, True, f"tc05 EC sweep L0.{li}")
+
+
+# 256 weight rows per tile: two 128-row sub-tiles share every x stage.
+@pytest.mark.parametrize("M", [1, 77, 300])
+def test_tc05_256rows_small(M):
+    L = make_layer("tc2", 31 + M, M, 768, 448, 0, outlier_frac=0.02, outlier_scale=10.0)
+    got, ref = run(L, M, 128, wrows=256)
+    check_close(got, ref, True, f"tc05 256 rows M={M}")
+
+
+@pytest.mark.parametrize("r", [16, 64, 128])
+@pytest.mark.parametrize("M", [128, 300])
+def test_tc05_256rows_ec_small(M, r):
+    L = make_layer("tc2ec", 41 + r + M, M, 512, 512, r, outlier_frac=0.02, outlier_scale=10.0, b_g=0.3)
+    got, ref, _, ws = run_ec(L, M, 128, wrows=256)
+    check_close(got, ref, True, f"tc05 256 rows EC M={M} r={r}")
+    assert int(ws[: (128 + 1024) * 1024].count_nonzero().item()) == 0, "EC flags not re-armed"
+
+
+def test_tc05_256rows_prefill_sampled():
+    L = config_layers(3)[0]
+    rows = np.array([0, 1, 255, 256, 1031, 2047])
+    got, ref = run(L, 2048, 128, rows=rows, wrows=256)
+    check_close(got, ref, True, "tc05 256 rows prefill")
+    got, ref, _, _ = run_ec(L, 2048, 128, rows=rows, wrows=256)
+    check_close(got, ref, True, "tc05 256 rows EC prefill")

@@ -162,9 +162,10 @@ spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K,
     if (p.kernel_id == SPEAR_KERNEL_TC05) {
         if (rank > TC05_MAX_RANK) return SPEAR_ERR_INVALID_ARG;
         if ((M + p.tile_m - 1) / p.tile_m > (int64_t)TC_BLOCKS_MAX) return SPEAR_ERR_INVALID_ARG;
-        if (p.tile_n != 128 || p.split_k != 1 ||
-            !(p.tile_m == 128 || p.tile_m == 160 || p.tile_m == 192 || p.tile_m == 256))
+        if (p.split_k != 1 || !(p.tile_m == 128 || p.tile_m == 160 || p.tile_m == 192 || p.tile_m == 256))
             return SPEAR_ERR_INVALID_ARG;
+        // 128 weight rows per tile, or 256 (two sub-tiles sharing x) with 128 tokens.
+        if (!(p.tile_n == 128 || (p.tile_n == 256 && p.tile_m == 128 && N % 256 == 0))) return SPEAR_ERR_INVALID_ARG;
         return SPEAR_OK;
     }
     if (p.kernel_id != SPEAR_KERNEL_SPLITK) return SPEAR_ERR_INVALID_ARG;
@@ -292,7 +293,7 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         t.err = ctrl;
         t.ec_ready = ctrl + TC_FLAGS_WORD;
         t.ec_consumed = t.ec_ready + TC_BLOCKS_MAX;
-        return launch_tc05(t, p.tile_m, s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
+        return launch_tc05(t, p.tile_m, p.tile_n, s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
     }
     const int nb = nb_for_tile_m(p.tile_m);
     const int g = p.tile_n / 16;

@@ -81,7 +81,8 @@ struct TcArgs {
 };
 
 // bn: tokens per tile (128 or 256).
-cudaError_t launch_tc05(const TcArgs& a, int bn, cudaStream_t stream);
+// bn = tokens per tile; rows = weight rows per tile (128, or 256 with bn = 128).
+cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream);
 
 cudaError_t launch_pack_w4(const void* W, bool w_is_bf16, int64_t N, int64_t K, void* packed, void* scale,
                            void* zero, cudaStream_t stream);

@@ -155,11 +155,12 @@ SPEAR_DEVI void named_bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory");
 // ---------------------------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------------------------
-template <int BN, int STAGES>
+template <int BN, int STAGES, int SUB>
 struct TcSmem {
     static constexpr int X_BYTES = BN * TC_BK * 2;        // bf16 x tile (or u chunk), 128-byte swizzle
     static constexpr int A_BYTES = TC_BM * TC_BK * 2;     // bf16 MN-major tile (A or B slice)
-    static constexpr int P_BYTES = TC_BM * TC_BK / 2;     // packed int4 tile
+    static constexpr int P_SUB = TC_BM * TC_BK / 2;       // packed int4 tile of 128 weight rows
+    static constexpr int P_BYTES = SUB * P_SUB;           // SUB of them per stage
     static constexpr int X_OFF = 0;
     static constexpr int A_OFF = X_OFF + STAGES * X_BYTES;
     static constexpr int P_OFF = A_OFF + STAGES * A_BYTES;
@@ -167,22 +168,24 @@ struct TcSmem {
     static constexpr int G_OFF = WG_OFF + STAGES * TC_BK * 2;            // gate values, 128 floats
     static constexpr int BAR_OFF = G_OFF + 128 * 4;
     static constexpr int TOTAL = BAR_OFF + 3 * STAGES * 8 + 16 + 16 + 1024;   // + alignment slack
-    // TMEM columns: D [0, BN); converted weight stages [BN, BN + 32 STAGES); E [BN, 2 BN) reuses
-    // the stage columns once the main K loop has retired.
-    static constexpr int NEED = BN + (STAGES * 32 > BN ? STAGES * 32 : BN);
+    // TMEM columns: D of sub-tile b at [b BN, (b + 1) BN); converted weight stages from SUB BN,
+    // 32 columns per (stage, sub-tile); E of sub-tile b at SUB BN + b BN reuses the stage columns
+    // once the main K loop has retired.
+    static constexpr int NEED = SUB * BN + (SUB * STAGES * 32 > SUB * BN ? SUB * STAGES * 32 : SUB * BN);
     static constexpr uint32_t TMEM_COLS = NEED <= 32 ? 32 : NEED <= 64 ? 64 : NEED <= 128 ? 128 : NEED <= 256 ? 256 : 512;
 };
 constexpr int TC_EB = 128;               // tokens per EC tile
 
 // Tiles: the first `ec_tiles` blocks are EC tiles (one per 128 tokens; compute u), the rest are
-// main tiles (weight tile nb, token block mb of BN tokens), token-block major.
-template <int BN, int STAGES>
+// main tiles (128 SUB weight rows, token block mb of BN tokens), token-block major.  With SUB = 2
+// the two 128-row sub-tiles share every x stage, which halves the x traffic from L2.
+template <int BN, int STAGES, int SUB>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                const __grid_constant__ CUtensorMap tmap_u, const __grid_constant__ CUtensorMap tmap_g,
                const __grid_constant__ CUtensorMap tmap_x128, TcArgs a) {
-    using L = TcSmem<BN, STAGES>;
+    using L = TcSmem<BN, STAGES, SUB>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);       // TMA landed
@@ -199,12 +202,13 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     const int ec_tiles = has_ec ? eblocks : 0;
     const bool is_ec = (int)blockIdx.x < ec_tiles;
     const int t = is_ec ? (int)blockIdx.x : (int)blockIdx.x - ec_tiles;
-    const int ntiles = (int)(a.N / TC_BM);
+    const int ntiles = (int)(a.N / (TC_BM * SUB));
     const int mb = is_ec ? t : t / ntiles;                                 // EC: 128-token block; main: BN block
-    const int64_t n0 = is_ec ? 0 : (int64_t)(t % ntiles) * TC_BM;
+    const int64_t n0 = is_ec ? 0 : (int64_t)(t % ntiles) * TC_BM * SUB;
     const int64_t m0 = (int64_t)mb * (is_ec ? TC_EB : BN);
     const int ksteps = (int)(a.K / TC_BK);
-    const int ec_chunks = (!is_ec && has_ec) ? (a.rank + 63) / 64 : 0;   // EC MMA steps of 64 columns
+    // EC MMA steps: 64 columns of u per chunk, one step per (chunk, sub-tile).
+    const int ec_chunks = (!is_ec && has_ec) ? ((a.rank + 63) / 64) * SUB : 0;
     const int rboxes = (a.rank + 63) / 64;                                 // 64-wide boxes of A per stage
     const int e_lo = (int)(m0 / TC_EB);                                    // EC blocks this main tile needs
     const int e_hi = min(eblocks, (int)((m0 + BN + TC_EB - 1) / TC_EB));
@@ -228,8 +232,8 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_d = *tmem_slot;
-    const uint32_t tmem_a = tmem_d + BN;       // converted weight stages (main K loop)
-    const uint32_t tmem_e = tmem_d + BN;       // EC accumulator (after the main K loop)
+    const uint32_t tmem_a = tmem_d + SUB * BN;   // converted weight stages (main K loop)
+    const uint32_t tmem_e = tmem_d + SUB * BN;   // EC accumulators (after the main K loop)
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -244,7 +248,9 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                     tma_load_2d(smem + L::WG_OFF + s * TC_BK * 2, &tmap_g, kt * TC_BK, 0, &full[s]);
                 } else {
                     mbar_arrive_expect_tx(&full[s], L::X_BYTES + L::P_BYTES);
-                    tma_load_2d(smem + L::P_OFF + s * L::P_BYTES, &tmap_w, kt * (TC_BK / 2), (int32_t)n0, &full[s]);
+                    for (int sb = 0; sb < SUB; ++sb)
+                        tma_load_2d(smem + L::P_OFF + s * L::P_BYTES + sb * L::P_SUB, &tmap_w, kt * (TC_BK / 2),
+                                    (int32_t)(n0 + sb * TC_BM), &full[s]);
                 }
             };
             const int pre = ksteps < STAGES ? ksteps : STAGES;
@@ -275,10 +281,11 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                     if (v >= STAGES && !mbar_wait(&empty[s], ((v / STAGES) - 1) & 1)) { atomicOr(a.err, 4u); ok = false; break; }
                     unsigned char* xs = smem + L::X_OFF + s * L::X_BYTES;
                     unsigned char* as = smem + L::A_OFF + s * L::A_BYTES;
+                    const int ch = c / SUB, nb0 = (int)n0 + (c % SUB) * TC_BM;
                     mbar_arrive_expect_tx(&full[s], L::X_BYTES + 2 * (64 * 64 * 2));
-                    tma_load_2d(xs, &tmap_u, c * 64, (int32_t)m0, &full[s]);                 // u[m, 64c ..]
-                    tma_load_2d(as, &tmap_b, (int32_t)n0, c * 64, &full[s]);                 // B[64c .., n0 .. +64]
-                    tma_load_2d(as + 64 * 64 * 2, &tmap_b, (int32_t)n0 + 64, c * 64, &full[s]);
+                    tma_load_2d(xs, &tmap_u, ch * 64, (int32_t)m0, &full[s]);                // u[m, 64ch ..]
+                    tma_load_2d(as, &tmap_b, nb0, ch * 64, &full[s]);                        // B[64ch .., nb0 .. +64]
+                    tma_load_2d(as + 64 * 64 * 2, &tmap_b, nb0 + 64, ch * 64, &full[s]);
                 }
                 // Every main tile of these tokens has seen the flags: the last one re-arms each.
                 // EC block e is read by every weight tile of each token block that overlaps it.
@@ -313,8 +320,11 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 } else {
                     constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, BN);
 #pragma unroll
-                    for (int kk = 0; kk < TC_BK / 16; ++kk)   // 16 bf16 = 8 TMEM columns = 2 descriptor units
-                        mma_bf16_ts(tmem_d, tmem_a + s * 32 + 8 * kk, bd + 2 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                    for (int sb = 0; sb < SUB; ++sb)
+#pragma unroll
+                        for (int kk = 0; kk < TC_BK / 16; ++kk)   // 16 bf16 = 8 TMEM columns = 2 descriptor units
+                            mma_bf16_ts(tmem_d + sb * BN, tmem_a + (s * SUB + sb) * 32 + 8 * kk, bd + 2 * kk, idesc,
+                                        (kt > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&empty[s]);
             }
@@ -334,7 +344,8 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 const uint64_t bd = smem_desc_k_sw128(smem + L::X_OFF + s * L::X_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tmem_e, ad + 128 * kk, bd + 2 * kk, idesc_ec, (c > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ss(tmem_e + (c % SUB) * BN, ad + 128 * kk, bd + 2 * kk, idesc_ec,
+                                (c / SUB > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&empty[s]);
             }
             mma_commit(acc_full);
@@ -346,7 +357,10 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         // 64, 96, 0, 32 (+lane).
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t zb = is_ec ? 0u : zero_bias_bf16x2((uint32_t)__half2float(a.zero[n0 + row]));
+        uint32_t zb[SUB];
+#pragma unroll
+        for (int sb = 0; sb < SUB; ++sb)
+            zb[sb] = is_ec ? 0u : zero_bias_bf16x2((uint32_t)__half2float(a.zero[n0 + sb * TC_BM + row]));
         float pg = 0.0f;                                   // EC tiles: gate pre-activation of token `row`
         bool ok = true;
         for (int kt = 0; kt < ksteps + ec_chunks; ++kt) {
@@ -368,18 +382,23 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                     }
                 }
             } else if (kt < ksteps) {
-                // 64 codes of weight row `row` -> 32 TMEM columns of bf16 pairs (q - z), natural order.
-                const uint4* prow = reinterpret_cast<const uint4*>(smem + L::P_OFF + s * L::P_BYTES + row * 32);
-                uint32_t o[32];
+                // 64 codes of weight row `row` of each sub-tile -> 32 TMEM columns of bf16 pairs
+                // (q - z), natural order.
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint4 w = prow[h];
-                    cvt_w4_pairs_natural(w.x, zb, o + 16 * h);
-                    cvt_w4_pairs_natural(w.y, zb, o + 16 * h + 4);
-                    cvt_w4_pairs_natural(w.z, zb, o + 16 * h + 8);
-                    cvt_w4_pairs_natural(w.w, zb, o + 16 * h + 12);
+                for (int sb = 0; sb < SUB; ++sb) {
+                    const uint4* prow =
+                        reinterpret_cast<const uint4*>(smem + L::P_OFF + s * L::P_BYTES + sb * L::P_SUB + row * 32);
+                    uint32_t o[32];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint4 w = prow[h];
+                        cvt_w4_pairs_natural(w.x, zb[sb], o + 16 * h);
+                        cvt_w4_pairs_natural(w.y, zb[sb], o + 16 * h + 4);
+                        cvt_w4_pairs_natural(w.z, zb[sb], o + 16 * h + 8);
+                        cvt_w4_pairs_natural(w.w, zb[sb], o + 16 * h + 12);
+                    }
+                    tmem_st32(tmem_a + lane_base + (s * SUB + sb) * 32, o);
                 }
-                tmem_st32(tmem_a + lane_base + s * 32, o);
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                 tc_fence_before();
             }
@@ -409,13 +428,14 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             named_bar_epi();
             if (row == 0 && acc_ok) asm volatile("st.release.gpu.global.u32 [%0], 1;" ::"l"(&a.ec_ready[mb]) : "memory");
         } else {
-            // y[m, n] = s[n] D[n, m] (+ E[n, m]).
-            const float sc = __half2float(a.scale[n0 + row]);
-            const int64_t n = n0 + row;
+            // y[m, n] = s[n] D[n, m] (+ E[n, m]), sub-tile by sub-tile.
+            for (int sb = 0; sb < SUB; ++sb) {
+            const float sc = __half2float(a.scale[n0 + sb * TC_BM + row]);
+            const int64_t n = n0 + sb * TC_BM + row;
             for (int c0 = 0; c0 < BN; c0 += 16) {
                 float v[16], e[16];
-                tmem_ld16(tmem_d + lane_base + (uint32_t)c0, v);
-                if (has_ec) tmem_ld16(tmem_e + lane_base + (uint32_t)c0, e);
+                tmem_ld16(tmem_d + (uint32_t)(sb * BN) + lane_base + (uint32_t)c0, v);
+                if (has_ec) tmem_ld16(tmem_e + (uint32_t)(sb * BN) + lane_base + (uint32_t)c0, e);
                 if (!acc_ok) continue;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -428,6 +448,7 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                             reinterpret_cast<__nv_bfloat16*>(a.y)[m * a.N + n] = __float2bfloat16_rn(yv);
                     }
                 }
+            }
             }
         }
     }
@@ -475,9 +496,9 @@ static bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int SUB>
 static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
-    using L = TcSmem<BN, STAGES>;
+    using L = TcSmem<BN, STAGES, SUB>;
     CUtensorMap mx, mw, ma, mb, mu, mg, mx128;
     if (!make_map_2d(&mx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.K, (uint64_t)a.M, TC_BK, BN,
                      CU_TENSOR_MAP_SWIZZLE_128B))
@@ -507,14 +528,14 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !opted[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(w4_tc05_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(w4_tc05_kernel<BN, STAGES, SUB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              L::TOTAL);
         if (e != cudaSuccess) return e;
         opted[dev] = true;
     }
     const unsigned mblocks = (unsigned)((a.M + BN - 1) / BN);
     const unsigned eblocks = (unsigned)((a.M + TC_EB - 1) / TC_EB);
-    const unsigned tiles = (unsigned)(a.N / TC_BM) * mblocks + (has_ec ? eblocks : 0u);
+    const unsigned tiles = (unsigned)(a.N / (TC_BM * SUB)) * mblocks + (has_ec ? eblocks : 0u);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles);
     cfg.blockDim = dim3(TC_THREADS);
@@ -525,14 +546,16 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, w4_tc05_kernel<BN, STAGES>, mx, mw, ma, mb, mu, mg, mx128, a);
+    return cudaLaunchKernelEx(&cfg, w4_tc05_kernel<BN, STAGES, SUB>, mx, mw, ma, mb, mu, mg, mx128, a);
 }
 
-cudaError_t launch_tc05(const TcArgs& a, int bn, cudaStream_t stream) {
-    if (bn == 128) return launch_tc_t<128, 4>(a, stream);
-    if (bn == 160) return launch_tc_t<160, 4>(a, stream);
-    if (bn == 192) return launch_tc_t<192, 3>(a, stream);
-    if (bn == 256) return launch_tc_t<256, 3>(a, stream);
+cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream) {
+    if (rows == 256) return bn == 128 ? launch_tc_t<128, 4, 2>(a, stream) : cudaErrorInvalidValue;
+    if (rows != 128) return cudaErrorInvalidValue;
+    if (bn == 128) return launch_tc_t<128, 6, 1>(a, stream);
+    if (bn == 160) return launch_tc_t<160, 4, 1>(a, stream);
+    if (bn == 192) return launch_tc_t<192, 3, 1>(a, stream);
+    if (bn == 256) return launch_tc_t<256, 4, 1>(a, stream);
     return cudaErrorInvalidValue;
 }
 
