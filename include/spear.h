@@ -61,8 +61,8 @@ typedef enum { SPEAR_BF16 = 0, SPEAR_FP32 = 1 } spear_dtype;
 /* Kernel families the dispatcher chooses from (section 2.2A's two phases). */
 typedef enum {
     SPEAR_KERNEL_AUTO = 0,      /* let spear_gemm_plan decide */
-    SPEAR_KERNEL_SPLITK = 1,    /* decode: split-K weight-streaming kernel (mma.sync on registers) plus
-                                   a separate EC pass, overlapped by programmatic dependent launch */
+    SPEAR_KERNEL_SPLITK = 1,    /* decode: split-K weight-streaming kernel (mma.sync on registers); EC
+                                   CTAs of the same launch reduce x A through int64 accumulators */
     SPEAR_KERNEL_TC05 = 2       /* prefill: TMA + tcgen05/TMEM kernel, EC applied in its epilogue */
 } spear_kernel;
 
@@ -82,7 +82,7 @@ typedef struct {
 typedef struct {
     int32_t kernel_id;        /* spear_kernel */
     int32_t tile_n;           /* weight rows per CTA */
-    int32_t split_k;          /* number of K slices reduced in the workspace (1 = none) */
+    int32_t split_k;          /* number of K slices (1 = none), reduced in a thread-block cluster */
     int32_t tile_m;           /* token rows per CTA (or per launch chunk) */
     int32_t flags;            /* reserved, 0 */
     int32_t reserved;
