@@ -133,3 +133,10 @@ def test_pack_and_unpack_host_checks():
     assert lib.spear_debug_unpack_w4(P(0x1000), P(0x2000), 8, 8, P(0), P(0), None) == INVALID
     assert lib.spear_debug_unpack_w4(P(0x1000), P(0x2000), 8, 9, P(0x3000), P(0), None) == SHAPE
     assert lib.spear_get_device_status(P(0), 0, None) == INVALID
+
+
+def test_prepared_layer_rejects_host_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        spear.W4ECLayer(torch.zeros((128, 32), dtype=torch.uint8), torch.zeros(128, dtype=torch.float16),
+                        torch.zeros(128, dtype=torch.float16))

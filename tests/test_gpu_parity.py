@@ -223,3 +223,26 @@ def test_empty_batch():
     x = torch.empty((0, d.L.K), dtype=torch.bfloat16, device="cuda")
     y = spear.spear_w4ec_gemm(x, d.packed, d.scale, d.zero, d.ec)
     assert y.shape == (0, d.L.N)
+
+
+# ----------------------------------------------------------------------------- prepared layer
+
+def test_prepared_layer_matches_call():
+    # W4ECLayer binds the weights once; its calls equal spear_w4ec_gemm's bit for bit.
+    d = dev_layer(1)
+    lay = spear.W4ECLayer(d.packed, d.scale, d.zero, d.ec)
+    stream = torch.cuda.Stream()
+    for M in (1, 4, 16, 1):
+        x = to_dev_bf16(d.L.x(M))
+        y = torch.empty((M, d.L.N), dtype=torch.bfloat16, device="cuda")
+        lay(x, y=y, stream=stream)
+        stream.synchronize()
+        assert torch.equal(y, d.run(M))
+    assert spear.spear_get_device_status(lay.workspace) == 0
+    x = to_dev_bf16(d.L.x(4))
+    with pytest.raises(ValueError):
+        lay(x.cpu())                                              # activations on the host
+    with pytest.raises(ValueError):
+        lay(x, y=torch.empty((4, d.L.N), dtype=torch.float32, device="cuda"))   # wrong output dtype
+    with pytest.raises(ValueError):
+        lay(x[:, :128].contiguous())                              # wrong K

@@ -215,6 +215,71 @@ def spear_w4ec_gemm_noalloc(x: torch.Tensor, packed: torch.Tensor, scale: torch.
     return y
 
 
+class W4ECLayer:
+    """One quantised layer bound once, called many times: y = x dequant(Wq)^T + g(x) (x A) B.
+
+    Checks and converts the weight-side arguments (packed weights, scales, zero-points and the
+    compensator) once, keeps one workspace and a plan per batch size, so that a call marshals
+    only x, y and the stream into one spear_w4ec_gemm call.  The tensors must stay alive and
+    unchanged while the layer is used.  Calls that share the layer's workspace must be ordered
+    on one stream; the first call with a new batch size may replace the workspace by a larger
+    one (plan() every size up front to avoid that).
+    """
+
+    def __init__(self, packed: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor, ec: Optional[EC] = None,
+                 y_dtype=torch.bfloat16):
+        for name, t in (("packed", packed), ("scale", scale), ("zero", zero)):
+            _dev(t, name)
+        self.N, self.K = int(packed.shape[0]), int(packed.shape[1]) * 2
+        self.device = packed.device
+        self._index = packed.get_device()
+        self.y_dtype = y_dtype
+        self._yd = SPEAR_FP32 if y_dtype == torch.float32 else SPEAR_BF16
+        self.rank = ec.rank if ec is not None else 0
+        self._keep = (packed, scale, zero, ec)
+        self._ec_c = ec.as_c() if ec is not None else None
+        self._ec_ref = ctypes.byref(self._ec_c) if ec is not None else None
+        self._w = (packed.data_ptr(), scale.data_ptr(), zero.data_ptr())
+        self._plans = {}
+        self._ws = None
+
+    def plan(self, M: int) -> spear_plan:
+        p = self._plans.get(M)
+        if p is None:
+            p = spear_gemm_plan(M, self.N, self.K, self.rank, self.device.index)
+            if self._ws is None or self._ws.numel() < p.workspace_bytes:
+                self._ws = alloc_workspace(p.workspace_bytes, self.device)
+            self._plans[M] = (p, ctypes.byref(p))
+            return p
+        return p[0]
+
+    @property
+    def workspace(self) -> torch.Tensor:
+        return self._ws
+
+    def __call__(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        M = int(x.shape[0])
+        entry = self._plans.get(M)
+        if entry is None:
+            self.plan(M)
+            entry = self._plans[M]
+        if (x.dtype != torch.bfloat16 or x.get_device() != self._index or not x.is_contiguous()
+                or x.dim() != 2 or x.shape[1] != self.K):
+            raise ValueError("x must be a contiguous bf16 [M, K] tensor on the layer's device")
+        if y is None:
+            y = torch.empty((M, self.N), dtype=self.y_dtype, device=self.device)
+        elif (y.dtype != self.y_dtype or y.get_device() != self._index or not y.is_contiguous()
+              or tuple(y.shape) != (M, self.N)):
+            raise ValueError("y must be a contiguous [M, N] tensor of the layer's output dtype on its device")
+        sh = stream.cuda_stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        ws = self._ws
+        st = _lib.spear_w4ec_gemm(entry[1], x.data_ptr(), M, self.N, self.K, self._w[0], self._w[1], self._w[2],
+                                  self._ec_ref, y.data_ptr(), self._yd, ws.data_ptr(), ws.numel(), sh)
+        if st != SPEAR_OK:
+            raise SpearError("spear_w4ec_gemm", st)
+        return y
+
+
 def spear_get_device_status(workspace: torch.Tensor, clear: bool = True, stream=None) -> int:
     return int(_lib.spear_get_device_status(_p(workspace), int(clear), _stream(stream)))
 
