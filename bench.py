@@ -487,13 +487,18 @@ def sweep_plans(args):
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         base = spear.spear_gemm_plan(M, N, K, r)
         # Room for the tcgen05 kernel's u buffer (bf16 [M, r]) whatever the default plan is.
-        ws = spear.alloc_workspace(base.workspace_bytes + (M * r * 2 + 255) // 256 * 256)
-        candidates = [(1, tile_n, split) for tile_n in (16, 32, 64, 128) for split in (1, 2, 4, 8)]
-        candidates.append((2, 128, 1))          # the tcgen05 kernel, 128-token tiles
-        for kernel_id, tile_n, split in candidates:
+        ws = spear.alloc_workspace(base.workspace_bytes + (M * r * 2 + 255) // 256 * 256 + min(M, 256) * N * 4)
+        # (kernel, tile_n, split_k, flags): every split-K decode tiling, fused and with the separate
+        # EC pass, and the tcgen05 kernel with 128-token tiles.
+        candidates = [(1, tile_n, split, fl) for tile_n in (16, 32, 64, 128) for split in (1, 2, 4, 8)
+                      for fl in (0, 1)]
+        candidates.append((2, 128, 1, 0))
+        for kernel_id, tile_n, split, fl in candidates:
                 for use_ec in (True, False):
+                    if fl and not use_ec:
+                        continue
                     plan = spear.spear_plan.from_buffer_copy(base)
-                    plan.kernel_id, plan.tile_n, plan.split_k = kernel_id, tile_n, split
+                    plan.kernel_id, plan.tile_n, plan.split_k, plan.flags = kernel_id, tile_n, split, fl
                     if kernel_id == 2:
                         plan.tile_m = 128
                     elif base.kernel_id == 2:
@@ -525,7 +530,8 @@ def sweep_plans(args):
                         e1.synchronize()
                         best = min(best, e0.elapsed_time(e1) * 1e3 / n_calls)
                     del g
-                    rows.append({"M": M, "N": N, "K": K, "rank": r if use_ec else 0, "kernel": kernel_id, "tile_n": tile_n,
+                    rows.append({"M": M, "N": N, "K": K, "rank": r if use_ec else 0, "kernel": kernel_id, "flags": fl,
+                                 "tile_n": tile_n,
                                  "split_k": split, "us": best,
                                  "GBps": layer_bytes(M, N, K, r if use_ec else 0) / best / 1e3})
     print(json.dumps({"workload": args.workload, "sweep": rows}))

@@ -66,6 +66,16 @@ typedef enum {
     SPEAR_KERNEL_TC05 = 2       /* prefill: TMA + tcgen05/TMEM kernel, EC applied in its epilogue */
 } spear_kernel;
 
+/* spear_plan.flags bits. */
+enum {
+    /* Split-K decode kernel only: the weight-streaming CTAs write their fp32 main term to the
+     * workspace and a second kernel, chained by programmatic dependent launch, applies the
+     * compensator (section 2.2A's "split-K kernel with a separate EC pass").  It spares the
+     * weight-streaming CTAs the wait for the compensator, which matters when their grid takes
+     * several waves. */
+    SPEAR_PLAN_SEPARATE_EC = 1
+};
+
 /* Error compensator of one layer.  Pass NULL for a layer without EC (section
  * 2.1B: compensators sit only at the selected, error-sensitive modules). */
 typedef struct {
@@ -84,7 +94,7 @@ typedef struct {
     int32_t tile_n;           /* weight rows per CTA */
     int32_t split_k;          /* number of K slices (1 = none), reduced in a thread-block cluster */
     int32_t tile_m;           /* token rows per CTA (or per launch chunk) */
-    int32_t flags;            /* reserved, 0 */
+    int32_t flags;            /* SPEAR_PLAN_* bits; 0 = none */
     int32_t reserved;
     size_t workspace_bytes;   /* minimum workspace for this (M, N, K, rank) */
 } spear_plan;

@@ -116,6 +116,13 @@ def test_gemm_rejects_bad_plans():
         setattr(q, field, val)
         assert _gemm(plan=ctypes.byref(q)) == INVALID, field
     # tcgen05 plans: 256 weight rows only with 128-token tiles; token widths 128, 160, 192, 256.
+    # Plan flags: only SPEAR_PLAN_SEPARATE_EC (1), and only on the split-K decode kernel.
+    for kid, fl in ((1, 2), (1, 3), (2, 1)):
+        q = spear.spear_plan.from_buffer_copy(p)
+        q.kernel_id, q.flags = kid, fl
+        if kid == 2:
+            q.tile_n, q.split_k, q.tile_m = 128, 1, 128
+        assert _gemm(plan=ctypes.byref(q)) == INVALID, (kid, fl)
     for tile_n, tile_m in ((256, 256), (256, 160), (64, 128), (128, 144)):
         q = spear.spear_plan.from_buffer_copy(p)
         q.kernel_id, q.split_k, q.tile_n, q.tile_m = 2, 1, tile_n, tile_m

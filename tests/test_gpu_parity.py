@@ -246,3 +246,52 @@ def test_prepared_layer_matches_call():
         lay(x, y=torch.empty((4, d.L.N), dtype=torch.float32, device="cuda"))   # wrong output dtype
     with pytest.raises(ValueError):
         lay(x[:, :128].contiguous())                              # wrong K
+
+
+# ----------------------------------------------------------------------------- separate EC pass
+
+@pytest.mark.parametrize("idx,M", [(1, 1), (1, 4), (1, 16), (2, 8), (0, 4)])
+def test_separate_ec_pass(idx, M):
+    # Plan flag SPEAR_PLAN_SEPARATE_EC: the weight-streaming CTAs write fp32 main terms and a second
+    # kernel applies the compensator.  Twice in a row on one workspace (the accumulators re-arm).
+    d = dev_layer(idx)
+    L = d.L
+    ref = d.oracle_y(M)
+    plan = spear.spear_gemm_plan(M, L.N, L.K, L.rank)
+    if plan.kernel_id != spear.SPEAR_KERNEL_SPLITK:
+        pytest.skip("not a split-K decode plan")
+    plan.flags = spear.SPEAR_PLAN_SEPARATE_EC
+    ws = spear.alloc_workspace((1 << 21) + min(M, 256) * L.N * 4)
+    for _ in range(2):
+        check_close(host_f64(d.run(M, plan=plan, workspace=ws)), ref, True, f"separate EC {L.name} M={M}")
+    assert spear.spear_get_device_status(ws) == 0
+    assert int(ws[: (128 + 1024) * 1024].count_nonzero().item()) == 0, "accumulators not re-armed"
+
+
+@pytest.mark.parametrize("M", [23, 300])
+def test_separate_ec_pass_ragged(M):
+    L = make_layer("sep", 71 + M, M, 384, 1024, 32, outlier_frac=0.01, outlier_scale=20.0, b_g=0.3)
+    d = Dev(L)
+    plan = spear.spear_gemm_plan(M, L.N, L.K, L.rank)
+    plan.kernel_id, plan.tile_n, plan.split_k, plan.tile_m = spear.SPEAR_KERNEL_SPLITK, 32, 2, 16
+    plan.flags = spear.SPEAR_PLAN_SEPARATE_EC
+    ws = spear.alloc_workspace((1 << 21) + min(M, 256) * L.N * 4)
+    check_close(host_f64(d.run(M, plan=plan, workspace=ws)), d.oracle_y(M), True, f"separate EC M={M}")
+    assert spear.spear_get_device_status(ws) == 0
+    assert int(ws[: (128 + 1024) * 1024].count_nonzero().item()) == 0
+
+
+def test_separate_ec_pass_gate_off():
+    # g = 0 exactly: the applied term adds zeros, so y equals the plain layer within the tolerance
+    # and the fp32 debug output equals the fused kernel's plain result exactly.
+    L = make_layer("sepg", 5, 8, 512, 1024, 64)
+    d = Dev(L)
+    plan = spear.spear_gemm_plan(8, L.N, L.K, L.rank)
+    plan.flags = spear.SPEAR_PLAN_SEPARATE_EC
+    ws = spear.alloc_workspace((1 << 21) + 8 * L.N * 4)
+    ec_off = spear.EC(d.ec.A, d.ec.B, d.ec.w_g, float("-inf"))
+    y_off = d.run(8, plan=plan, workspace=ws, ec=ec_off, y_dtype=torch.float32)
+    plain_plan = spear.spear_plan.from_buffer_copy(plan)
+    plain_plan.flags = 0
+    y_plain = d.run(8, plan=plain_plan, workspace=spear.alloc_workspace(1 << 21), ec=None, y_dtype=torch.float32)
+    assert torch.equal(y_off, y_plain)

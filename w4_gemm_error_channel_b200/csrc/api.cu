@@ -51,9 +51,11 @@ int ec_jr_for(int32_t rank, int64_t S) {
 }
 // Workspace: the zeroed prefix (control block + EC accumulators); split-K partial sums meet in
 // distributed shared memory.  The prefill kernel with a compensator also keeps u (bf16 [M][r]).
-size_t workspace_bytes_for(const spear_plan& p, int64_t M, int32_t rank) {
+size_t workspace_bytes_for(const spear_plan& p, int64_t M, int64_t N_for_ws, int32_t rank) {
     size_t b = ZEROED_BYTES;
     if (p.kernel_id == SPEAR_KERNEL_TC05 && rank > 0) b += ((size_t)M * rank * 2 + 255) / 256 * 256;
+    if (p.kernel_id == SPEAR_KERNEL_SPLITK && (p.flags & SPEAR_PLAN_SEPARATE_EC) && rank > 0)
+        b += (size_t)(M < LAUNCH_TOKENS_MAX ? M : LAUNCH_TOKENS_MAX) * N_for_ws * 4;   // fp32 main term
     return b;
 }
 
@@ -64,7 +66,7 @@ size_t workspace_bytes_for(const spear_plan& p, int64_t M, int32_t rank) {
 // Measured plans (plans/gen_table.py): the fastest tiling per swept shape on one B200.
 struct MeasuredPlan {
     int64_t M, N, K;
-    int has_ec, kernel_id, tile_n, split_k;
+    int has_ec, kernel_id, tile_n, split_k, flags;
     double us;
 };
 spear_status plan_tc05(int64_t M, int64_t N, int sms, spear_plan* p);
@@ -88,7 +90,7 @@ bool lookup_measured(int64_t M, int64_t N, int64_t K, int has_ec, int sms, spear
     p->tile_n = best->tile_n;
     p->split_k = best->split_k;
     p->tile_m = 8 * nb;
-    p->flags = 0;
+    p->flags = has_ec ? (best->flags & SPEAR_PLAN_SEPARATE_EC) : 0;
     p->reserved = 0;
     return true;
 }
@@ -160,7 +162,7 @@ bool use_tc05(int64_t M, int32_t rank) { return M >= TC05_MIN_M && rank <= TC05_
 spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K, int32_t rank) {
     (void)M;
     if (p.kernel_id == SPEAR_KERNEL_TC05) {
-        if (rank > TC05_MAX_RANK) return SPEAR_ERR_INVALID_ARG;
+        if (rank > TC05_MAX_RANK || p.flags != 0) return SPEAR_ERR_INVALID_ARG;
         if ((M + p.tile_m - 1) / p.tile_m > (int64_t)TC_BLOCKS_MAX) return SPEAR_ERR_INVALID_ARG;
         if (p.split_k != 1 || !(p.tile_m == 128 || p.tile_m == 160 || p.tile_m == 192 || p.tile_m == 256))
             return SPEAR_ERR_INVALID_ARG;
@@ -169,6 +171,7 @@ spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K,
         return SPEAR_OK;
     }
     if (p.kernel_id != SPEAR_KERNEL_SPLITK) return SPEAR_ERR_INVALID_ARG;
+    if (p.flags & ~SPEAR_PLAN_SEPARATE_EC) return SPEAR_ERR_INVALID_ARG;
     if (!(p.split_k == 1 || p.split_k == 2 || p.split_k == 4 || p.split_k == 8)) return SPEAR_ERR_INVALID_ARG;
     const int nb = nb_for_tile_m(p.tile_m);
     if (p.tile_m != 8 * nb) return SPEAR_ERR_INVALID_ARG;
@@ -233,7 +236,7 @@ spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int 
     if (use_tc05(M, rank)) st = plan_tc05(M, N, sms, &p);
     else st = plan_decode(M > 0 ? M : 1, N, K, rank, sms, &p);
     if (st != SPEAR_OK) return st;
-    p.workspace_bytes = workspace_bytes_for(p, M, rank);
+    p.workspace_bytes = workspace_bytes_for(p, M, N, rank);
     *out = p;
     return SPEAR_OK;
 }
@@ -268,7 +271,7 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
     }
     st = validate_plan(p, M, N, K, rank);
     if (st != SPEAR_OK) return st;
-    if (workspace_bytes < workspace_bytes_for(p, M, rank)) return SPEAR_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace_bytes < workspace_bytes_for(p, M, N, rank)) return SPEAR_ERR_WORKSPACE_TOO_SMALL;
 
     cudaStream_t s = (cudaStream_t)stream;
     unsigned char* ws = (unsigned char*)workspace;
@@ -320,6 +323,8 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
     a.arrivals = ctrl + CTRL_HEADER_WORDS;
     a.consumed = a.arrivals + CHUNKS_MAX;
     a.consumed1 = a.consumed + CHUNKS_MAX;
+    const bool separate = rank > 0 && (p.flags & SPEAR_PLAN_SEPARATE_EC);
+    a.ymain = separate ? (float*)(ws + ZEROED_BYTES) : nullptr;
     const size_t ysz = y_dtype == SPEAR_FP32 ? 4 : 2;
     // Launches of at most LAUNCH_TOKENS_MAX tokens, in token order on one stream.
     for (int64_t m0 = 0; m0 < M; m0 += LAUNCH_TOKENS_MAX) {
@@ -331,6 +336,7 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         const int e = a.ec_splits * a.mchunks;
         a.ec_ctas = (e + p.split_k - 1) / p.split_k * p.split_k;
         if (launch_decode(a, nb, g, wpw_for(a.k_slice), s) != cudaSuccess) return SPEAR_ERR_CUDA;
+        if (separate && launch_apply(a, s) != cudaSuccess) return SPEAR_ERR_CUDA;
     }
     return SPEAR_OK;
 }

@@ -257,7 +257,9 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
     const int64_t kbeg = (int64_t)ks * a.k_slice;
     const int64_t kend = imin64(kbeg + a.k_slice, a.K);
     const int64_t row_bytes = a.K / 2;
-    const bool has_ec = a.rank > 0;
+    // With a separate EC pass the CTA writes its fp32 main term to the workspace and leaves the
+    // compensator to the apply kernel.
+    const bool has_ec = a.rank > 0 && a.ymain == nullptr;
     const int j0 = ks * a.ec_jr;
     const int nj = has_ec ? max(0, min(a.rank, j0 + a.ec_jr) - j0) : 0;
 
@@ -492,7 +494,9 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
     }
 
     auto store4 = [&](int64_t m, int r4, float4 o) {
-        if (a.y_fp32) {
+        if (a.ymain != nullptr) {
+            reinterpret_cast<float4*>(a.ymain + m * a.N + n0)[r4] = o;
+        } else if (a.y_fp32) {
             reinterpret_cast<float4*>(reinterpret_cast<float*>(a.y) + m * a.N + n0)[r4] = o;
         } else {
             const __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y), hi = __floats2bfloat162_rn(o.z, o.w);
@@ -588,6 +592,119 @@ __global__ void __launch_bounds__(DK_THREADS, 4) w4ec_decode_kernel(DecodeArgs a
     const int ks = bid % a.split;          // = the rank within the cluster
     const int rest = bid / a.split;
     gemm_role<NB, G, WPW>(a, rest % a.row_tiles, ks, rest / a.row_tiles, dyn_smem);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Separate EC pass (apply kernel).  Launched right after the decode kernel with programmatic
+// dependent launch, so its wait returns once every EC and GEMM CTA of that launch is complete:
+// the accumulators and the fp32 main term are final and need no polling.  CTA b takes 128 output
+// rows (thread i <-> row 128 b + i) and every token of the launch:
+//   u[m, j] = sigmoid(p[m] + b_g) t[m, j]          (from the accumulator words, in shared memory)
+//   y[m, n] = main[m, n] + sum_j u[m, j] B[j, n]   (B tile prefetched before the wait)
+// The last CTA to finish clears the accumulators for the next call.
+// ---------------------------------------------------------------------------------------------
+constexpr int AP_ROWS = 128;
+constexpr int AP_TOK = 16;              // tokens per pass over u
+
+__global__ void __launch_bounds__(AP_ROWS) w4ec_apply_kernel(DecodeArgs a) {
+    extern __shared__ __align__(16) unsigned char dyn_smem[];
+    const int r = a.rank;
+    uint16_t* Bs = reinterpret_cast<uint16_t*>(dyn_smem);                          // [r][AP_ROWS]
+    float* us = reinterpret_cast<float*>(dyn_smem + (size_t)r * AP_ROWS * 2);      // [AP_TOK][r]
+    __shared__ unsigned s_last;
+    const int64_t n0 = (int64_t)blockIdx.x * AP_ROWS;
+    const int64_t n = n0 + threadIdx.x;
+    constexpr int CH = AP_ROWS / 8;
+    for (int c = threadIdx.x; c < r * CH; c += AP_ROWS) {
+        const int jj = c / CH, cc = c % CH;
+        cp_async_16(Bs + jj * AP_ROWS + cc * 8, a.B + (int64_t)jj * a.N + n0 + cc * 8);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+
+    pdl_wait_primary();
+    asm volatile("cp.async.wait_all;" ::: "memory");
+
+    for (int64_t mb = 0; mb < a.M; mb += AP_TOK) {
+        const int tk = (int)imin64(AP_TOK, a.M - mb);
+        __syncthreads();                          // the previous pass is done with us
+        // u of these tokens: all loads of a thread's elements in flight together.
+        constexpr int UB = (AP_TOK * 256 + AP_ROWS - 1) / AP_ROWS;   // ranks up to 256
+        long long tv[UB], pv[UB];
+#pragma unroll
+        for (int u = 0; u < UB; ++u) {
+            const int c = threadIdx.x + u * AP_ROWS;
+            const int mm = c / r, j = c % r;
+            const bool ok = c < tk * r;
+            const long long* row = a.tacc + (mb + (ok ? mm : 0)) * (int64_t)(r + 1);
+            tv[u] = ok ? __ldcg(row + j) : 0ll;
+            pv[u] = ok ? __ldcg(row + r) : 0ll;
+        }
+#pragma unroll
+        for (int u = 0; u < UB; ++u) {
+            const int c = threadIdx.x + u * AP_ROWS;
+            if (c < tk * r) {
+                const float t_ = __ll2float_rn(tv[u] >> FIX_COUNT_BITS) * (1.0f / FIX_ONE);
+                const float p_ = __ll2float_rn(pv[u] >> FIX_COUNT_BITS) * (1.0f / FIX_ONE);
+                us[c] = t_ / (1.0f + expf(-(p_ + a.b_g)));
+            }
+        }
+        float mv[AP_TOK];
+#pragma unroll
+        for (int mm = 0; mm < AP_TOK; ++mm) mv[mm] = mm < tk ? __ldcg(a.ymain + (mb + mm) * a.N + n) : 0.0f;
+        __syncthreads();
+#pragma unroll
+        for (int mm = 0; mm < AP_TOK; ++mm) {
+            if (mm >= tk) break;
+            const int64_t m = mb + mm;
+            float v = mv[mm];
+            const float* ur = us + mm * r;
+#pragma unroll 8
+            for (int j = 0; j < r; ++j) v = fmaf(ur[j], bf16_bits_to_f32(Bs[j * AP_ROWS + threadIdx.x]), v);
+            if (a.y_fp32)
+                reinterpret_cast<float*>(a.y)[m * a.N + n] = v;
+            else
+                reinterpret_cast<__nv_bfloat16*>(a.y)[m * a.N + n] = __float2bfloat16_rn(v);
+        }
+    }
+    pdl_launch_dependents();
+
+    // Every CTA has read the accumulators before its acq_rel count; the last one clears them.
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned prev;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(a.consumed) : "memory");
+        s_last = (prev == gridDim.x - 1) ? 1u : 0u;
+    }
+    __syncthreads();
+    if (s_last) {
+        for (int64_t c = threadIdx.x; c < a.M * (int64_t)(r + 1); c += AP_ROWS) a.tacc[c] = 0ll;
+        if (threadIdx.x == 0) *a.consumed = 0u;
+    }
+}
+
+size_t apply_dyn_smem_bytes(int rank) { return (size_t)rank * AP_ROWS * 2 + (size_t)AP_TOK * rank * 4; }
+
+cudaError_t launch_apply(const DecodeArgs& a, cudaStream_t stream) {
+    const size_t dyn = apply_dyn_smem_bytes(a.rank);
+    static size_t opted[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dyn > 48 * 1024 && dev >= 0 && dev < 64 && dyn > opted[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(w4ec_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+        if (e != cudaSuccess) return e;
+        opted[dev] = dyn;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.N / AP_ROWS));
+    cfg.blockDim = dim3(AP_ROWS);
+    cfg.dynamicSmemBytes = dyn;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, w4ec_apply_kernel, a);
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -58,6 +58,7 @@ struct DecodeArgs {
     unsigned* arrivals;     // [mchunks]
     unsigned* consumed;     // [mchunks] level-2 consumer counters
     unsigned* consumed1;    // [mchunks][GROUPS_MAX] level-1 consumer counters
+    float* ymain;           // separate EC pass: fp32 main term [M][N] (workspace); null when fused
 };
 
 // Prefill (tcgen05) kernel arguments.
@@ -95,6 +96,9 @@ bool decode_config_supported(int nb, int g, int wpw);
 // Largest K with a compensator: the decode kernel counts K slices of 512 rows in 8 bits.
 constexpr int64_t EC_K_MAX = 65536;
 int decode_ec_ctas_per_chunk(int64_t K, int rank);
+// Separate EC pass after the decode kernel (it reads DecodeArgs::ymain, tacc, B).
+cudaError_t launch_apply(const DecodeArgs& a, cudaStream_t stream);
+size_t apply_dyn_smem_bytes(int rank);
 size_t decode_dyn_smem_bytes(int nb, int g, int ec_jr, int rank);
 cudaError_t launch_decode(const DecodeArgs& a, int nb, int g, int wpw, cudaStream_t stream);
 

@@ -79,7 +79,7 @@ extern "C" spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const vo
         return SPEAR_ERR_INVALID_ARG;
     }
     // Only the weight-streaming decode kernel runs here.
-    if (p.kernel_id != SPEAR_KERNEL_SPLITK) return SPEAR_ERR_INVALID_ARG;
+    if (p.kernel_id != SPEAR_KERNEL_SPLITK || p.flags != 0) return SPEAR_ERR_INVALID_ARG;
     if (!(p.split_k == 1 || p.split_k == 2 || p.split_k == 4 || p.split_k == 8)) return SPEAR_ERR_INVALID_ARG;
     const int nb = nb_of(p.tile_m);
     if (p.tile_m != 8 * nb || p.tile_n <= 0 || p.tile_n % 16 != 0 || N % p.tile_n != 0) return SPEAR_ERR_INVALID_ARG;
@@ -124,5 +124,6 @@ extern "C" spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const vo
     a.arrivals = ctrl + CTRL_HEADER_WORDS;
     a.consumed = a.arrivals + CHUNKS_MAX;
     a.consumed1 = a.consumed + CHUNKS_MAX;
+    a.ymain = nullptr;                                    // the compensator stays fused here
     return launch_decode(a, nb, p.tile_n / 16, wpw_of(ksl), s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
 }
