@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--once", type=int, default=0, metavar="M",
                     help="run 5 layer calls of the workload with M tokens and exit (for profilers)")
     ap.add_argument("--no-ec", action="store_true", help="with --once: the plain W4 layer")
+    ap.add_argument("--svd-demo", action="store_true",
+                    help="static SVD-initialised compensator on the workload's layer: share of the 4-bit "
+                         "output error removed and time per call, for several ranks")
     return ap.parse_args()
 
 
@@ -560,8 +563,64 @@ def run_once(args):
                       "device_status": spear.spear_get_device_status(ws)}))
 
 
+def svd_demo(args):
+    """Static SVD-initialised compensator (gate held at 1) on the workload's layer, M = its largest
+    decode batch: the share of the 4-bit layer's output error it removes against fp64 x W^T, and
+    its device time per call in a chained CUDA graph, for ranks 16..128."""
+    import torch
+    import w4_gemm_error_channel_b200 as spear
+    from w4_gemm_error_channel_b200.svd_init import svd_compensator
+    from oracle import svd_ec
+    from synthetic import config_layers, f32_from_bf16_bits
+    torch.cuda.set_device(0)
+    cfg, batches, kind = WORKLOADS[args.workload]
+    M = max(b for b in batches if b <= 64)
+    L = config_layers(cfg, M=M)[0]
+    dev = torch.device("cuda")
+    W = torch.from_numpy(L.W).to(dev)
+    packed, scale, zero = spear.spear_pack_w4(W)
+    x = torch.from_numpy(L.x(M).view(np.int16)).to(dev).view(torch.bfloat16)
+    xf = f32_from_bf16_bits(L.x(M)).astype(np.float64)
+    y_fp = xf @ L.W.astype(np.float64).T
+    stream = torch.cuda.Stream()
+
+    def timed(ec):
+        lay = spear.W4ECLayer(packed, scale, zero, ec, y_dtype=torch.float32)
+        y = lay(x, stream=stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(32):
+                    lay(x, y=y, stream=stream)
+        best = 1e9
+        for _ in range(5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1) * 1e3 / 32)
+        del g
+        return y.double().cpu().numpy(), best
+
+    y_w4, t_w4 = timed(None)
+    rows = [{"rank": 0, "gap_recovered": 0.0, "us": t_w4}]
+    for r in (16, 32, 64, 128):
+        ec = svd_compensator(W, packed, scale, zero, r)
+        y, t = timed(ec)
+        rows.append({"rank": r, "gap_recovered": svd_ec.gap_recovered(y, y_fp, y_w4), "us": t})
+    print(json.dumps({"svd_demo": {"workload": f"{args.workload}: M={M}, N={L.N}, K={L.K}, synthetic",
+                                   "error": "|y - x W^T|_F relative to the plain 4-bit layer's",
+                                   "ranks": rows}}))
+
+
 def main():
     args = parse()
+    if args.svd_demo:
+        svd_demo(args)
+        return
     if args.once:
         run_once(args)
         return
