@@ -570,7 +570,6 @@ def svd_demo(args):
     import torch
     import w4_gemm_error_channel_b200 as spear
     from w4_gemm_error_channel_b200.svd_init import svd_compensator
-    from oracle import svd_ec
     from synthetic import config_layers, f32_from_bf16_bits
     torch.cuda.set_device(0)
     cfg, batches, kind = WORKLOADS[args.workload]
@@ -610,7 +609,8 @@ def svd_demo(args):
     for r in (16, 32, 64, 128):
         ec = svd_compensator(W, packed, scale, zero, r)
         y, t = timed(ec)
-        rows.append({"rank": r, "gap_recovered": svd_ec.gap_recovered(y, y_fp, y_w4), "us": t})
+        removed = 1.0 - float(np.linalg.norm(y - y_fp) / np.linalg.norm(y_w4 - y_fp))
+        rows.append({"rank": r, "gap_recovered": removed, "us": t})
     print(json.dumps({"svd_demo": {"workload": f"{args.workload}: M={M}, N={L.N}, K={L.K}, synthetic",
                                    "error": "|y - x W^T|_F relative to the plain 4-bit layer's",
                                    "ranks": rows}}))

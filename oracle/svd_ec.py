@@ -1,7 +1,7 @@
 """Static SVD-initialised error compensator in fp64.
 
-TEST INFRASTRUCTURE, like the rest of ``oracle/``: only the tests and the benchmark's demo leg use
-it, and the CUDA library never does.
+TEST INFRASTRUCTURE, like the rest of ``oracle/``: only the tests use it, and the CUDA library
+never does.
 
 SPEAR technical summary, section 1: the post-quantisation compensators that precede SPEAR apply
 one static low-rank correction to every token; section 3.1 reports how much of the gap between
