@@ -40,6 +40,8 @@ WORKLOADS = {
     "decode-mlp": (2, [1, 8, 32, 64], "decode"),
     "prefill": (3, [2048], "prefill"),
 }
+# Plan sweeps only (--sweep): the four linear shapes of the 16-layer model (rank-32 compensator).
+SWEEP_ONLY = {"sweep-1b": (4, [1, 16, 256])}
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -49,7 +51,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode-qo", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="decode-qo", choices=sorted(WORKLOADS) + sorted(SWEEP_ONLY))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the secondary prefill measurement")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -58,6 +60,9 @@ def parse():
     ap.add_argument("--once", type=int, default=0, metavar="M",
                     help="run 5 layer calls of the workload with M tokens and exit (for profilers)")
     ap.add_argument("--no-ec", action="store_true", help="with --once: the plain W4 layer")
+    ap.add_argument("--model-sweep", action="store_true",
+                    help="the 16-layer sweep workload (hidden 2048, MLP 8192, EC r=32 on layers 0, 1, 7, 15): "
+                         "all 64 linears of one pass per batch size, with the dispatcher's plans")
     ap.add_argument("--svd-demo", action="store_true",
                     help="static SVD-initialised compensator on the workload's layer: share of the 4-bit "
                          "output error removed and time per call, for several ranks")
@@ -476,8 +481,19 @@ def sweep_plans(args):
     import w4_gemm_error_channel_b200 as spear
     from synthetic import config_layers
     torch.cuda.set_device(0)
-    cfg, batches, kind = WORKLOADS[args.workload]
-    L = config_layers(cfg, M=max(batches))[0]
+    if args.workload in SWEEP_ONLY:
+        cfg, batches = SWEEP_ONLY[args.workload]
+        shapes = config_layers(cfg, M=max(batches), layers=(0,))        # layer 0 carries an EC
+    else:
+        cfg, batches, kind = WORKLOADS[args.workload]
+        shapes = config_layers(cfg, M=max(batches))[:1]
+    rows = []
+    for L in shapes:
+        rows += _sweep_shape(torch, spear, L, batches)
+    print(json.dumps({"workload": args.workload, "sweep": rows}))
+
+
+def _sweep_shape(torch, spear, L, batches):
     N, K, r = L.N, L.K, L.rank
     per_set = layer_bytes(max(batches), N, K, r)
     copies = max(2, int(np.ceil(2 * L2_BYTES / per_set)) + 1)
@@ -537,7 +553,9 @@ def sweep_plans(args):
                                  "tile_n": tile_n,
                                  "split_k": split, "us": best,
                                  "GBps": layer_bytes(M, N, K, r if use_ec else 0) / best / 1e3})
-    print(json.dumps({"workload": args.workload, "sweep": rows}))
+    del sets
+    torch.cuda.empty_cache()
+    return rows
 
 
 def run_once(args):
@@ -616,8 +634,88 @@ def svd_demo(args):
                                    "ranks": rows}}))
 
 
+def model_sweep(args):
+    """Config 4: one pass over the 64 linears of the 16-layer model (qkv, o, up+gate, down per
+    layer; compensators of rank 32 on layers 0, 1, 7, 15) for M in {1, 16, 256, 4096}, each call
+    planned by spear_gemm_plan.  Weights are distinct per linear (512 MiB of W4 in all, > 2x L2);
+    each linear reads a synthetic x of its K.  Timed as a CUDA graph of the whole pass."""
+    import torch
+    import w4_gemm_error_channel_b200 as spear
+    from synthetic import make_layer
+    from synthetic.workloads import SWEEP_EC_LAYERS, SWEEP_LAYERS, SWEEP_LINEARS, SWEEP_RANK
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda")
+    batches = [1, 16, 256, 4096]
+    Mmax = max(batches)
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+    linears = []
+    for layer in range(SWEEP_LAYERS):
+        for li, (lname, N, K) in enumerate(SWEEP_LINEARS):
+            rank = SWEEP_RANK if layer in SWEEP_EC_LAYERS else 0
+            L = make_layer(f"L{layer}.{lname}", np.random.SeedSequence([1004, layer, li]), 1, N, K, rank,
+                           outlier_frac=0.01, outlier_scale=20.0)
+            W = torch.from_numpy(L.W).to(dev)
+            packed, scale, zero = spear.spear_pack_w4(W)
+            del W
+            ec = spear.EC(bf(L.A_bits), bf(L.B_bits), bf(L.wg_bits), L.b_g) if rank else None
+            linears.append((N, K, rank, spear.W4ECLayer(packed, scale, zero, ec)))
+    xs = {K: bf(make_layer(f"x{K}", 1004 + K, Mmax, 128, K, 0, outlier_frac=0.01, outlier_scale=20.0).x_bits)
+          for K in sorted({K for (_, K, _, _) in linears})}
+    ys = {N: torch.empty((Mmax, N), dtype=torch.bfloat16, device=dev) for N in sorted({N for (N, _, _, _) in linears})}
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    hbm = peaks.get("hbm_gbs", 6650.0)
+    tc = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1590.0))
+    stream = torch.cuda.Stream()
+    rows = []
+    for M in batches:
+        kinds = {}
+        for (N, K, rank, lay) in linears:
+            p = lay.plan(M)
+            key = "tcgen05" if p.kernel_id == spear.SPEAR_KERNEL_TC05 else "split-K decode"
+            kinds[key] = kinds.get(key, 0) + 1
+
+        def one_pass():
+            for (N, K, rank, lay) in linears:
+                lay(xs[K][:M], y=ys[N][:M], stream=stream)
+        with torch.cuda.stream(stream):
+            one_pass()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                one_pass()
+        for _ in range(2):
+            g.replay()
+        stream.synchronize()
+        n = 10 if M <= 256 else 3
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(n):
+                g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        t = e0.elapsed_time(e1) / 1e3 / n
+        del g
+        byts = sum(layer_bytes(M, N, K, r) for (N, K, r, _) in linears)
+        flops = sum(layer_flops(M, N, K, r) for (N, K, r, _) in linears)
+        bound = max(byts / (hbm * 1e9), flops / (tc * 1e12))
+        status = max(spear.spear_get_device_status(lay.workspace) for (_, _, _, lay) in linears)
+        rows.append({"M": M, "us_per_pass": t * 1e6, "GBps": byts / t / 1e9, "TFLOPs": flops / t / 1e12,
+                     "roofline_frac": bound / t, "bound": "hbm" if byts / (hbm * 1e9) >= flops / (tc * 1e12) else "tensor",
+                     "kernels": kinds, "device_status": status})
+    print(json.dumps({"model_sweep": {"workload": "16 layers x (qkv 6144x2048, o 2048x2048, up 16384x2048, "
+                                                  "down 2048x8192), EC r=32 on layers 0, 1, 7, 15, synthetic",
+                                      "peaks": {"hbm_gbs": hbm, "bf16_tflops": tc, "note": "sustained bf16 peak"},
+                                      "passes": rows}}))
+
+
 def main():
     args = parse()
+    if args.model_sweep:
+        model_sweep(args)
+        return
     if args.svd_demo:
         svd_demo(args)
         return
@@ -627,6 +725,8 @@ def main():
     if args.sweep:
         sweep_plans(args)
         return
+    if args.workload in SWEEP_ONLY:
+        raise SystemExit(f"--workload {args.workload} is for --sweep only")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -81,6 +81,7 @@ bool lookup_measured(int64_t M, int64_t N, int64_t K, int has_ec, int sms, spear
     for (const MeasuredPlan& e : kMeasured) {
         const int enb = e.M <= 8 ? 1 : (e.M <= 16 ? 2 : 4);
         if (e.N != N || e.K != K || e.has_ec != has_ec || enb != nb) continue;
+        if (e.M > 2 * M || 2 * e.M < M) continue;        // measured within a factor of two of M
         // Same token-tile size; prefer the measured batch closest to M.
         if (!best || std::llabs(e.M - M) < std::llabs(best->M - M)) best = &e;
     }
@@ -233,7 +234,9 @@ spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int 
     if (st != SPEAR_OK) return st;
     const int sms = device_sms(device);
     spear_plan p = {};
-    if (use_tc05(M, rank)) st = plan_tc05(M, N, sms, &p);
+    // A measured plan for this shape (either kernel) first, then the rules.
+    if (lookup_measured(M > 0 ? M : 1, N, K, rank > 0 ? 1 : 0, sms, &p)) st = SPEAR_OK;
+    else if (use_tc05(M, rank)) st = plan_tc05(M, N, sms, &p);
     else st = plan_decode(M > 0 ? M : 1, N, K, rank, sms, &p);
     if (st != SPEAR_OK) return st;
     p.workspace_bytes = workspace_bytes_for(p, M, N, rank);
@@ -265,7 +268,8 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
     if (plan) {
         p = *plan;
     } else {
-        if (use_tc05(M, rank)) st = plan_tc05(M, N, sms, &p);
+        if (lookup_measured(M, N, K, rank > 0 ? 1 : 0, sms, &p)) st = SPEAR_OK;
+        else if (use_tc05(M, rank)) st = plan_tc05(M, N, sms, &p);
         else st = plan_decode(M, N, K, rank, sms, &p);
         if (st != SPEAR_OK) return st;
     }
