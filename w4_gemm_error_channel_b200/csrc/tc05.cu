@@ -70,6 +70,14 @@ SPEAR_DEVI void tma_load_2d(void* dst, const CUtensorMap* map, int32_t c0, int32
         ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar)) : "memory");
 }
 
+// Shared memory -> global tile store (no multicast); coordinates are never negative here.
+SPEAR_DEVI void tma_store_2d(const CUtensorMap* map, const void* src, int32_t c0, int32_t c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(map), "r"(smem_u32(src)), "r"(c0), "r"(c1) : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+SPEAR_DEVI void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 SPEAR_DEVI void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 SPEAR_DEVI void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 SPEAR_DEVI void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -184,7 +192,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                const __grid_constant__ CUtensorMap tmap_u, const __grid_constant__ CUtensorMap tmap_g,
-               const __grid_constant__ CUtensorMap tmap_x128, TcArgs a) {
+               const __grid_constant__ CUtensorMap tmap_x128, const __grid_constant__ CUtensorMap tmap_y,
+               TcArgs a) {
     using L = TcSmem<BN, STAGES, SUB>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -428,7 +437,11 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             named_bar_epi();
             if (row == 0 && acc_ok) asm volatile("st.release.gpu.global.u32 [%0], 1;" ::"l"(&a.ec_ready[mb]) : "memory");
         } else {
-            // y[m, n] = s[n] D[n, m] (+ E[n, m]), sub-tile by sub-tile.
+            // y[m, n] = s[n] D[n, m] (+ E[n, m]), sub-tile by sub-tile.  bf16 output: the tile is
+            // staged in the (now idle) x stages as y[m][n] rows and leaves in one TMA store,
+            // which also drops the rows past M; fp32 debug output is stored directly.
+            constexpr int YROWS = TC_BM * SUB;
+            __nv_bfloat16* ys = reinterpret_cast<__nv_bfloat16*>(smem + L::X_OFF);   // [BN][YROWS]
             for (int sb = 0; sb < SUB; ++sb) {
             const float sc = __half2float(a.scale[n0 + sb * TC_BM + row]);
             const int64_t n = n0 + sb * TC_BM + row;
@@ -440,15 +453,22 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int64_t m = m0 + c0 + i;
-                    if (m < a.M) {
-                        const float yv = has_ec ? fmaf(sc, v[i], e[i]) : sc * v[i];
-                        if (a.y_fp32)
-                            reinterpret_cast<float*>(a.y)[m * a.N + n] = yv;
-                        else
-                            reinterpret_cast<__nv_bfloat16*>(a.y)[m * a.N + n] = __float2bfloat16_rn(yv);
+                    const float yv = has_ec ? fmaf(sc, v[i], e[i]) : sc * v[i];
+                    if (a.y_fp32) {
+                        if (m < a.M) reinterpret_cast<float*>(a.y)[m * a.N + n] = yv;
+                    } else {
+                        ys[(c0 + i) * YROWS + sb * TC_BM + row] = __float2bfloat16_rn(yv);
                     }
                 }
             }
+            }
+            if (!a.y_fp32 && acc_ok) {
+                fence_proxy_async_smem();            // generic-proxy writes -> visible to the TMA
+                named_bar_epi();
+                if (row == 0) {
+                    tma_store_2d(&tmap_y, ys, (int32_t)n0, (int32_t)m0);
+                    tma_store_wait_read();
+                }
             }
         }
     }
@@ -509,6 +529,15 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
     if (!make_map_2d(&mx128, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.K, (uint64_t)a.M, TC_BK, TC_EB,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
+    CUtensorMap my;
+    if (!a.y_fp32) {
+        // y [M, N] bf16 written as BN (m) x 128 SUB (n) boxes.
+        if (!make_map_2d(&my, a.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.N, (uint64_t)a.M, TC_BM * SUB, BN,
+                         CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    } else {
+        my = mx;                                 // unused: fp32 output is stored directly
+    }
     const bool has_ec = a.rank > 0;
     if (has_ec) {
         // A [K, r] read as 64 (j) x 64 (k) boxes; B [r, N] as 64 (n) x 64 (j); u [M, r] as 64 (j) x BN (m).
@@ -546,7 +575,7 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, w4_tc05_kernel<BN, STAGES, SUB>, mx, mw, ma, mb, mu, mg, mx128, a);
+    return cudaLaunchKernelEx(&cfg, w4_tc05_kernel<BN, STAGES, SUB>, mx, mw, ma, mb, mu, mg, mx128, my, a);
 }
 
 cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream) {
