@@ -41,7 +41,7 @@ WORKLOADS = {
     "prefill": (3, [2048], "prefill"),
 }
 # Plan sweeps only (--sweep): the four linear shapes of the 16-layer model (rank-32 compensator).
-SWEEP_ONLY = {"sweep-1b": (4, [1, 16, 256])}
+SWEEP_ONLY = {"sweep-1b": (4, [1, 16, 256, 4096])}
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -509,17 +509,19 @@ def _sweep_shape(torch, spear, L, batches):
         ws = spear.alloc_workspace(base.workspace_bytes + (M * r * 2 + 255) // 256 * 256 + min(M, 256) * N * 4)
         # (kernel, tile_n, split_k, flags): every split-K decode tiling, fused and with the separate
         # EC pass, and the tcgen05 kernel with 128-token tiles.
-        candidates = [(1, tile_n, split, fl) for tile_n in (16, 32, 64, 128) for split in (1, 2, 4, 8)
-                      for fl in (0, 1)]
-        candidates.append((2, 128, 1, 0))
-        for kernel_id, tile_n, split, fl in candidates:
+        candidates = [] if M >= 1024 else [(1, tile_n, split, fl) for tile_n in (16, 32, 64, 128)
+                                           for split in (1, 2, 4, 8) for fl in (0, 1)]
+        candidates += [(2, 128, 1, 0, 128)] + ([(2, 128, 1, 0, 256)] if M >= 256 else [])
+        for cand in candidates:
+                kernel_id, tile_n, split, fl = cand[:4]
+                tc_tile_m = cand[4] if len(cand) > 4 else None
                 for use_ec in (True, False):
                     if fl and not use_ec:
                         continue
                     plan = spear.spear_plan.from_buffer_copy(base)
                     plan.kernel_id, plan.tile_n, plan.split_k, plan.flags = kernel_id, tile_n, split, fl
                     if kernel_id == 2:
-                        plan.tile_m = 128
+                        plan.tile_m = tc_tile_m
                     elif base.kernel_id == 2:
                         plan.tile_m = 8 if M <= 8 else (16 if M <= 16 else 32)
                     n_calls = 64
@@ -550,7 +552,7 @@ def _sweep_shape(torch, spear, L, batches):
                         best = min(best, e0.elapsed_time(e1) * 1e3 / n_calls)
                     del g
                     rows.append({"M": M, "N": N, "K": K, "rank": r if use_ec else 0, "kernel": kernel_id, "flags": fl,
-                                 "tile_n": tile_n,
+                                 "tile_n": tile_n, "tile_m": plan.tile_m,
                                  "split_k": split, "us": best,
                                  "GBps": layer_bytes(M, N, K, r if use_ec else 0) / best / 1e3})
     del sets

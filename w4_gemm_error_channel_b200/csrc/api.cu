@@ -66,7 +66,7 @@ size_t workspace_bytes_for(const spear_plan& p, int64_t M, int64_t N_for_ws, int
 // Measured plans (plans/gen_table.py): the fastest tiling per swept shape on one B200.
 struct MeasuredPlan {
     int64_t M, N, K;
-    int has_ec, kernel_id, tile_n, split_k, flags;
+    int has_ec, kernel_id, tile_n, split_k, tile_m, flags;
     double us;
 };
 spear_status plan_tc05(int64_t M, int64_t N, int sms, spear_plan* p);
@@ -86,7 +86,11 @@ bool lookup_measured(int64_t M, int64_t N, int64_t K, int has_ec, int sms, spear
         if (!best || std::llabs(e.M - M) < std::llabs(best->M - M)) best = &e;
     }
     if (!best) return false;
-    if (best->kernel_id == SPEAR_KERNEL_TC05) return plan_tc05(M, N, sms, p) == SPEAR_OK;
+    if (best->kernel_id == SPEAR_KERNEL_TC05) {
+        if (plan_tc05(M, N, sms, p) != SPEAR_OK) return false;
+        if (best->tile_m == 128 || best->tile_m == 256) p->tile_m = best->tile_m;   // the measured width
+        return true;
+    }
     p->kernel_id = SPEAR_KERNEL_SPLITK;
     p->tile_n = best->tile_n;
     p->split_k = best->split_k;

@@ -181,6 +181,9 @@ struct TcSmem {
     // once the main K loop has retired.
     static constexpr int NEED = SUB * BN + (SUB * STAGES * 32 > SUB * BN ? SUB * STAGES * 32 : SUB * BN);
     static constexpr uint32_t TMEM_COLS = NEED <= 32 ? 32 : NEED <= 64 ? 64 : NEED <= 128 ? 128 : NEED <= 256 ? 256 : 512;
+    // Two CTAs share an SM when both fit (shared memory and TMEM): one tile's prologue and
+    // epilogue then overlap the other's MMAs.
+    static constexpr int MIN_BLOCKS = (TOTAL <= 112 * 1024 && TMEM_COLS <= 256) ? 2 : 1;
 };
 constexpr int TC_EB = 128;               // tokens per EC tile
 
@@ -188,7 +191,7 @@ constexpr int TC_EB = 128;               // tokens per EC tile
 // main tiles (128 SUB weight rows, token block mb of BN tokens), token-block major.  With SUB = 2
 // the two 128-row sub-tiles share every x stage, which halves the x traffic from L2.
 template <int BN, int STAGES, int SUB>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(TC_THREADS, (TcSmem<BN, STAGES, SUB>::MIN_BLOCKS))
 w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                const __grid_constant__ CUtensorMap tmap_u, const __grid_constant__ CUtensorMap tmap_g,
@@ -581,7 +584,7 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
 cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream) {
     if (rows == 256) return bn == 128 ? launch_tc_t<128, 4, 2>(a, stream) : cudaErrorInvalidValue;
     if (rows != 128) return cudaErrorInvalidValue;
-    if (bn == 128) return launch_tc_t<128, 6, 1>(a, stream);
+    if (bn == 128) return launch_tc_t<128, 3, 1>(a, stream);
     if (bn == 160) return launch_tc_t<160, 4, 1>(a, stream);
     if (bn == 192) return launch_tc_t<192, 3, 1>(a, stream);
     if (bn == 256) return launch_tc_t<256, 4, 1>(a, stream);
