@@ -11,15 +11,19 @@ namespace spear {
 // Zeroed part of every workspace: it must start zeroed and every call leaves it zeroed again
 // (unless a bounded wait timed out).
 //   control block, CTRL_BYTES, in 32-bit words:
-//     [0]                     device error word (bit 0: an arrival wait gave up; bit 1: an EC
-//                             partial sum was outside the fixed-point range)
-//     [64, +CHUNKS)           EC arrival counters, one per token chunk of a launch
-//     [.., +CHUNKS)           consumer counters (level 2: finished groups), one per token chunk
+//     [0]                     device error word (bit 0: a wait for the EC accumulators gave up;
+//                             bit 1: an EC partial sum was outside the fixed-point range;
+//                             bits 2, 3: prefill kernel waits)
+//     [64, +CHUNKS)           reserved (cleared by the decode kernel; no longer counted)
+//     [.., +CHUNKS)           consumer counters (level 2: finished groups), one per token chunk;
+//                             word 0 also counts the CTAs of the separate EC pass
 //     [.., +CHUNKS*GROUPS)    consumer counters (level 1: CTAs of a group of 64 GEMM CTAs)
 //     [.., +TC_BLOCKS)        prefill kernel: u-ready flags, one per token block
 //     [.., +TC_BLOCKS)        prefill kernel: flag consumer counters
 //   EC accumulators, TACC_BYTES: int64 [tokens of a launch][r + 1] (t, then the gate
-//   pre-activation), fixed point with 32 fraction bits.
+//   pre-activation), fixed point with 32 fraction bits above an 8-bit count of the K slices added.
+// After the zeroed part: the prefill kernel's u (bf16 [M][r]) or the separate EC pass's fp32
+// main term ([tokens of a launch][N]).
 constexpr size_t CTRL_BYTES = 128 * 1024;
 constexpr size_t CTRL_HEADER_WORDS = 64;
 constexpr size_t CHUNKS_MAX = 32;                          // token chunks per launch (>= 8 tokens each)
@@ -55,7 +59,7 @@ struct DecodeArgs {
     int mchunks;            // ceil(M / (8 NB))
     long long* tacc;        // [M][r + 1] EC accumulators (zeroed part of the workspace)
     unsigned* err;          // error word
-    unsigned* arrivals;     // [mchunks]
+    unsigned* arrivals;     // [mchunks] reserved words, cleared with the accumulators
     unsigned* consumed;     // [mchunks] level-2 consumer counters
     unsigned* consumed1;    // [mchunks][GROUPS_MAX] level-1 consumer counters
     float* ymain;           // separate EC pass: fp32 main term [M][N] (workspace); null when fused
