@@ -69,6 +69,8 @@ class Oracle:
                                          ctypes.c_int32, P]
         lib.oracle_w4ec_gemm_sampled.argtypes = [P, I64, I64, I64, P, P, P, P, P, P, ctypes.c_float,
                                                  ctypes.c_int32, P, P, I64, P]
+        lib.oracle_w4ec_gemm_mlp.argtypes = [P, I64, I64, I64, P, P, P, P, P, ctypes.c_int32, P, P, P, P,
+                                             ctypes.c_int32, ctypes.c_float, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         self._lib = lib
         self.path = lib_path
@@ -151,6 +153,22 @@ class Oracle:
                                    _ptr(_c(z_bits, np.uint16)), _ptr(_c(A_bits, np.uint16)),
                                    _ptr(_c(B_bits, np.uint16)), _ptr(_c(wg_bits, np.uint16)),
                                    ctypes.c_float(b_g), r, _ptr(y))
+        return y
+
+    def w4ec_gemm_mlp(self, x_bits, packed, s_bits, z_bits, A_bits, B_bits, W1, b1, W2, b2, alpha: float = 1.0):
+        """The layer with the bottleneck-MLP gate (see oracle_w4ec_gemm_mlp): fp64 y [M, N]."""
+        x_bits = _c(x_bits, np.uint16)
+        M, K = x_bits.shape
+        N = packed.shape[0]
+        A_bits, B_bits = _c(A_bits, np.uint16), _c(B_bits, np.uint16)
+        r = A_bits.shape[1]
+        W1, b1, W2, b2 = (_c(a, np.float32) for a in (W1, b1, W2, b2))
+        H = W1.shape[0]
+        assert W1.shape == (H, r) and b1.shape == (H,) and W2.shape == (r, H) and b2.shape == (r,)
+        y = np.empty((M, N), dtype=np.float64)
+        self._lib.oracle_w4ec_gemm_mlp(_ptr(x_bits), M, N, K, _ptr(_c(packed, np.uint8)), _ptr(_c(s_bits, np.uint16)),
+                                      _ptr(_c(z_bits, np.uint16)), _ptr(A_bits), _ptr(B_bits), r, _ptr(W1), _ptr(b1),
+                                      _ptr(W2), _ptr(b2), H, ctypes.c_float(alpha), _ptr(y))
         return y
 
     def w4ec_gemm_sampled(self, x_bits, packed, s_bits, z_bits, A_bits, B_bits, wg_bits, b_g,

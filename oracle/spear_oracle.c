@@ -285,6 +285,54 @@ void oracle_w4ec_gemm(const uint16_t* x, int64_t M, int64_t N, int64_t K,
     free(t); free(p); free(g);
 }
 
+/* The pages' gate form (technical summary section 2.1A): effective weight
+ * W + alpha * B diag(gamma(Ax)) A, gamma a bottleneck MLP.  The pages do not
+ * spell the MLP out; this follows the plainest reading of "bottleneck MLP" over
+ * the rank-r projection t = x A, one output per rank component:
+ *   h[m,i]     = max(0, sum_j W1[i,j] t[m,j] + b1[i])          i < H   (W1 [H, r])
+ *   gamma[m,j] = 1 / (1 + exp(-(sum_i W2[j,i] h[m,i] + b2[j])))   (W2 [r, H])
+ *   u[m,j]     = alpha * gamma[m,j] * t[m,j]
+ *   y[m,n]     = sum_k x[m,k] What[n,k] + sum_j u[m,j] B[j,n]
+ * W1, b1, W2, b2 are fp32; everything is evaluated in fp64.  y is fp64 [M,N]. */
+void oracle_w4ec_gemm_mlp(const uint16_t* x, int64_t M, int64_t N, int64_t K,
+                          const uint8_t* packed, const uint16_t* s_bits, const uint16_t* z_bits,
+                          const uint16_t* A, const uint16_t* B, int32_t r,
+                          const float* W1, const float* b1, const float* W2, const float* b2, int32_t H,
+                          float alpha, double* y)
+{
+    /* t = x A from the scalar-gate path (its gate outputs are not used here). */
+    uint16_t* wg0 = (uint16_t*)calloc((size_t)K, sizeof(uint16_t));
+    double* t = (double*)malloc(sizeof(double) * (size_t)(M * r));
+    double* p = (double*)malloc(sizeof(double) * (size_t)M);
+    double* g = (double*)malloc(sizeof(double) * (size_t)M);
+    oracle_ec_gate(x, M, K, A, r, wg0, 0.0f, t, p, g);
+    double* u = (double*)malloc(sizeof(double) * (size_t)(M * r));
+    double* h = (double*)malloc(sizeof(double) * (size_t)H);
+    for (int64_t m = 0; m < M; ++m) {
+        const double* tm = t + m * r;
+        for (int32_t i = 0; i < H; ++i) {
+            double pre = (double)b1[i];
+            for (int32_t j = 0; j < r; ++j) pre += (double)W1[(int64_t)i * r + j] * tm[j];
+            h[i] = pre > 0.0 ? pre : 0.0;
+        }
+        for (int32_t j = 0; j < r; ++j) {
+            double pre = (double)b2[j];
+            for (int32_t i = 0; i < H; ++i) pre += (double)W2[(int64_t)j * H + i] * h[i];
+            u[m * r + j] = (double)alpha * (1.0 / (1.0 + exp(-pre))) * tm[j];
+        }
+    }
+    /* Main term: the plain layer; then the compensator term. */
+    oracle_w4ec_gemm(x, M, N, K, packed, s_bits, z_bits, NULL, NULL, NULL, 0.0f, 0, y);
+    #pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t m = 0; m < M; ++m) {
+            double e = 0.0;
+            for (int32_t j = 0; j < r; ++j) e += u[m * r + j] * oracle_bf16_to_f64(B[(int64_t)j * N + n]);
+            y[m * N + n] += e;
+        }
+    free(wg0); free(t); free(p); free(g); free(u); free(h);
+}
+
 /* Same layer, evaluated only at `count` sampled outputs (mi[c], ni[c]) -> y[c].
  * Used where the full product is too large for the CPU (the full-size workloads). */
 void oracle_w4ec_gemm_sampled(const uint16_t* x, int64_t M, int64_t N, int64_t K,

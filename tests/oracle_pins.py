@@ -278,6 +278,53 @@ def pin_sampled_and_prefix(o):
     assert np.array_equal(o.w4ec_gemm(x[:4], packed, s, z, A, B, wg, b_g), y[:4])
 
 
+def pin_mlp_gate(o):
+    """Bottleneck-MLP gate (gamma(t) = sigmoid(W2 relu(W1 t + b1) + b2), u = alpha gamma t) against
+    cases that reduce to the scalar-gate oracle or to the plain layer, plus its invariances."""
+    x, W, A, B, wg, _ = small_layer(31, M=5, N=32, K=64, r=8)
+    packed, s, z = o.pack_w4(W)
+    r, H = 8, 3
+    rng = np.random.default_rng(32)
+    W1 = rng.standard_normal((H, r)).astype(np.float32)
+    b1 = rng.standard_normal(H).astype(np.float32) * 0.1
+    W2 = rng.standard_normal((r, H)).astype(np.float32)
+    b2 = rng.standard_normal(r).astype(np.float32) * 0.1
+    y0 = o.w4ec_gemm(x, packed, s, z)
+    zeros_wg = np.zeros_like(wg)
+    scale = 1e-12 * np.abs(y0).max()
+    # gamma = 1 (W2 = 0, b2 = +inf): the scalar gate at g = 1.
+    inf = np.full(r, np.inf, np.float32)
+    y1 = o.w4ec_gemm_mlp(x, packed, s, z, A, B, W1, b1, np.zeros_like(W2), inf, 1.0)
+    assert np.allclose(y1, o.w4ec_gemm(x, packed, s, z, A, B, zeros_wg, float("inf")), rtol=0, atol=scale)
+    # gamma = 0 (b2 = -inf): the plain layer.
+    assert np.allclose(o.w4ec_gemm_mlp(x, packed, s, z, A, B, W1, b1, np.zeros_like(W2), -inf, 1.0), y0,
+                       rtol=0, atol=scale)
+    # Dead hidden units (b1 very negative) and equal output biases c: gamma = sigmoid(c) everywhere,
+    # the scalar gate with w_g = 0, b_g = c.
+    c = np.float32(-0.75)
+    yd = o.w4ec_gemm_mlp(x, packed, s, z, A, B, W1, np.full(H, -1e30, np.float32), W2, np.full(r, c, np.float32), 1.0)
+    assert np.allclose(yd, o.w4ec_gemm(x, packed, s, z, A, B, zeros_wg, float(c)), rtol=0, atol=scale)
+    # One hidden unit that reads rank j0 (W1 = e_j0, a large b1 keeps relu linear, b2 = -b1):
+    # gamma_j = sigmoid(t_j0) for every j, the scalar gate with w_g = column j0 of A.
+    j0 = 5
+    e = np.zeros((1, r), np.float32)
+    e[0, j0] = 1.0
+    big = np.float32(100.0)
+    ys = o.w4ec_gemm_mlp(x, packed, s, z, A, B, e, np.array([big], np.float32), np.ones((r, 1), np.float32),
+                         np.full(r, -big, np.float32), 1.0)
+    col = np.ascontiguousarray(A[:, j0])
+    assert np.allclose(ys, o.w4ec_gemm(x, packed, s, z, A, B, col, 0.0), rtol=0, atol=1e-9 * np.abs(ys).max())
+    # alpha scales the compensator term linearly.
+    ya = o.w4ec_gemm_mlp(x, packed, s, z, A, B, W1, b1, W2, b2, 1.0)
+    yb = o.w4ec_gemm_mlp(x, packed, s, z, A, B, W1, b1, W2, b2, 2.5)
+    assert np.allclose(yb - y0, 2.5 * (ya - y0), rtol=0, atol=scale)
+    assert np.abs(ya - y0).max() > 1e3 * scale
+    # Duplicated hidden units with halved output weights leave the layer unchanged.
+    yu = o.w4ec_gemm_mlp(x, packed, s, z, A, B, np.vstack([W1, W1]), np.concatenate([b1, b1]),
+                         np.hstack([W2, W2]) / 2, b2, 1.0)
+    assert np.allclose(yu, ya, rtol=0, atol=scale)
+
+
 ALL_PINS = [pin_f16_encoder, pin_golden_rows, pin_grid_round_trip, pin_rtn_bruteforce, pin_scale_pow2,
             pin_main_term_vs_numpy, pin_ec_vs_numpy, pin_gate_limits, pin_bruteforce_rational,
-            pin_sampled_and_prefix]
+            pin_sampled_and_prefix, pin_mlp_gate]

@@ -30,6 +30,11 @@ MUTATIONS = {
     "zero_point_sign": ("rintf(negl / s)", "rintf(lo / s)"),
     "f16_ties_away": ("if (rem > half || (rem == half && (kept & 1u))) q += 1;",
                       "if (rem >= half) q += 1;"),
+    "mlp_relu_dropped": ("h[i] = pre > 0.0 ? pre : 0.0;", "h[i] = pre;"),
+    "mlp_alpha_inside_sigmoid": ("u[m * r + j] = (double)alpha * (1.0 / (1.0 + exp(-pre))) * tm[j];",
+                                 "u[m * r + j] = (1.0 / (1.0 + exp(-(double)alpha * pre))) * tm[j];"),
+    "mlp_W1_transposed": ("(double)W1[(int64_t)i * r + j] * tm[j]", "(double)W1[(int64_t)j * H + i] * tm[j]"),
+    "mlp_W2_transposed": ("(double)W2[(int64_t)j * H + i] * h[i]", "(double)W2[(int64_t)i * r + j] * h[i]"),
     "main_term_dropped_last_k": ("for (int64_t k = 0; k < K; ++k) acc += xr[k] * wrow[k];",
                                  "for (int64_t k = 0; k < K - 1; ++k) acc += xr[k] * wrow[k];"),
 }
