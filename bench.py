@@ -63,6 +63,9 @@ def parse():
     ap.add_argument("--model-sweep", action="store_true",
                     help="the 16-layer sweep workload (hidden 2048, MLP 8192, EC r=32 on layers 0, 1, 7, 15): "
                          "all 64 linears of one pass per batch size, with the dispatcher's plans")
+    ap.add_argument("--gate-compare", action="store_true",
+                    help="time the layer with the scalar gate and with the bottleneck-MLP gate (H=16) on "
+                         "decode-qo M=16 and the prefill layer")
     ap.add_argument("--svd-demo", action="store_true",
                     help="static SVD-initialised compensator on the workload's layer: share of the 4-bit "
                          "output error removed and time per call, for several ranks")
@@ -713,8 +716,69 @@ def model_sweep(args):
                                       "passes": rows}}))
 
 
+def gate_compare(args):
+    """Device time per call of the same layer with the scalar gate and with the bottleneck-MLP gate
+    (H = 16, random fp32 gate weights), in a chained CUDA graph of calls over rotating weight copies."""
+    import torch
+    import w4_gemm_error_channel_b200 as spear
+    from synthetic import config_layers
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda")
+    stream = torch.cuda.Stream()
+    rows = []
+    for wname, M in (("decode-qo", 16), ("prefill", 2048)):
+        cfg = WORKLOADS[wname][0]
+        L = config_layers(cfg, M=M)[0]
+        per_set = layer_bytes(M, L.N, L.K, L.rank)
+        copies = max(2, int(np.ceil(2 * L2_BYTES / per_set)) + 1)
+        sets = make_device_layer(torch, spear, L, copies)
+        x = torch.from_numpy(L.x(M).view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((M, L.N), dtype=torch.bfloat16, device=dev)
+        rng = np.random.default_rng(5)
+        H = 16
+        gate = [torch.from_numpy((rng.standard_normal(sh) * 0.3).astype(np.float32)).to(dev)
+                for sh in ((H, L.rank), (H,), (L.rank, H), (L.rank,))]
+        res = {"workload": f"{wname} M={M}", "rank": L.rank, "hidden": H}
+        for kind in ("scalar", "mlp"):
+            def ec_of(A, B, wg):
+                if kind == "scalar":
+                    return spear.EC(A, B, wg, L.b_g)
+                return spear.EC(A, B, wg, L.b_g, gate_w1=gate[0], gate_b1=gate[1], gate_w2=gate[2],
+                                gate_b2=gate[3], alpha=1.0)
+            layers = [spear.W4ECLayer(p, s_, z, ec_of(A, B, wg)) for (p, s_, z, A, B, wg) in sets]
+            n = 32 if M <= 64 else 8
+            with torch.cuda.stream(stream):
+                for lay in layers:
+                    lay(x, y=y, stream=stream)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(n):
+                        layers[i % copies](x, y=y, stream=stream)
+            best = 1e9
+            for _ in range(5):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    g.replay()
+                    e1.record(stream)
+                e1.synchronize()
+                best = min(best, e0.elapsed_time(e1) * 1e3 / n)
+            del g
+            res[f"us_{kind}"] = best
+            res[f"status_{kind}"] = max(spear.spear_get_device_status(lay.workspace) for lay in layers)
+        rows.append(res)
+        del sets
+        torch.cuda.empty_cache()
+    print(json.dumps({"gate_compare": rows}))
+
+
 def main():
     args = parse()
+    if args.gate_compare:
+        gate_compare(args)
+        return
     if args.model_sweep:
         model_sweep(args)
         return

@@ -84,6 +84,17 @@ typedef struct {
     const void* w_g;  /* device, bf16 [K]         gate weights */
     float b_g;        /* gate bias (host value); -INFINITY gives g = 0 exactly */
     int32_t rank;     /* r: 16..256, a multiple of 16 */
+    /* Optional: the pages' gate form (section 2.1A), effective weight W + alpha B diag(gamma(Ax)) A
+     * with gamma a bottleneck MLP over t = x A:
+     *   gamma(t) = sigmoid(W2 relu(W1 t + b1) + b2),   u = alpha * gamma(t) * t  (elementwise).
+     * gate_w1 == NULL keeps the scalar gate above; otherwise w_g and b_g do not enter the result
+     * (w_g must still be a readable [K] array).  All four arrays are fp32 on the device. */
+    const void* gate_w1;   /* [gate_hidden, rank] */
+    const void* gate_b1;   /* [gate_hidden] */
+    const void* gate_w2;   /* [rank, gate_hidden] */
+    const void* gate_b2;   /* [rank] */
+    int32_t gate_hidden;   /* H: 1..64 */
+    float alpha;           /* compensator scale (MLP gate only) */
 } spear_ec;
 
 /* A launch plan.  Produced by spear_gemm_plan and read by spear_w4ec_gemm.  A
@@ -158,8 +169,9 @@ SPEAR_API spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t 
  *
  * Requires N % 128 == 0, K % 64 == 0 (and K <= 65536 with a compensator),
  * M >= 0 (M = 0 launches nothing).  The accumulation is fp32 throughout (the
- * EC factors u = g t enter the prefill tensor cores as a bf16 hi/lo pair).  The output is deterministic for a given
- * plan: no atomics take part in any floating-point sum.
+ * EC factors u = g t enter the prefill tensor cores rounded to bf16).  The
+ * output is deterministic for a given plan: no atomics take part in any
+ * floating-point sum.
  */
 SPEAR_API spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, int64_t N, int64_t K,
                              const void* packed, const void* scale, const void* zero,
@@ -180,7 +192,8 @@ SPEAR_API spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, in
  *
  *   Arguments as for spear_w4ec_gemm, minus the workspace.  plan may be NULL; a given plan must
  *   select SPEAR_KERNEL_SPLITK.
- *   Limits: 1 <= M <= 64 (larger M returns SPEAR_ERR_UNSUPPORTED_SHAPE), rank 0 or 16..256.
+ *   Limits: 1 <= M <= 64 (larger M returns SPEAR_ERR_UNSUPPORTED_SHAPE), rank 0 or 16..256, the
+ *   scalar gate only (ec->gate_w1 != NULL returns SPEAR_ERR_INVALID_ARG).
  *   The first call on a device looks up that device's scratch address (once per device, with the
  *   device current); make that first call before any stream capture.  Every call first clears the
  *   part of the scratch it uses, then launches the fused decode kernel.

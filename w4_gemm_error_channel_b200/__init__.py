@@ -48,7 +48,9 @@ class spear_plan(ctypes.Structure):
 
 class spear_ec(ctypes.Structure):
     _fields_ = [("A", ctypes.c_void_p), ("B", ctypes.c_void_p), ("w_g", ctypes.c_void_p),
-                ("b_g", ctypes.c_float), ("rank", ctypes.c_int32)]
+                ("b_g", ctypes.c_float), ("rank", ctypes.c_int32),
+                ("gate_w1", ctypes.c_void_p), ("gate_b1", ctypes.c_void_p), ("gate_w2", ctypes.c_void_p),
+                ("gate_b2", ctypes.c_void_p), ("gate_hidden", ctypes.c_int32), ("alpha", ctypes.c_float)]
 
 
 def _load():
@@ -109,11 +111,21 @@ def spear_version() -> int:
 
 @dataclasses.dataclass
 class EC:
-    """One layer's error compensator: A bf16 [K,r], B bf16 [r,N], w_g bf16 [K], b_g float."""
+    """One layer's error compensator: A bf16 [K,r], B bf16 [r,N], w_g bf16 [K], b_g float.
+
+    Optional bottleneck-MLP gate (the pages' gamma): gate_w1 fp32 [H,r], gate_b1 [H], gate_w2 [r,H],
+    gate_b2 [r] and alpha; with it, u = alpha * sigmoid(W2 relu(W1 t + b1) + b2) * t and the scalar
+    gate (w_g, b_g) does not enter the result.
+    """
     A: torch.Tensor
     B: torch.Tensor
     w_g: torch.Tensor
     b_g: float = 0.0
+    gate_w1: Optional[torch.Tensor] = None
+    gate_b1: Optional[torch.Tensor] = None
+    gate_w2: Optional[torch.Tensor] = None
+    gate_b2: Optional[torch.Tensor] = None
+    alpha: float = 1.0
 
     @property
     def rank(self) -> int:
@@ -125,7 +137,19 @@ class EC:
             _dev(t, name)
             if t.dtype != torch.bfloat16:
                 raise ValueError(f"EC.{name} must be bf16")
-        return spear_ec(self.A.data_ptr(), self.B.data_ptr(), self.w_g.data_ptr(), float(self.b_g), self.rank)
+        c = spear_ec(self.A.data_ptr(), self.B.data_ptr(), self.w_g.data_ptr(), float(self.b_g), self.rank)
+        if self.gate_w1 is not None:
+            for name in ("gate_w1", "gate_b1", "gate_w2", "gate_b2"):
+                t = getattr(self, name)
+                if t is None:
+                    raise ValueError(f"EC.{name} is required with the MLP gate")
+                _dev(t, name)
+                if t.dtype != torch.float32:
+                    raise ValueError(f"EC.{name} must be fp32")
+            c.gate_w1, c.gate_b1 = self.gate_w1.data_ptr(), self.gate_b1.data_ptr()
+            c.gate_w2, c.gate_b2 = self.gate_w2.data_ptr(), self.gate_b2.data_ptr()
+            c.gate_hidden, c.alpha = int(self.gate_w1.shape[0]), float(self.alpha)
+        return c
 
 
 def spear_pack_w4(W: torch.Tensor, packed=None, scale=None, zero=None, stream=None):

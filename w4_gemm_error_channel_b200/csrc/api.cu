@@ -40,6 +40,29 @@ spear_status check_shape(int64_t M, int64_t N, int64_t K, int32_t rank) {
     return SPEAR_OK;
 }
 
+// The optional bottleneck-MLP gate: all four arrays or none, H in 1..GATE_HIDDEN_MAX.
+spear_status check_gate_mlp(const spear_ec* ec) {
+    if (!ec || !ec->gate_w1) return SPEAR_OK;
+    if (!ec->gate_b1 || !ec->gate_w2 || !ec->gate_b2) return SPEAR_ERR_INVALID_ARG;
+    if (ec->gate_hidden < 1 || ec->gate_hidden > GATE_HIDDEN_MAX || isnan(ec->alpha)) return SPEAR_ERR_INVALID_ARG;
+    if (!aligned16(ec->gate_w1) || !aligned16(ec->gate_b1) || !aligned16(ec->gate_w2) || !aligned16(ec->gate_b2))
+        return SPEAR_ERR_MISALIGNED;
+    return SPEAR_OK;
+}
+
+GateMlp gate_mlp_of(const spear_ec* ec) {
+    GateMlp g = {};
+    if (ec && ec->gate_w1) {
+        g.w1 = (const float*)ec->gate_w1;
+        g.b1 = (const float*)ec->gate_b1;
+        g.w2 = (const float*)ec->gate_w2;
+        g.b2 = (const float*)ec->gate_b2;
+        g.hidden = ec->gate_hidden;
+        g.alpha = ec->alpha;
+    }
+    return g;
+}
+
 int nb_for_tile_m(int tile_m) { return tile_m <= 8 ? 1 : (tile_m <= 16 ? 2 : 4); }
 
 // K codes per slice for S slices: a multiple of 64, so every lane's 32-code piece is whole.
@@ -265,6 +288,8 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         !aligned16(zero) || !aligned16(workspace))
         return SPEAR_ERR_MISALIGNED;
     if (ec && (!aligned16(ec->A) || !aligned16(ec->B) || !aligned16(ec->w_g))) return SPEAR_ERR_MISALIGNED;
+    st = check_gate_mlp(ec);
+    if (st != SPEAR_OK) return st;
     if (M == 0) return SPEAR_OK;
 
     const int sms = device_sms(-1);
@@ -294,6 +319,7 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         t.B = ec ? (const uint16_t*)ec->B : nullptr;
         t.wg = ec ? (const uint16_t*)ec->w_g : nullptr;
         t.b_g = ec ? ec->b_g : 0.0f;
+        t.mlp = gate_mlp_of(ec);
         t.rank = rank;
         t.u = rank > 0 ? (__nv_bfloat16*)(ws + ZEROED_BYTES) : nullptr;
         t.y = y;
@@ -317,6 +343,7 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
     a.B = ec ? (const uint16_t*)ec->B : nullptr;
     a.wg = ec ? (const uint16_t*)ec->w_g : nullptr;
     a.b_g = ec ? ec->b_g : 0.0f;
+    a.mlp = gate_mlp_of(ec);
     a.rank = rank;
     a.y_fp32 = (y_dtype == SPEAR_FP32);
     a.N = N;

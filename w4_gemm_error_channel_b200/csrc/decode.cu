@@ -248,6 +248,8 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
     __shared__ unsigned s_flag;
     uint16_t* Bs = reinterpret_cast<uint16_t*>(dyn);                           // [ec_jr][RT] bf16
     float* us = reinterpret_cast<float*>(dyn + (size_t)a.ec_jr * RT * 2);      // [TM][ec_jr + 1]
+    float* mlp_t = us + TM * (a.ec_jr + 1);                                    // MLP gate: [TM][r + 1] t
+    float* mlp_h = mlp_t + TM * (a.rank + 1);                                  //           [TM][H + 1] hidden
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -398,7 +400,85 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
         const long long* tc = a.tacc + (int64_t)chunk * TM * (a.rank + 1);
         const int ujr = a.ec_jr + 1, total = tm * nj;
         const unsigned long long want = (unsigned long long)ec_slices(a.K) & FIX_COUNT_MASK;
-        if (nj > 0) {
+        if (nj > 0 && a.mlp.w1 != nullptr) {
+            // The bottleneck-MLP gate reads every column of t: all tm x r words (bounded wait on
+            // their slice counts), then h = relu(W1 t + b1), then gamma and u for this CTA's columns.
+            const int r = a.rank, H = a.mlp.hidden, tot = tm * r;
+            constexpr int UB = 8;
+            // First wait on this CTA's own columns only (CTAs of a chunk watch different words, as
+            // with the scalar gate), then read every column, by then almost surely complete.
+            {
+                const int own = tm * nj;
+                unsigned it = 0;
+                for (;;) {
+                    bool done = true;
+                    for (int c = threadIdx.x; c < own; c += DK_THREADS) {
+                        const long long v = ld_relaxed_s64(tc + (int64_t)(c / nj) * (r + 1) + j0 + c % nj);
+                        done = done && ((unsigned long long)v & FIX_COUNT_MASK) == want;
+                    }
+                    if (__syncthreads_and(done)) break;
+                    if (++it > SPIN_LIMIT) break;     // the reads below give up and flag it
+                    if (it > 16) __nanosleep(64);
+                }
+            }
+            for (int base = 0; base < tot; base += UB * DK_THREADS) {   // uniform trip count
+                const long long* ptr[UB];
+                bool valid[UB];
+#pragma unroll
+                for (int u = 0; u < UB; ++u) {
+                    const int c = base + (int)threadIdx.x + u * DK_THREADS;
+                    valid[u] = c < tot;
+                    ptr[u] = tc + (valid[u] ? (int64_t)(c / r) * (r + 1) + c % r : 0);
+                }
+                long long tv[UB];
+                unsigned it = 0;
+                for (;;) {
+                    bool done = true;
+#pragma unroll
+                    for (int u = 0; u < UB; ++u) tv[u] = valid[u] ? ld_relaxed_s64(ptr[u]) : 0ll;
+#pragma unroll
+                    for (int u = 0; u < UB; ++u)
+                        done = done && (!valid[u] || ((unsigned long long)tv[u] & FIX_COUNT_MASK) == want);
+                    if (__syncthreads_and(done)) break;
+                    if (++it > SPIN_LIMIT) {
+                        if (threadIdx.x == 0) atomicOr(a.err, 1u);
+#pragma unroll
+                        for (int u = 0; u < UB; ++u) tv[u] = 0ll;
+                        break;
+                    }
+                    if (it > 16) __nanosleep(64);
+                }
+#pragma unroll
+                for (int u = 0; u < UB; ++u) {
+                    const int c = base + (int)threadIdx.x + u * DK_THREADS;
+                    if (valid[u]) mlp_t[(c / r) * (r + 1) + c % r] = __ll2float_rn(tv[u] >> FIX_COUNT_BITS) * (1.0f / FIX_ONE);
+                }
+            }
+            __syncthreads();
+            // One thread per output, token index fastest: the threads of a warp read one or two rows
+            // of W1 (W2) at a time (broadcast loads), and the padded rows of t (h) keep the
+            // shared-memory reads free of bank conflicts.
+            for (int o = threadIdx.x; o < tm * H; o += DK_THREADS) {
+                const int mm = o % tm, i = o / tm;
+                const float* w1 = a.mlp.w1 + (int64_t)i * r;
+                const float* tr = mlp_t + mm * (r + 1);
+                float pre = __ldg(a.mlp.b1 + i);
+#pragma unroll 8
+                for (int j = 0; j < r; ++j) pre = fmaf(__ldg(w1 + j), tr[j], pre);
+                mlp_h[mm * (H + 1) + i] = fmaxf(pre, 0.0f);
+            }
+            __syncthreads();
+            for (int c = threadIdx.x; c < tm * nj; c += DK_THREADS) {
+                const int mm = c % tm, jj = c / tm, j = j0 + jj;
+                const float* w2 = a.mlp.w2 + (int64_t)j * H;
+                const float* hr = mlp_h + mm * (H + 1);
+                float pre = __ldg(a.mlp.b2 + j);
+#pragma unroll 8
+                for (int i = 0; i < H; ++i) pre = fmaf(__ldg(w2 + i), hr[i], pre);
+                us[mm * ujr + jj] = a.mlp.alpha * mlp_t[mm * (r + 1) + j] / (1.0f + expf(-pre));
+            }
+            asm volatile("cp.async.wait_all;" ::: "memory");
+        } else if (nj > 0) {
             const int dmm = DK_THREADS / nj, djj = DK_THREADS % nj;
             int mm = threadIdx.x / nj, jj = threadIdx.x % nj;
             constexpr int UB = 8;         // elements per thread per pass, loads issued together
@@ -611,6 +691,8 @@ __global__ void __launch_bounds__(AP_ROWS) w4ec_apply_kernel(DecodeArgs a) {
     const int r = a.rank;
     uint16_t* Bs = reinterpret_cast<uint16_t*>(dyn_smem);                          // [r][AP_ROWS]
     float* us = reinterpret_cast<float*>(dyn_smem + (size_t)r * AP_ROWS * 2);      // [AP_TOK][r]
+    float* hs = us + AP_TOK * r;                                                   // MLP gate: [AP_TOK][H]
+    const bool mlp = a.mlp.w1 != nullptr;
     __shared__ unsigned s_last;
     const int64_t n0 = (int64_t)blockIdx.x * AP_ROWS;
     const int64_t n = n0 + threadIdx.x;
@@ -645,7 +727,29 @@ __global__ void __launch_bounds__(AP_ROWS) w4ec_apply_kernel(DecodeArgs a) {
             if (c < tk * r) {
                 const float t_ = __ll2float_rn(tv[u] >> FIX_COUNT_BITS) * (1.0f / FIX_ONE);
                 const float p_ = __ll2float_rn(pv[u] >> FIX_COUNT_BITS) * (1.0f / FIX_ONE);
-                us[c] = t_ / (1.0f + expf(-(p_ + a.b_g)));
+                us[c] = mlp ? t_ : t_ / (1.0f + expf(-(p_ + a.b_g)));
+            }
+        }
+        if (mlp) {
+            // Bottleneck-MLP gate: h = relu(W1 t + b1), then u = alpha sigmoid(W2 h + b2) t in place.
+            const int H = a.mlp.hidden;
+            __syncthreads();
+            for (int o = threadIdx.x; o < tk * H; o += AP_ROWS) {
+                const int mm = o % tk, i = o / tk;
+                const float* w1 = a.mlp.w1 + (int64_t)i * r;
+                float pre = __ldg(a.mlp.b1 + i);
+#pragma unroll 8
+                for (int j = 0; j < r; ++j) pre = fmaf(__ldg(w1 + j), us[mm * r + j], pre);
+                hs[mm * (H + 1) + i] = fmaxf(pre, 0.0f);
+            }
+            __syncthreads();
+            for (int c = threadIdx.x; c < tk * r; c += AP_ROWS) {
+                const int mm = c / r, j = c % r;
+                const float* w2 = a.mlp.w2 + (int64_t)j * H;
+                float pre = __ldg(a.mlp.b2 + j);
+#pragma unroll 8
+                for (int i = 0; i < H; ++i) pre = fmaf(__ldg(w2 + i), hs[mm * (H + 1) + i], pre);
+                us[c] = a.mlp.alpha * us[c] / (1.0f + expf(-pre));
             }
         }
         float mv[AP_TOK];
@@ -682,10 +786,12 @@ __global__ void __launch_bounds__(AP_ROWS) w4ec_apply_kernel(DecodeArgs a) {
     }
 }
 
-size_t apply_dyn_smem_bytes(int rank) { return (size_t)rank * AP_ROWS * 2 + (size_t)AP_TOK * rank * 4; }
+size_t apply_dyn_smem_bytes(int rank, int gate_hidden) {
+    return (size_t)rank * AP_ROWS * 2 + (size_t)AP_TOK * rank * 4 + (size_t)AP_TOK * (gate_hidden + 1) * 4;
+}
 
 cudaError_t launch_apply(const DecodeArgs& a, cudaStream_t stream) {
-    const size_t dyn = apply_dyn_smem_bytes(a.rank);
+    const size_t dyn = apply_dyn_smem_bytes(a.rank, a.mlp.w1 ? a.mlp.hidden : 0);
     static size_t opted[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -710,9 +816,10 @@ cudaError_t launch_apply(const DecodeArgs& a, cudaStream_t stream) {
 // ---------------------------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------------------------
-size_t decode_dyn_smem_bytes(int nb, int g, int ec_jr, int rank) {
+size_t decode_dyn_smem_bytes(int nb, int g, int ec_jr, int rank, int gate_hidden) {
     if (rank <= 0) return 0;
-    const size_t gemm = (size_t)ec_jr * 16 * g * 2 + (size_t)8 * nb * (ec_jr + 1) * 4;
+    size_t gemm = (size_t)ec_jr * 16 * g * 2 + (size_t)8 * nb * (ec_jr + 1) * 4;
+    if (gate_hidden > 0) gemm += (size_t)8 * nb * (rank + 1 + gate_hidden + 1) * 4;   // MLP gate: t, hidden rows
     const size_t ec = (size_t)DK_WARPS * 8 * nb * EC_RS * 4;
     return gemm > ec ? gemm : ec;
 }
@@ -731,7 +838,7 @@ template <int NB, int G, int WPW>
 static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     static_assert(WPW * G <= 8, "weight registers");
     const unsigned grid = (unsigned)(a.ec_ctas + a.row_tiles * a.split * a.mchunks);
-    const size_t dyn = decode_dyn_smem_bytes(NB, G, a.ec_jr, a.rank);
+    const size_t dyn = decode_dyn_smem_bytes(NB, G, a.ec_jr, a.rank, a.mlp.w1 ? a.mlp.hidden : 0);
     // Static plus dynamic shared memory above 48 KB needs the opt-in attribute (per device).
     static size_t opted[64] = {0};
     int dev = 0;

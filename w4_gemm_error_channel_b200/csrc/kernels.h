@@ -37,6 +37,18 @@ constexpr int64_t M_MAX = 65536;
 constexpr size_t TC_FLAGS_WORD = CTRL_HEADER_WORDS + 2 * CHUNKS_MAX + CHUNKS_MAX * GROUPS_MAX;
 static_assert(TC_FLAGS_WORD + 2 * TC_BLOCKS_MAX <= CTRL_BYTES / 4, "control block");
 
+// The pages' bottleneck-MLP gate over t = x A: gamma = sigmoid(w2 relu(w1 t + b1) + b2),
+// u = alpha gamma t.  w1 == null selects the scalar gate sigmoid(x w_g + b_g).
+constexpr int GATE_HIDDEN_MAX = 64;
+struct GateMlp {
+    const float* w1;        // [H][r]
+    const float* b1;        // [H]
+    const float* w2;        // [r][H]
+    const float* b2;        // [r]
+    int hidden;             // H
+    float alpha;
+};
+
 struct DecodeArgs {
     const uint16_t* x;      // bf16 [M, K]
     const uint8_t* packed;  // [N, K/2]
@@ -63,6 +75,7 @@ struct DecodeArgs {
     unsigned* consumed;     // [mchunks] level-2 consumer counters
     unsigned* consumed1;    // [mchunks][GROUPS_MAX] level-1 consumer counters
     float* ymain;           // separate EC pass: fp32 main term [M][N] (workspace); null when fused
+    GateMlp mlp;            // bottleneck-MLP gate (w1 == null: the scalar gate)
 };
 
 // Prefill (tcgen05) kernel arguments.
@@ -83,6 +96,7 @@ struct TcArgs {
     unsigned* err;          // error word (bit 2: an mbarrier wait gave up; bit 3: an EC-ready wait gave up)
     unsigned* ec_ready;     // [token blocks] u of the block is ready
     unsigned* ec_consumed;  // [token blocks] main tiles that have seen the flag
+    GateMlp mlp;            // bottleneck-MLP gate (w1 == null: the scalar gate)
 };
 
 // bn: tokens per tile (128 or 256).
@@ -102,8 +116,8 @@ constexpr int64_t EC_K_MAX = 65536;
 int decode_ec_ctas_per_chunk(int64_t K, int rank);
 // Separate EC pass after the decode kernel (it reads DecodeArgs::ymain, tacc, B).
 cudaError_t launch_apply(const DecodeArgs& a, cudaStream_t stream);
-size_t apply_dyn_smem_bytes(int rank);
-size_t decode_dyn_smem_bytes(int nb, int g, int ec_jr, int rank);
+size_t apply_dyn_smem_bytes(int rank, int gate_hidden);
+size_t decode_dyn_smem_bytes(int nb, int g, int ec_jr, int rank, int gate_hidden);
 cudaError_t launch_decode(const DecodeArgs& a, int nb, int g, int wpw, cudaStream_t stream);
 
 }  // namespace spear

@@ -64,6 +64,7 @@ extern "C" spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const vo
     if (y_dtype != SPEAR_BF16 && y_dtype != SPEAR_FP32) return SPEAR_ERR_INVALID_ARG;
     const int32_t rank = ec ? ec->rank : 0;
     if (ec && (!ec->A || !ec->B || !ec->w_g || isnan(ec->b_g))) return SPEAR_ERR_INVALID_ARG;
+    if (ec && ec->gate_w1) return SPEAR_ERR_INVALID_ARG;   // the scalar gate only here
     if (M <= 0 || N <= 0 || K <= 0) return SPEAR_ERR_INVALID_ARG;
     if (M > NOALLOC_M_MAX) return SPEAR_ERR_UNSUPPORTED_SHAPE;       // the scratch is sized for 64 tokens
     if (N % 128 != 0 || K % 64 != 0) return SPEAR_ERR_UNSUPPORTED_SHAPE;
@@ -125,5 +126,6 @@ extern "C" spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const vo
     a.consumed = a.arrivals + CHUNKS_MAX;
     a.consumed1 = a.consumed + CHUNKS_MAX;
     a.ymain = nullptr;                                    // the compensator stays fused here
+    a.mlp = GateMlp{};                                    // the scalar gate
     return launch_decode(a, nb, p.tile_n / 16, wpw_of(ksl), s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
 }

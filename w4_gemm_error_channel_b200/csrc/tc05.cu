@@ -183,6 +183,9 @@ struct TcSmem {
     static constexpr uint32_t TMEM_COLS = NEED <= 32 ? 32 : NEED <= 64 ? 64 : NEED <= 128 ? 128 : NEED <= 256 ? 256 : 512;
     // Two CTAs share an SM when both fit (shared memory and TMEM): one tile's prologue and
     // epilogue then overlap the other's MMAs.
+    // The EC tile with the MLP gate stages t [128][r + 1 <= 129] and h [128][H + 1 <= 65] in fp32
+    // from X_OFF.
+    static_assert(WG_OFF - X_OFF >= 128 * 129 * 4 + 128 * 65 * 4, "MLP-gate staging fits in the stages");
     static constexpr int MIN_BLOCKS = (TOTAL <= 112 * 1024 && TMEM_COLS <= 256) ? 2 : 1;
 };
 constexpr int TC_EB = 128;               // tokens per EC tile
@@ -421,6 +424,43 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         if (!acc_ok) atomicOr(a.err, 4u);
         tc_fence_after();
         if (is_ec) {
+            if (a.mlp.w1 != nullptr) {
+                // Bottleneck-MLP gate: t is staged as [token][j] in the idle stages, then thread row
+                // takes token m0 + row: h = relu(W1 t + b1), u[m, j] = alpha sigmoid(W2 h + b2)_j t_j.
+                const int r = a.rank, H = a.mlp.hidden;
+                // Odd row strides: each thread walks its own row, so rows must start in different banks.
+                const int rs = r + 1, hsd = H + 1;
+                float* ts = reinterpret_cast<float*>(smem + L::X_OFF);            // [TC_EB][r + 1]
+                float* hs = ts + TC_EB * rs;                                       // [TC_EB][H + 1]
+                for (int c0 = 0; c0 < TC_EB; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tmem_d + lane_base + (uint32_t)c0, v);
+                    if (row < r) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) ts[(c0 + i) * rs + row] = v[i];
+                    }
+                }
+                named_bar_epi();
+                const int64_t m = m0 + row;
+                if (acc_ok && m < a.M) {
+                    const float* tr = ts + row * rs;
+                    float* hr = hs + row * hsd;
+                    for (int i = 0; i < H; ++i) {
+                        const float* w1 = a.mlp.w1 + (int64_t)i * r;
+                        float pre = __ldg(a.mlp.b1 + i);
+#pragma unroll 8
+                        for (int j = 0; j < r; ++j) pre = fmaf(__ldg(w1 + j), tr[j], pre);
+                        hr[i] = fmaxf(pre, 0.0f);
+                    }
+                    for (int j = 0; j < r; ++j) {
+                        const float* w2 = a.mlp.w2 + (int64_t)j * H;
+                        float pre = __ldg(a.mlp.b2 + j);
+#pragma unroll 8
+                        for (int i = 0; i < H; ++i) pre = fmaf(__ldg(w2 + i), hr[i], pre);
+                        a.u[m * r + j] = __float2bfloat16_rn(a.mlp.alpha * tr[j] / (1.0f + expf(-pre)));
+                    }
+                }
+            } else {
             // g[m] = sigmoid(p[m] + b_g); u[m, j] = g[m] t[j, m] for j = row < r, as bf16.
             s_gate[row] = 1.0f / (1.0f + expf(-(pg + a.b_g)));
             named_bar_epi();
@@ -434,6 +474,7 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                     const int64_t m = m0 + c0 + i;
                     if (m < a.M) a.u[m * a.rank + j] = __float2bfloat16_rn(s_gate[c0 + i] * v[i]);
                 }
+            }
             }
             asm volatile("fence.proxy.async.global;" ::: "memory");   // u is read by other CTAs' TMA
             __threadfence();
