@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--sweep", action="store_true",
                     help="time every valid decode tiling for the workload's batches and print a table")
+    ap.add_argument("--batches", default="", metavar="M1,M2,..",
+                    help="with --sweep: time only these batch sizes of the workload")
     ap.add_argument("--once", type=int, default=0, metavar="M",
                     help="run 5 layer calls of the workload with M tokens and exit (for profilers)")
     ap.add_argument("--no-ec", action="store_true", help="with --once: the plain W4 layer")
@@ -447,8 +449,15 @@ def prefill_summary(torch, spear):
     x = torch.from_numpy(L.x(M).view(np.int16)).to(dev).view(torch.bfloat16)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     res = {}
-    for use_ec in (True, False):
+    for variant in ("ec", "no_ec", "ec_semifused"):
+        use_ec = variant != "no_ec"
         plan = spear.spear_gemm_plan(M, N, K, r if use_ec else 0)
+        if variant == "ec_semifused":
+            # The same tiling with the compensator as its own kernels beside the GEMM.
+            plan.kernel_id, plan.split_k, plan.flags = spear.SPEAR_KERNEL_TC05, 1, spear.SPEAR_PLAN_SEPARATE_EC
+            if plan.tile_n not in (128, 256):
+                plan.tile_n, plan.tile_m = 128, 256
+            spear.spear_plan_update(plan, M, N, K, r)
         ws = spear.alloc_workspace(plan.workspace_bytes)
         stream = torch.cuda.Stream()
 
@@ -470,11 +479,11 @@ def prefill_summary(torch, spear):
             e1.record(stream)
         e1.synchronize()
         t = e0.elapsed_time(e1) / 1e3 / n
-        res["ec" if use_ec else "no_ec"] = {"us": t * 1e6,
-                                            "TFLOPs": layer_flops(M, N, K, r if use_ec else 0) / t / 1e12,
-                                            "plan": {"kernel": plan.kernel_id, "tile_n": plan.tile_n,
-                                                     "split_k": plan.split_k}}
+        res[variant] = {"us": t * 1e6, "TFLOPs": layer_flops(M, N, K, r if use_ec else 0) / t / 1e12,
+                        "plan": {"kernel": plan.kernel_id, "tile_n": plan.tile_n, "tile_m": plan.tile_m,
+                                 "split_k": plan.split_k, "flags": plan.flags}}
     res["ec_overhead"] = res["ec"]["us"] / res["no_ec"]["us"] - 1.0
+    res["ec_semifused_overhead"] = res["ec_semifused"]["us"] / res["no_ec"]["us"] - 1.0
     return res
 
 
@@ -490,6 +499,8 @@ def sweep_plans(args):
     else:
         cfg, batches, kind = WORKLOADS[args.workload]
         shapes = config_layers(cfg, M=max(batches))[:1]
+    if args.batches:
+        batches = [int(b) for b in args.batches.split(",")]
     rows = []
     for L in shapes:
         rows += _sweep_shape(torch, spear, L, batches)
@@ -508,13 +519,16 @@ def _sweep_shape(torch, spear, L, batches):
         x = torch.from_numpy(L.x(M).view(np.int16)).to(dev).view(torch.bfloat16)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         base = spear.spear_gemm_plan(M, N, K, r)
-        # Room for the tcgen05 kernel's u buffer (bf16 [M, r]) whatever the default plan is.
-        ws = spear.alloc_workspace(base.workspace_bytes + (M * r * 2 + 255) // 256 * 256 + min(M, 256) * N * 4)
-        # (kernel, tile_n, split_k, flags): every split-K decode tiling, fused and with the separate
-        # EC pass, and the tcgen05 kernel with 128-token tiles.
+        # Room for the tcgen05 kernel's u buffer (bf16 [M, r]) and the fp32 main term of the
+        # separate EC pass ([min(M, 256), N]) or of the semi-fused prefill path ([M, N]).
+        ws = spear.alloc_workspace(base.workspace_bytes + (M * r * 2 + 255) // 256 * 256 + M * N * 4)
+        # (kernel, tile_n, split_k, flags[, tile_m]): every split-K decode tiling, fused and with the
+        # separate EC pass, and the tcgen05 kernel with 128- or 256-token tiles, fused and
+        # semi-fused (flags 1).
         candidates = [] if M >= 1024 else [(1, tile_n, split, fl) for tile_n in (16, 32, 64, 128)
                                            for split in (1, 2, 4, 8) for fl in (0, 1)]
-        candidates += [(2, 128, 1, 0, 128)] + ([(2, 128, 1, 0, 256)] if M >= 256 else [])
+        for fl in ((0, 1) if M >= 128 else (0,)):
+            candidates += [(2, 128, 1, fl, 128)] + ([(2, 128, 1, fl, 256)] if M >= 256 else [])
         for cand in candidates:
                 kernel_id, tile_n, split, fl = cand[:4]
                 tc_tile_m = cand[4] if len(cand) > 4 else None

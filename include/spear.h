@@ -68,11 +68,17 @@ typedef enum {
 
 /* spear_plan.flags bits. */
 enum {
-    /* Split-K decode kernel only: the weight-streaming CTAs write their fp32 main term to the
+    /* The compensator leaves the GEMM's epilogue (section 2.2A); ignored without a compensator.
+     * Split-K decode kernel: the weight-streaming CTAs write their fp32 main term to the
      * workspace and a second kernel, chained by programmatic dependent launch, applies the
-     * compensator (section 2.2A's "split-K kernel with a separate EC pass").  It spares the
-     * weight-streaming CTAs the wait for the compensator, which matters when their grid takes
-     * several waves. */
+     * compensator (the "split-K kernel with a separate EC pass").  It spares the weight-streaming
+     * CTAs the wait for the compensator, which matters when their grid takes several waves.
+     * Prefill kernel: the semi-fused path.  The EC tiles run alone on a side stream of the
+     * library (highest priority; one per device, created on first use) beside the main tiles on
+     * the caller's stream, which write the fp32 main term [M][N] to the workspace; after both, a
+     * third kernel adds u B and rounds y.  The call forks and joins through events, so a CUDA
+     * graph captured from the caller's stream holds the two as parallel branches (a static DAG).
+     * Concurrent calls from several host threads are ordered by a lock around the enqueue. */
     SPEAR_PLAN_SEPARATE_EC = 1
 };
 
@@ -153,6 +159,18 @@ SPEAR_API spear_status spear_debug_unpack_w4(const void* packed, const void* zer
  */
 SPEAR_API spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int device,
                              spear_plan* out);
+
+/*
+ * spear_plan_update -- check a plan whose fields the caller has changed (kernel, tiling, flags)
+ * for this shape and recompute plan->workspace_bytes in place.  The semi-fused prefill path
+ * (SPEAR_KERNEL_TC05 with SPEAR_PLAN_SEPARATE_EC and a compensator), for one, needs M * N * 4
+ * more bytes than the fused one.  Host only; launches nothing.
+ *
+ *   plan       host, in/out
+ * Returns SPEAR_ERR_INVALID_ARG for a NULL plan or a field the kernels do not support, and
+ * SPEAR_ERR_UNSUPPORTED_SHAPE as spear_gemm_plan does; the plan is unchanged then.
+ */
+SPEAR_API spear_status spear_plan_update(spear_plan* plan, int64_t M, int64_t N, int64_t K, int32_t rank);
 
 /*
  * spear_w4ec_gemm -- y = x dequant(Wq)^T + g(x) * ((x A) B)  (section 2.1A).

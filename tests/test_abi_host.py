@@ -116,8 +116,8 @@ def test_gemm_rejects_bad_plans():
         setattr(q, field, val)
         assert _gemm(plan=ctypes.byref(q)) == INVALID, field
     # tcgen05 plans: 256 weight rows only with 128-token tiles; token widths 128, 160, 192, 256.
-    # Plan flags: only SPEAR_PLAN_SEPARATE_EC (1), and only on the split-K decode kernel.
-    for kid, fl in ((1, 2), (1, 3), (2, 1)):
+    # Plan flags: only SPEAR_PLAN_SEPARATE_EC (1).
+    for kid, fl in ((1, 2), (1, 3), (2, 2), (2, 3)):
         q = spear.spear_plan.from_buffer_copy(p)
         q.kernel_id, q.flags = kid, fl
         if kid == 2:
@@ -147,3 +147,55 @@ def test_prepared_layer_rejects_host_tensors():
     with pytest.raises(ValueError):
         spear.W4ECLayer(torch.zeros((128, 32), dtype=torch.uint8), torch.zeros(128, dtype=torch.float16),
                         torch.zeros(128, dtype=torch.float16))
+
+
+def test_mlp_gate_host_checks():
+    # The optional bottleneck-MLP gate: all four arrays or none, 1 <= H <= 64, 16-byte aligned,
+    # alpha not NaN; the no-allocation entry point takes the scalar gate only.  Fake, never
+    # dereferenced addresses: every case is decided on the host.
+    def ec(**kw):
+        e = spear.spear_ec(0x7000, 0x8000, 0x9000, 0.0, 16)
+        e.gate_w1, e.gate_b1, e.gate_w2, e.gate_b2, e.gate_hidden, e.alpha = 0xA000, 0xB000, 0xC000, 0xD000, 8, 1.0
+        for k, v in kw.items():
+            setattr(e, k, v)
+        return e
+    for kw, want in (({"gate_b1": 0}, INVALID), ({"gate_w2": 0}, INVALID), ({"gate_hidden": 0}, INVALID),
+                     ({"gate_hidden": 65}, INVALID), ({"alpha": math.nan}, INVALID), ({"gate_w1": 0xA004}, MISALIGNED),
+                     ({"gate_b2": 0xD008}, MISALIGNED)):
+        e = ec(**kw)
+        assert _gemm(ec=ctypes.byref(e)) == want, kw
+    e = ec()
+    P = ctypes.c_void_p
+    assert spear._lib.spear_w4ec_gemm_noalloc(None, P(0x1000), 4, 512, 512, P(0x2000), P(0x3000), P(0x4000),
+                                              ctypes.byref(e), P(0x5000), 0, None) == INVALID
+
+
+def test_plan_update_and_semifused_workspace():
+    # The semi-fused prefill plan (tcgen05 kernel + SPEAR_PLAN_SEPARATE_EC) keeps the fp32 main
+    # term [M][N] in the workspace after u (bf16 [M][r], padded to 256 bytes).
+    M, N, K, r = 300, 512, 512, 16
+    st, p = _plan(M, N, K, r)
+    assert st == OK
+    q = spear.spear_plan.from_buffer_copy(p)
+    q.kernel_id, q.tile_n, q.split_k, q.tile_m, q.flags = 2, 128, 1, 128, 0
+    assert spear._lib.spear_plan_update(ctypes.byref(q), M, N, K, r) == OK
+    fused = q.workspace_bytes
+    assert fused == (128 + 1024) * 1024 + (M * r * 2 + 255) // 256 * 256
+    q.flags = spear.SPEAR_PLAN_SEPARATE_EC
+    assert spear._lib.spear_plan_update(ctypes.byref(q), M, N, K, r) == OK
+    assert q.workspace_bytes == fused + M * N * 4
+    ec = spear.spear_ec(0x7000, 0x8000, 0x9000, 0.0, r)
+    assert _gemm(M=M, N=N, K=K, ec=ctypes.byref(ec), plan=ctypes.byref(q), ws_bytes=q.workspace_bytes - 1) == WS_SMALL
+    # Without a compensator the flag changes nothing.
+    assert spear._lib.spear_plan_update(ctypes.byref(q), M, N, K, 0) == OK
+    assert q.workspace_bytes == (128 + 1024) * 1024
+    # Bad fields and shapes are refused and leave the plan as it was.
+    before = bytes(q)
+    q2 = spear.spear_plan.from_buffer_copy(q)
+    q2.flags = 2
+    assert spear._lib.spear_plan_update(ctypes.byref(q2), M, N, K, r) == INVALID
+    assert spear._lib.spear_plan_update(ctypes.byref(q), M, 500, K, r) == SHAPE
+    assert spear._lib.spear_plan_update(None, M, N, K, r) == INVALID
+    assert bytes(q) == before
+    with pytest.raises(spear.SpearError):
+        spear.spear_plan_update(q2, M, N, K, r)

@@ -26,7 +26,7 @@ SPEAR_PLAN_SEPARATE_EC = 1
 STATUS_NAMES = {0: "SPEAR_OK", 1: "SPEAR_ERR_INVALID_ARG", 2: "SPEAR_ERR_UNSUPPORTED_SHAPE",
                 3: "SPEAR_ERR_MISALIGNED", 4: "SPEAR_ERR_WORKSPACE_TOO_SMALL", 5: "SPEAR_ERR_CUDA",
                 6: "SPEAR_ERR_TIMEOUT"}
-EXPORTED = ["spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_w4ec_gemm",
+EXPORTED = ["spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_plan_update", "spear_w4ec_gemm",
             "spear_w4ec_gemm_noalloc", "spear_get_device_status", "spear_status_string", "spear_version"]
 
 
@@ -43,7 +43,7 @@ class spear_plan(ctypes.Structure):
 
     def __repr__(self):
         return (f"spear_plan(kernel_id={self.kernel_id}, tile_n={self.tile_n}, split_k={self.split_k}, "
-                f"tile_m={self.tile_m}, workspace_bytes={self.workspace_bytes})")
+                f"tile_m={self.tile_m}, flags={self.flags}, workspace_bytes={self.workspace_bytes})")
 
 
 class spear_ec(ctypes.Structure):
@@ -62,6 +62,7 @@ def _load():
     lib.spear_pack_w4.argtypes = [P, ctypes.c_int, I64, I64, P, P, P, P]
     lib.spear_debug_unpack_w4.argtypes = [P, P, I64, I64, P, P, P]
     lib.spear_gemm_plan.argtypes = [I64, I64, I64, ctypes.c_int32, ctypes.c_int, ctypes.POINTER(spear_plan)]
+    lib.spear_plan_update.argtypes = [ctypes.POINTER(spear_plan), I64, I64, I64, ctypes.c_int32]
     lib.spear_w4ec_gemm.argtypes = [ctypes.POINTER(spear_plan), P, I64, I64, I64, P, P, P,
                                     ctypes.POINTER(spear_ec), P, ctypes.c_int, P, ctypes.c_size_t, P]
     lib.spear_w4ec_gemm_noalloc.argtypes = [ctypes.POINTER(spear_plan), P, I64, I64, I64, P, P, P,
@@ -70,7 +71,7 @@ def _load():
     lib.spear_status_string.argtypes = [ctypes.c_int]
     lib.spear_status_string.restype = ctypes.c_char_p
     lib.spear_version.restype = ctypes.c_int
-    for fn in ("spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_w4ec_gemm",
+    for fn in ("spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_plan_update", "spear_w4ec_gemm",
                "spear_w4ec_gemm_noalloc", "spear_get_device_status"):
         getattr(lib, fn).restype = ctypes.c_int
     return lib
@@ -184,6 +185,12 @@ def spear_debug_unpack_w4(packed: torch.Tensor, zero: torch.Tensor, K: int, want
 def spear_gemm_plan(M: int, N: int, K: int, rank: int = 0, device: int = -1) -> spear_plan:
     plan = spear_plan()
     _check("spear_gemm_plan", _lib.spear_gemm_plan(M, N, K, rank, device, ctypes.byref(plan)))
+    return plan
+
+
+def spear_plan_update(plan: spear_plan, M: int, N: int, K: int, rank: int = 0) -> spear_plan:
+    """Checks a plan whose fields were changed and recomputes its workspace_bytes (in place)."""
+    _check("spear_plan_update", _lib.spear_plan_update(ctypes.byref(plan), M, N, K, rank))
     return plan
 
 

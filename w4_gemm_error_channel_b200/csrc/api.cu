@@ -72,11 +72,16 @@ int ec_jr_for(int32_t rank, int64_t S) {
     if (rank <= 0) return 0;
     return (int)(((rank + S - 1) / S + 3) / 4 * 4);
 }
+// u of the prefill kernel, bf16 [M][r], padded to 256 bytes.
+size_t tc05_u_bytes(int64_t M, int32_t rank) { return ((size_t)M * rank * 2 + 255) / 256 * 256; }
+
 // Workspace: the zeroed prefix (control block + EC accumulators); split-K partial sums meet in
 // distributed shared memory.  The prefill kernel with a compensator also keeps u (bf16 [M][r]).
 size_t workspace_bytes_for(const spear_plan& p, int64_t M, int64_t N_for_ws, int32_t rank) {
     size_t b = ZEROED_BYTES;
-    if (p.kernel_id == SPEAR_KERNEL_TC05 && rank > 0) b += ((size_t)M * rank * 2 + 255) / 256 * 256;
+    if (p.kernel_id == SPEAR_KERNEL_TC05 && rank > 0) b += tc05_u_bytes(M, rank);
+    if (p.kernel_id == SPEAR_KERNEL_TC05 && (p.flags & SPEAR_PLAN_SEPARATE_EC) && rank > 0)
+        b += (size_t)M * N_for_ws * 4;                                              // fp32 main term
     if (p.kernel_id == SPEAR_KERNEL_SPLITK && (p.flags & SPEAR_PLAN_SEPARATE_EC) && rank > 0)
         b += (size_t)(M < LAUNCH_TOKENS_MAX ? M : LAUNCH_TOKENS_MAX) * N_for_ws * 4;   // fp32 main term
     return b;
@@ -190,7 +195,7 @@ bool use_tc05(int64_t M, int32_t rank) { return M >= TC05_MIN_M && rank <= TC05_
 spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K, int32_t rank) {
     (void)M;
     if (p.kernel_id == SPEAR_KERNEL_TC05) {
-        if (rank > TC05_MAX_RANK || p.flags != 0) return SPEAR_ERR_INVALID_ARG;
+        if (rank > TC05_MAX_RANK || (p.flags & ~SPEAR_PLAN_SEPARATE_EC)) return SPEAR_ERR_INVALID_ARG;
         if ((M + p.tile_m - 1) / p.tile_m > (int64_t)TC_BLOCKS_MAX) return SPEAR_ERR_INVALID_ARG;
         if (p.split_k != 1 || !(p.tile_m == 128 || p.tile_m == 160 || p.tile_m == 192 || p.tile_m == 256))
             return SPEAR_ERR_INVALID_ARG;
@@ -271,6 +276,16 @@ spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int 
     return SPEAR_OK;
 }
 
+spear_status spear_plan_update(spear_plan* plan, int64_t M, int64_t N, int64_t K, int32_t rank) {
+    if (!plan) return SPEAR_ERR_INVALID_ARG;
+    spear_status st = check_shape(M, N, K, rank);
+    if (st != SPEAR_OK) return st;
+    st = validate_plan(*plan, M, N, K, rank);
+    if (st != SPEAR_OK) return st;
+    plan->workspace_bytes = workspace_bytes_for(*plan, M, N, rank);
+    return SPEAR_OK;
+}
+
 spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, int64_t N, int64_t K,
                              const void* packed, const void* scale, const void* zero, const spear_ec* ec, void* y,
                              spear_dtype y_dtype, void* workspace, size_t workspace_bytes, void* stream) {
@@ -330,7 +345,13 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         t.err = ctrl;
         t.ec_ready = ctrl + TC_FLAGS_WORD;
         t.ec_consumed = t.ec_ready + TC_BLOCKS_MAX;
-        return launch_tc05(t, p.tile_m, p.tile_n, s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
+        t.ec_only = 0;
+        cudaError_t e;
+        if (rank > 0 && (p.flags & SPEAR_PLAN_SEPARATE_EC))
+            e = launch_semifused(t, p.tile_m, p.tile_n, (float*)(ws + ZEROED_BYTES + tc05_u_bytes(M, rank)), s);
+        else
+            e = launch_tc05(t, p.tile_m, p.tile_n, s);
+        return e == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
     }
     const int nb = nb_for_tile_m(p.tile_m);
     const int g = p.tile_n / 16;

@@ -22,8 +22,9 @@ namespace spear {
 //     [.., +TC_BLOCKS)        prefill kernel: flag consumer counters
 //   EC accumulators, TACC_BYTES: int64 [tokens of a launch][r + 1] (t, then the gate
 //   pre-activation), fixed point with 32 fraction bits above an 8-bit count of the K slices added.
-// After the zeroed part: the prefill kernel's u (bf16 [M][r]) or the separate EC pass's fp32
-// main term ([tokens of a launch][N]).
+// After the zeroed part: the prefill kernel's u (bf16 [M][r], padded to 256 bytes), then, on
+// the semi-fused prefill path, its fp32 main term ([M][N]); or the decode kernel's separate EC
+// pass's fp32 main term ([tokens of a launch][N]).
 constexpr size_t CTRL_BYTES = 128 * 1024;
 constexpr size_t CTRL_HEADER_WORDS = 64;
 constexpr size_t CHUNKS_MAX = 32;                          // token chunks per launch (>= 8 tokens each)
@@ -97,11 +98,16 @@ struct TcArgs {
     unsigned* ec_ready;     // [token blocks] u of the block is ready
     unsigned* ec_consumed;  // [token blocks] main tiles that have seen the flag
     GateMlp mlp;            // bottleneck-MLP gate (w1 == null: the scalar gate)
+    int ec_only;            // 1: launch the EC tiles alone (u only, no ready flags); 0: the whole layer
 };
 
-// bn: tokens per tile (128 or 256).
-// bn = tokens per tile; rows = weight rows per tile (128, or 256 with bn = 128).
-cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream);
+// bn = tokens per tile; rows = weight rows per tile (128, or 256 with bn = 128).  pdl: launch as a
+// programmatic dependent of the previous kernel in the stream; priority: 0 or a launch priority.
+cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream, bool pdl = true, int priority = 0);
+
+// Semi-fused prefill: the EC tiles alone on a side stream of the library, beside the main tiles
+// (fp32 main term into ymain [M][N]) on the caller's stream, joined by ec_up_add (y = ymain + u B).
+cudaError_t launch_semifused(const TcArgs& a, int bn, int rows, float* ymain, cudaStream_t stream);
 
 cudaError_t launch_pack_w4(const void* W, bool w_is_bf16, int64_t N, int64_t K, void* packed, void* scale,
                            void* zero, cudaStream_t stream);

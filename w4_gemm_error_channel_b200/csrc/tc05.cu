@@ -479,7 +479,9 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             asm volatile("fence.proxy.async.global;" ::: "memory");   // u is read by other CTAs' TMA
             __threadfence();
             named_bar_epi();
-            if (row == 0 && acc_ok) asm volatile("st.release.gpu.global.u32 [%0], 1;" ::"l"(&a.ec_ready[mb]) : "memory");
+            // EC tiles launched alone (the semi-fused path) have no main tiles to signal.
+            if (row == 0 && acc_ok && !a.ec_only)
+                asm volatile("st.release.gpu.global.u32 [%0], 1;" ::"l"(&a.ec_ready[mb]) : "memory");
         } else {
             // y[m, n] = s[n] D[n, m] (+ E[n, m]), sub-tile by sub-tile.  bf16 output: the tile is
             // staged in the (now idle) x stages as y[m][n] rows and leaves in one TMA store,
@@ -561,7 +563,7 @@ static bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
 }
 
 template <int BN, int STAGES, int SUB>
-static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
+static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream, bool pdl, int priority) {
     using L = TcSmem<BN, STAGES, SUB>;
     CUtensorMap mx, mw, ma, mb, mu, mg, mx128;
     if (!make_map_2d(&mx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.K, (uint64_t)a.M, TC_BK, BN,
@@ -608,27 +610,36 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream) {
     }
     const unsigned mblocks = (unsigned)((a.M + BN - 1) / BN);
     const unsigned eblocks = (unsigned)((a.M + TC_EB - 1) / TC_EB);
-    const unsigned tiles = (unsigned)(a.N / (TC_BM * SUB)) * mblocks + (has_ec ? eblocks : 0u);
+    const unsigned tiles = a.ec_only ? eblocks : (unsigned)(a.N / (TC_BM * SUB)) * mblocks + (has_ec ? eblocks : 0u);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles);
     cfg.blockDim = dim3(TC_THREADS);
     cfg.dynamicSmemBytes = L::TOTAL;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    unsigned na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (priority != 0) {
+        attr[na].id = cudaLaunchAttributePriority;
+        attr[na].val.priority = priority;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, w4_tc05_kernel<BN, STAGES, SUB>, mx, mw, ma, mb, mu, mg, mx128, my, a);
 }
 
-cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream) {
-    if (rows == 256) return bn == 128 ? launch_tc_t<128, 4, 2>(a, stream) : cudaErrorInvalidValue;
+cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream, bool pdl, int priority) {
+    if (rows == 256) return bn == 128 ? launch_tc_t<128, 4, 2>(a, stream, pdl, priority) : cudaErrorInvalidValue;
     if (rows != 128) return cudaErrorInvalidValue;
-    if (bn == 128) return launch_tc_t<128, 3, 1>(a, stream);
-    if (bn == 160) return launch_tc_t<160, 4, 1>(a, stream);
-    if (bn == 192) return launch_tc_t<192, 3, 1>(a, stream);
-    if (bn == 256) return launch_tc_t<256, 4, 1>(a, stream);
+    if (bn == 128) return launch_tc_t<128, 3, 1>(a, stream, pdl, priority);
+    if (bn == 160) return launch_tc_t<160, 4, 1>(a, stream, pdl, priority);
+    if (bn == 192) return launch_tc_t<192, 3, 1>(a, stream, pdl, priority);
+    if (bn == 256) return launch_tc_t<256, 4, 1>(a, stream, pdl, priority);
     return cudaErrorInvalidValue;
 }
 
