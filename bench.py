@@ -65,6 +65,9 @@ def parse():
     ap.add_argument("--model-sweep", action="store_true",
                     help="the 16-layer sweep workload (hidden 2048, MLP 8192, EC r=32 on layers 0, 1, 7, 15): "
                          "all 64 linears of one pass per batch size, with the dispatcher's plans")
+    ap.add_argument("--slo-check", action="store_true",
+                    help="SLO-constrained prefill chunk picker on the 16-layer model: picked chunk, predicted "
+                         "and measured step time per ITL target")
     ap.add_argument("--gate-compare", action="store_true",
                     help="time the layer with the scalar gate and with the bottleneck-MLP gate (H=16) on "
                          "decode-qo M=16 and the prefill layer")
@@ -653,19 +656,12 @@ def svd_demo(args):
                                    "ranks": rows}}))
 
 
-def model_sweep(args):
-    """Config 4: one pass over the 64 linears of the 16-layer model (qkv, o, up+gate, down per
-    layer; compensators of rank 32 on layers 0, 1, 7, 15) for M in {1, 16, 256, 4096}, each call
-    planned by spear_gemm_plan.  Weights are distinct per linear (512 MiB of W4 in all, > 2x L2);
-    each linear reads a synthetic x of its K.  Timed as a CUDA graph of the whole pass."""
-    import torch
-    import w4_gemm_error_channel_b200 as spear
+def _sweep_model(torch, spear, Mmax):
+    """The 16-layer model of config 4 on the device: (N, K, rank, W4ECLayer) per linear in model
+    order (distinct W4 weights per linear, 512 MiB in all), and synthetic x per K, y per N."""
     from synthetic import make_layer
     from synthetic.workloads import SWEEP_EC_LAYERS, SWEEP_LAYERS, SWEEP_LINEARS, SWEEP_RANK
-    torch.cuda.set_device(0)
     dev = torch.device("cuda")
-    batches = [1, 16, 256, 4096]
-    Mmax = max(batches)
     bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
     linears = []
     for layer in range(SWEEP_LAYERS):
@@ -681,6 +677,87 @@ def model_sweep(args):
     xs = {K: bf(make_layer(f"x{K}", 1004 + K, Mmax, 128, K, 0, outlier_frac=0.01, outlier_scale=20.0).x_bits)
           for K in sorted({K for (_, K, _, _) in linears})}
     ys = {N: torch.empty((Mmax, N), dtype=torch.bfloat16, device=dev) for N in sorted({N for (N, _, _, _) in linears})}
+    return linears, xs, ys
+
+
+def _time_calls(torch, stream, calls, reps):
+    """Device time (s) of one run of `calls` (a list of thunks), captured as one CUDA graph."""
+    def run():
+        for c in calls:
+            c()
+    with torch.cuda.stream(stream):
+        run()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            run()
+    for _ in range(2):
+        g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    e1.synchronize()
+    del g
+    return e0.elapsed_time(e1) / 1e3 / reps
+
+
+def slo_check(args):
+    """The SLO-constrained chunk picker on the 16-layer model of config 4 with 16 decode tokens:
+    for each ITL target, the chunk picked from a latency table, the predicted step time and the
+    device time of the real step (one CUDA graph of all 64 linears on 16 + chunk tokens).  Two
+    tables: the built-in one (each shape's calls measured on their own) and one measured inside
+    this model (per linear type, its calls in model order on this model's weights)."""
+    import torch
+    import w4_gemm_error_channel_b200 as spear
+    torch.cuda.set_device(0)
+    D, Mmax, granule = 16, 4096, 128
+    linears, xs, ys = _sweep_model(torch, spear, Mmax)
+    stream = torch.cuda.Stream()
+    types = {}
+    for (N, K, rank, lay) in linears:
+        types.setdefault((N, K, rank), []).append(lay)
+    desc = [(N, K, rank, len(lays)) for (N, K, rank), lays in sorted(types.items())]
+
+    def step_us(M):
+        calls = [(lambda lay=lay, N=N, K=K: lay(xs[K][:M], y=ys[N][:M], stream=stream)) for (N, K, _, lay) in linears]
+        return _time_calls(torch, stream, calls, 10 if M <= 512 else 3) * 1e6
+
+    lut = []
+    for M in (16, 144, 528, 1040, 2064, 4096):
+        for (N, K, rank), lays in sorted(types.items()):
+            calls = [(lambda lay=lay, N=N, K=K: lay(xs[K][:M], y=ys[N][:M], stream=stream)) for lay in lays]
+            t = _time_calls(torch, stream, calls, 10 if M <= 512 else 3)
+            lut.append((M, N, K, int(rank > 0), t * 1e6 / len(lays)))
+    rows = []
+    for table, tname in ((None, "built-in"), (lut, "in-model")):
+        for slo in (1000.0, 2000.0, 4000.0, 8000.0, 12000.0):
+            chunk, pred = spear.spear_pick_prefill_chunk(desc, D, Mmax - D, slo, granule=granule, lut=table)
+            meas = step_us(D + chunk)
+            nxt = step_us(D + chunk + granule) if D + chunk + granule <= Mmax else None
+            rows.append({"table": tname, "slo_us": slo, "chunk": chunk, "predicted_us": pred, "measured_us": meas,
+                         "meets_slo": meas <= slo, "next_chunk_measured_us": nxt})
+    print(json.dumps({"slo_check": {"workload": "16 layers x (qkv 6144x2048, o 2048x2048, up 16384x2048, "
+                                                "down 2048x8192), EC r=32 on layers 0, 1, 7, 15, 16 decode tokens, "
+                                                f"chunk granule {granule}, synthetic",
+                                    "in_model_table": lut, "picks": rows}}))
+
+
+def model_sweep(args):
+    """Config 4: one pass over the 64 linears of the 16-layer model (qkv, o, up+gate, down per
+    layer; compensators of rank 32 on layers 0, 1, 7, 15) for M in {1, 16, 256, 4096}, each call
+    planned by spear_gemm_plan.  Weights are distinct per linear (512 MiB of W4 in all, > 2x L2);
+    each linear reads a synthetic x of its K.  Timed as a CUDA graph of the whole pass."""
+    import torch
+    import w4_gemm_error_channel_b200 as spear
+    torch.cuda.set_device(0)
+    batches = [1, 16, 256, 4096]
+    Mmax = max(batches)
+    linears, xs, ys = _sweep_model(torch, spear, Mmax)
     peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
         os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
     hbm = peaks.get("hbm_gbs", 6650.0)
@@ -801,6 +878,9 @@ def main():
         return
     if args.once:
         run_once(args)
+        return
+    if args.slo_check:
+        slo_check(args)
         return
     if args.sweep:
         sweep_plans(args)

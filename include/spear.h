@@ -231,6 +231,62 @@ SPEAR_API spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const voi
  */
 SPEAR_API spear_status spear_get_device_status(void* workspace, int clear, void* stream);
 
+/*
+ * EC-aware, SLO-constrained prefill chunk picker (section 2.2C): the largest prefill chunk whose
+ * predicted step latency meets the inter-token-latency target, from tables of measured kernel
+ * latencies.  Host only; nothing here touches a GPU.
+ *
+ * A step runs every linear of the model once on M = decode_tokens + chunk tokens.  Predicted step
+ * latency = fixed_us + sum_i count_i * T(M, N_i, K_i, rank_i > 0), where T reads the latency table:
+ * for one (N, K, compensator or not) its samples are made nondecreasing in M, then interpolated
+ * linearly between measured M, held at the smallest measured M below it, and scaled by
+ * M / M_max above the largest.  The step latency is therefore nondecreasing in M.
+ */
+typedef struct {
+    int64_t N, K;       /* the linear's W [N, K] */
+    int32_t rank;       /* its compensator's rank; 0 = none (where compensators sit is what the
+                           picker adapts to) */
+    int32_t count;      /* how many linears of this shape and rank one step runs (>= 0) */
+} spear_linear_desc;
+
+typedef struct {
+    int64_t M, N, K;    /* tokens and weight shape of one call */
+    int32_t has_ec;     /* nonzero: with a compensator */
+    int32_t reserved;
+    double us;          /* device time of one call, microseconds */
+} spear_latency_entry;
+
+/*
+ * spear_latency_table -- copy the library's built-in latency table: for each shape measured on
+ * a B200, the device time per call of its fastest plan in a chained CUDA graph (the dispatcher's
+ * table).  out may be NULL to query *len_out only; otherwise capacity must be >= *len_out.
+ */
+SPEAR_API spear_status spear_latency_table(spear_latency_entry* out, int32_t capacity, int32_t* len_out);
+
+/*
+ * spear_predict_step_us -- predicted latency of one step on M tokens (0 <= M <= 65536).
+ *   linears, n_linears   host array (n_linears >= 1)
+ *   fixed_us             time of the step outside these linears (>= 0), added as is
+ *   lut, lut_len         host latency table, or NULL to use the built-in one
+ * Returns SPEAR_ERR_UNSUPPORTED_SHAPE if a linear with count > 0 has no row of its (N, K,
+ * compensator or not) in the table, SPEAR_ERR_INVALID_ARG for bad arguments or table rows.
+ */
+SPEAR_API spear_status spear_predict_step_us(const spear_linear_desc* linears, int32_t n_linears, int64_t M,
+                                             double fixed_us, const spear_latency_entry* lut, int32_t lut_len,
+                                             double* us_out);
+
+/*
+ * spear_pick_prefill_chunk -- the largest chunk = c * granule (c >= 0, chunk <= max_chunk and
+ * decode_tokens + chunk <= 65536) whose predicted step latency on decode_tokens + chunk tokens
+ * is <= slo_us; *predicted_us_out is that step's predicted latency.  If the decode tokens alone
+ * already miss the target, *chunk_out = 0 and *predicted_us_out > slo_us.  Other arguments and
+ * errors as for spear_predict_step_us; slo_us > 0, granule >= 1.
+ */
+SPEAR_API spear_status spear_pick_prefill_chunk(const spear_linear_desc* linears, int32_t n_linears,
+                                                int64_t decode_tokens, int64_t max_chunk, int64_t granule,
+                                                double slo_us, double fixed_us, const spear_latency_entry* lut,
+                                                int32_t lut_len, int64_t* chunk_out, double* predicted_us_out);
+
 /* Static string for a status code (never NULL). */
 SPEAR_API const char* spear_status_string(spear_status status);
 

@@ -27,7 +27,8 @@ STATUS_NAMES = {0: "SPEAR_OK", 1: "SPEAR_ERR_INVALID_ARG", 2: "SPEAR_ERR_UNSUPPO
                 3: "SPEAR_ERR_MISALIGNED", 4: "SPEAR_ERR_WORKSPACE_TOO_SMALL", 5: "SPEAR_ERR_CUDA",
                 6: "SPEAR_ERR_TIMEOUT"}
 EXPORTED = ["spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_plan_update", "spear_w4ec_gemm",
-            "spear_w4ec_gemm_noalloc", "spear_get_device_status", "spear_status_string", "spear_version"]
+            "spear_w4ec_gemm_noalloc", "spear_get_device_status", "spear_status_string", "spear_version",
+            "spear_latency_table", "spear_predict_step_us", "spear_pick_prefill_chunk"]
 
 
 class SpearError(RuntimeError):
@@ -44,6 +45,15 @@ class spear_plan(ctypes.Structure):
     def __repr__(self):
         return (f"spear_plan(kernel_id={self.kernel_id}, tile_n={self.tile_n}, split_k={self.split_k}, "
                 f"tile_m={self.tile_m}, flags={self.flags}, workspace_bytes={self.workspace_bytes})")
+
+
+class spear_linear_desc(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("K", ctypes.c_int64), ("rank", ctypes.c_int32), ("count", ctypes.c_int32)]
+
+
+class spear_latency_entry(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("has_ec", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("us", ctypes.c_double)]
 
 
 class spear_ec(ctypes.Structure):
@@ -68,11 +78,19 @@ def _load():
     lib.spear_w4ec_gemm_noalloc.argtypes = [ctypes.POINTER(spear_plan), P, I64, I64, I64, P, P, P,
                                             ctypes.POINTER(spear_ec), P, ctypes.c_int, P]
     lib.spear_get_device_status.argtypes = [P, ctypes.c_int, P]
+    LD, LE = ctypes.POINTER(spear_linear_desc), ctypes.POINTER(spear_latency_entry)
+    lib.spear_latency_table.argtypes = [LE, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
+    lib.spear_predict_step_us.argtypes = [LD, ctypes.c_int32, I64, ctypes.c_double, LE, ctypes.c_int32,
+                                          ctypes.POINTER(ctypes.c_double)]
+    lib.spear_pick_prefill_chunk.argtypes = [LD, ctypes.c_int32, I64, I64, I64, ctypes.c_double, ctypes.c_double,
+                                             LE, ctypes.c_int32, ctypes.POINTER(ctypes.c_int64),
+                                             ctypes.POINTER(ctypes.c_double)]
     lib.spear_status_string.argtypes = [ctypes.c_int]
     lib.spear_status_string.restype = ctypes.c_char_p
     lib.spear_version.restype = ctypes.c_int
     for fn in ("spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_plan_update", "spear_w4ec_gemm",
-               "spear_w4ec_gemm_noalloc", "spear_get_device_status"):
+               "spear_w4ec_gemm_noalloc", "spear_get_device_status", "spear_latency_table",
+               "spear_predict_step_us", "spear_pick_prefill_chunk"):
         getattr(lib, fn).restype = ctypes.c_int
     return lib
 
@@ -192,6 +210,54 @@ def spear_plan_update(plan: spear_plan, M: int, N: int, K: int, rank: int = 0) -
     """Checks a plan whose fields were changed and recomputes its workspace_bytes (in place)."""
     _check("spear_plan_update", _lib.spear_plan_update(ctypes.byref(plan), M, N, K, rank))
     return plan
+
+
+def _linears(linears):
+    """(N, K, rank, count) tuples -> a ctypes array of spear_linear_desc."""
+    arr = (spear_linear_desc * len(linears))()
+    for i, (N, K, rank, count) in enumerate(linears):
+        arr[i].N, arr[i].K, arr[i].rank, arr[i].count = N, K, rank, count
+    return arr
+
+
+def _lut(lut):
+    """None (the built-in table) or (M, N, K, has_ec, us) tuples -> (pointer, length)."""
+    if lut is None:
+        return None, 0
+    arr = (spear_latency_entry * len(lut))()
+    for i, (M, N, K, has_ec, us) in enumerate(lut):
+        arr[i].M, arr[i].N, arr[i].K, arr[i].has_ec, arr[i].us = M, N, K, int(bool(has_ec)), us
+    return arr, len(lut)
+
+
+def spear_latency_table():
+    """The built-in kernel-latency table as (M, N, K, has_ec, us) tuples."""
+    n = ctypes.c_int32()
+    _check("spear_latency_table", _lib.spear_latency_table(None, 0, ctypes.byref(n)))
+    arr = (spear_latency_entry * n.value)()
+    _check("spear_latency_table", _lib.spear_latency_table(arr, n.value, ctypes.byref(n)))
+    return [(e.M, e.N, e.K, e.has_ec, e.us) for e in arr]
+
+
+def spear_predict_step_us(linears, M: int, fixed_us: float = 0.0, lut=None) -> float:
+    """Predicted latency (us) of one step that runs every (N, K, rank, count) linear on M tokens."""
+    la, (lp, ln) = _linears(linears), _lut(lut)
+    out = ctypes.c_double()
+    _check("spear_predict_step_us",
+           _lib.spear_predict_step_us(la, len(linears), M, fixed_us, lp, ln, ctypes.byref(out)))
+    return out.value
+
+
+def spear_pick_prefill_chunk(linears, decode_tokens: int, max_chunk: int, slo_us: float, granule: int = 128,
+                             fixed_us: float = 0.0, lut=None):
+    """(chunk, predicted_us): the largest prefill chunk (a multiple of granule) whose step with
+    decode_tokens + chunk tokens is predicted to meet slo_us."""
+    la, (lp, ln) = _linears(linears), _lut(lut)
+    chunk, pred = ctypes.c_int64(), ctypes.c_double()
+    _check("spear_pick_prefill_chunk",
+           _lib.spear_pick_prefill_chunk(la, len(linears), decode_tokens, max_chunk, granule, slo_us, fixed_us,
+                                         lp, ln, ctypes.byref(chunk), ctypes.byref(pred)))
+    return chunk.value, pred.value
 
 
 def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
