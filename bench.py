@@ -298,8 +298,9 @@ def run_ours(args, rank, world, torch, dist):
             step_calls(i)
     stream.synchronize()
     g_main = graph_of(args.steps)
-    g_main.replay()
-    stream.synchronize()
+    with torch.cuda.stream(stream):
+        g_main.replay()
+    torch.cuda.synchronize()
 
     # Timed region: barrier + sync on both sides, K steps, max over ranks.
     clk = ClockSampler(torch.cuda.current_device()).start()
@@ -692,9 +693,9 @@ def _time_calls(torch, stream, calls, reps):
     with torch.cuda.stream(stream):
         with torch.cuda.graph(g, stream=stream):
             run()
-    for _ in range(2):
-        g.replay()
-    stream.synchronize()
+        for _ in range(2):                   # warm replays on the timed stream, finished before timing
+            g.replay()
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
@@ -781,9 +782,9 @@ def model_sweep(args):
         with torch.cuda.stream(stream):
             with torch.cuda.graph(g, stream=stream):
                 one_pass()
-        for _ in range(2):
-            g.replay()
-        stream.synchronize()
+            for _ in range(2):               # warm replays on the timed stream, finished before timing
+                g.replay()
+        torch.cuda.synchronize()
         n = 10 if M <= 256 else 3
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
