@@ -69,6 +69,8 @@ class Oracle:
                                          ctypes.c_int32, P]
         lib.oracle_w4ec_gemm_sampled.argtypes = [P, I64, I64, I64, P, P, P, P, P, P, ctypes.c_float,
                                                  ctypes.c_int32, P, P, I64, P]
+        lib.oracle_w4ec_gemm_grouped.argtypes = [P, I64, I64, I64, I64, P, P, P, P, P, P, ctypes.c_float,
+                                                 ctypes.c_int32, P]
         lib.oracle_w4ec_gemm_mlp.argtypes = [P, I64, I64, I64, P, P, P, P, P, ctypes.c_int32, P, P, P, P,
                                              ctypes.c_int32, ctypes.c_float, P]
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -153,6 +155,28 @@ class Oracle:
                                    _ptr(_c(z_bits, np.uint16)), _ptr(_c(A_bits, np.uint16)),
                                    _ptr(_c(B_bits, np.uint16)), _ptr(_c(wg_bits, np.uint16)),
                                    ctypes.c_float(b_g), r, _ptr(y))
+        return y
+
+    def pack_w4_grouped(self, W: np.ndarray, G: int):
+        """Group-wise RTN: the per-channel format of W viewed as [N * K/G, G].
+        Returns packed [N, K/2], s and z binary16 bits [N, K/G]."""
+        N, K = W.shape
+        packed, s, z = self.pack_w4(np.ascontiguousarray(W, dtype=np.float32).reshape(N * (K // G), G))
+        return packed.reshape(N, K // 2), s.reshape(N, K // G), z.reshape(N, K // G)
+
+    def w4ec_gemm_grouped(self, x_bits, packed, s_bits, z_bits, G: int, A_bits=None, B_bits=None, wg_bits=None,
+                          b_g: float = 0.0):
+        """y fp64 [M, N] of the layer with group-wise scales (s, z [N, K/G]); no EC if A_bits is None."""
+        x = _c(x_bits, np.uint16)
+        M, K = x.shape
+        N = packed.shape[0]
+        r = 0 if A_bits is None else A_bits.shape[1]
+        y = np.empty((M, N), dtype=np.float64)
+        self._lib.oracle_w4ec_gemm_grouped(
+            _ptr(x), M, N, K, G, _ptr(_c(packed, np.uint8)), _ptr(_c(s_bits, np.uint16)), _ptr(_c(z_bits, np.uint16)),
+            None if A_bits is None else _ptr(_c(A_bits, np.uint16)),
+            None if B_bits is None else _ptr(_c(B_bits, np.uint16)),
+            None if wg_bits is None else _ptr(_c(wg_bits, np.uint16)), b_g, r, _ptr(y))
         return y
 
     def w4ec_gemm_mlp(self, x_bits, packed, s_bits, z_bits, A_bits, B_bits, W1, b1, W2, b2, alpha: float = 1.0):

@@ -285,6 +285,55 @@ void oracle_w4ec_gemm(const uint16_t* x, int64_t M, int64_t N, int64_t K,
     free(t); free(p); free(g);
 }
 
+/* Group-wise scales (the GPTQ/AWQ-style backends the technical summary's section 3.1 lists as
+ * compatible): every G consecutive k of a row have their own scale and zero-point, found by the
+ * same RTN steps as above applied to that group alone, so the grouped format of W [N, K] is the
+ * per-channel format of W viewed as [N * K/G, G]: packed [N, K/2] unchanged, s and z [N, K/G].
+ *   What[n,k] = (q[n,k] - z[n, k/G]) * s[n, k/G]
+ *   y[m,n]    = sum_k x[m,k] What[n,k] + g[m] sum_j t[m,j] B[j,n]
+ * A == NULL or r == 0 -> no compensator.  y is fp64 [M,N]. */
+void oracle_w4ec_gemm_grouped(const uint16_t* x, int64_t M, int64_t N, int64_t K, int64_t G,
+                              const uint8_t* packed, const uint16_t* s_bits, const uint16_t* z_bits,
+                              const uint16_t* A, const uint16_t* B, const uint16_t* wg, float b_g, int32_t r,
+                              double* y)
+{
+    int has_ec = (A != NULL && B != NULL && wg != NULL && r > 0);
+    int64_t ng = K / G;
+    double *t = NULL, *p = NULL, *g = NULL;
+    if (has_ec) {
+        t = (double*)malloc(sizeof(double) * (size_t)(M * r));
+        p = (double*)malloc(sizeof(double) * (size_t)M);
+        g = (double*)malloc(sizeof(double) * (size_t)M);
+        oracle_ec_gate(x, M, K, A, r, wg, b_g, t, p, g);
+    }
+    #pragma omp parallel
+    {
+        double* what = (double*)malloc(sizeof(double) * (size_t)K);
+        #pragma omp for schedule(static)
+        for (int64_t n = 0; n < N; ++n) {
+            for (int64_t k = 0; k < K; ++k) {
+                uint8_t v = packed[n * (K / 2) + k / 2];
+                double q = (double)((k & 1) ? (v >> 4) : (v & 0xF));
+                int64_t grp = k / G;
+                what[k] = (q - oracle_f16_to_f64(z_bits[n * ng + grp])) * oracle_f16_to_f64(s_bits[n * ng + grp]);
+            }
+            for (int64_t m = 0; m < M; ++m) {
+                double sum = 0.0;
+                for (int64_t k = 0; k < K; ++k) sum += oracle_bf16_to_f64(x[m * K + k]) * what[k];
+                if (has_ec) {
+                    double ec = 0.0;
+                    for (int32_t j = 0; j < r; ++j)
+                        ec += t[m * r + j] * oracle_bf16_to_f64(B[(int64_t)j * N + n]);
+                    sum += g[m] * ec;
+                }
+                y[m * N + n] = sum;
+            }
+        }
+        free(what);
+    }
+    free(t); free(p); free(g);
+}
+
 /* The pages' gate form (technical summary section 2.1A): effective weight
  * W + alpha * B diag(gamma(Ax)) A, gamma a bottleneck MLP.  The pages do not
  * spell the MLP out; this follows the plainest reading of "bottleneck MLP" over

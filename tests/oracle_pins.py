@@ -325,6 +325,49 @@ def pin_mlp_gate(o):
     assert np.allclose(yu, ya, rtol=0, atol=scale)
 
 
+def pin_grouped(o):
+    """Group-wise scales (G consecutive k per scale and zero-point): G = K is the per-channel
+    layer; for G < K the layer equals numpy's matmul with weights dequantised group by group
+    (scales broadcast with np.repeat), plus the EC term; each group's RTN error stays within
+    half its step, and no group's step exceeds its row's per-channel step."""
+    x, W, A, B, wg, b_g = small_layer(41, M=5, N=24, K=256, r=8)
+    K, N = 256, 24
+    packed, s, z = o.pack_w4(W)
+    pg, sg, zg = o.pack_w4_grouped(W, K)
+    assert np.array_equal(pg, packed) and np.array_equal(sg[:, 0], s) and np.array_equal(zg[:, 0], z)
+    y_pc = o.w4ec_gemm(x, packed, s, z, A, B, wg, b_g)
+    y_g = o.w4ec_gemm_grouped(x, pg, sg, zg, K, A, B, wg, b_g)
+    assert np.allclose(y_g, y_pc, rtol=0, atol=1e-12 * np.abs(y_pc).max())
+    xf = f32_from_bf16_bits(x).astype(np.float64)
+    t, _, g = o.ec_gate(x, A, wg, b_g)
+    ec = g[:, None] * (t @ f32_from_bf16_bits(B).astype(np.float64))
+    for G in (32, 64, 128):
+        pg, sg, zg = o.pack_w4_grouped(W, G)
+        assert pg.shape == (N, K // 2) and sg.shape == (N, K // G)
+        q = numpy_unpack(pg, K).astype(np.float64)
+        sf = np.repeat(f16_bits_to_f64(sg), G, axis=1)
+        zf = np.repeat(f16_bits_to_f64(zg), G, axis=1)
+        What = (q - zf) * sf
+        assert np.all(np.abs(W.astype(np.float64) - What) <= 0.5 * sf * (1 + 1e-6) + 1e-12)
+        assert np.all(f16_bits_to_f64(sg) <= f16_bits_to_f64(s)[:, None])
+        want = xf @ What.T
+        y = o.w4ec_gemm_grouped(x, pg, sg, zg, G)
+        assert np.allclose(y, want, rtol=0, atol=1e-12 * np.abs(want).max())
+        y = o.w4ec_gemm_grouped(x, pg, sg, zg, G, A, B, wg, b_g)
+        assert np.allclose(y, want + ec, rtol=0, atol=1e-12 * np.abs(want + ec).max())
+    # A change inside one group moves only that group's codes, scale and zero-point.
+    G = 64
+    W2 = W.copy()
+    W2[3, 70] = 0.5
+    pa, sa, za = o.pack_w4_grouped(W, G)
+    pb, sb, zb = o.pack_w4_grouped(W2, G)
+    diff_s = np.argwhere(sa != sb)
+    assert diff_s.tolist() == [[3, 1]] and (za != zb).sum() <= 1
+    qa, qb = numpy_unpack(pa, K), numpy_unpack(pb, K)
+    rows, cols = np.nonzero(qa != qb)
+    assert set(rows.tolist()) == {3} and cols.min() >= 64 and cols.max() < 128
+
+
 ALL_PINS = [pin_f16_encoder, pin_golden_rows, pin_grid_round_trip, pin_rtn_bruteforce, pin_scale_pow2,
             pin_main_term_vs_numpy, pin_ec_vs_numpy, pin_gate_limits, pin_bruteforce_rational,
-            pin_sampled_and_prefix, pin_mlp_gate]
+            pin_sampled_and_prefix, pin_mlp_gate, pin_grouped]

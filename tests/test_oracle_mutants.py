@@ -35,6 +35,9 @@ MUTATIONS = {
                                  "u[m * r + j] = (1.0 / (1.0 + exp(-(double)alpha * pre))) * tm[j];"),
     "mlp_W1_transposed": ("(double)W1[(int64_t)i * r + j] * tm[j]", "(double)W1[(int64_t)j * H + i] * tm[j]"),
     "mlp_W2_transposed": ("(double)W2[(int64_t)j * H + i] * h[i]", "(double)W2[(int64_t)i * r + j] * h[i]"),
+    "grouped_index_modulo": ("int64_t grp = k / G;", "int64_t grp = k % ng;"),
+    "grouped_zero_of_first_group": ("(q - oracle_f16_to_f64(z_bits[n * ng + grp]))", "(q - oracle_f16_to_f64(z_bits[n * ng]))"),
+    "grouped_scale_of_next_row": ("* oracle_f16_to_f64(s_bits[n * ng + grp]);", "* oracle_f16_to_f64(s_bits[((n + 1) % N) * ng + grp]);"),
     "main_term_dropped_last_k": ("for (int64_t k = 0; k < K; ++k) acc += xr[k] * wrow[k];",
                                  "for (int64_t k = 0; k < K - 1; ++k) acc += xr[k] * wrow[k];"),
 }
