@@ -68,6 +68,8 @@ def parse():
     ap.add_argument("--slo-check", action="store_true",
                     help="SLO-constrained prefill chunk picker on the 16-layer model: picked chunk, predicted "
                          "and measured step time per ITL target")
+    ap.add_argument("--grouped-compare", action="store_true",
+                    help="per-channel vs group-wise (128) scales on the decode-qo layer, EC on and off")
     ap.add_argument("--gate-compare", action="store_true",
                     help="time the layer with the scalar gate and with the bottleneck-MLP gate (H=16) on "
                          "decode-qo M=16 and the prefill layer")
@@ -808,6 +810,70 @@ def model_sweep(args):
                                       "passes": rows}}))
 
 
+def grouped_compare(args):
+    """Device time per call of the decode-qo layer (4096 x 4096, EC r = 64) with per-channel scales
+    (the dispatcher's plan) and with group-wise scales (groups of 128), EC on and off, M in
+    {1, 16, 256}: a chained CUDA graph of 32 calls over rotating weight copies, best of 5."""
+    import torch
+    import w4_gemm_error_channel_b200 as spear
+    from synthetic import config_layers
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda")
+    G = 128
+    L = config_layers(1, M=256)[0]
+    N, K, r = L.N, L.K, L.rank
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+    W = torch.from_numpy(L.W).to(dev)
+    copies = max(2, int(np.ceil(2 * L2_BYTES / layer_bytes(256, N, K, r))) + 1)
+    pc = [spear.spear_pack_w4(W) for _ in range(copies)]
+    gp = [spear.spear_pack_w4_grouped(W, G) for _ in range(copies)]
+    del W
+    A, B, wg = bf(L.A_bits), bf(L.B_bits), bf(L.wg_bits)
+    stream = torch.cuda.Stream()
+    rows = []
+    for M in (1, 16, 256):
+        x = bf(L.x(M))
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for grouped in (False, True):
+            for use_ec in (True, False):
+                ec = spear.EC(A, B, wg, L.b_g) if use_ec else None
+                rk = r if use_ec else 0
+                if grouped:
+                    ws = spear.alloc_workspace(spear.spear_grouped_workspace_bytes(M, N, K, G, rk))
+                    call = lambda i: spear.spear_w4ec_gemm_grouped(x, *gp[i % copies], G, ec, y=y, workspace=ws,
+                                                                   stream=stream)
+                else:
+                    plan = spear.spear_gemm_plan(M, N, K, rk)
+                    ws = spear.alloc_workspace(plan.workspace_bytes)
+                    call = lambda i: spear.spear_w4ec_gemm(x, *pc[i % copies], ec, y=y, workspace=ws, plan=plan,
+                                                           stream=stream)
+                n = 32
+                with torch.cuda.stream(stream):
+                    call(0)
+                stream.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(stream):
+                    with torch.cuda.graph(g, stream=stream):
+                        for i in range(n):
+                            call(i)
+                best = 1e9
+                for _ in range(5):
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    with torch.cuda.stream(stream):
+                        e0.record(stream)
+                        g.replay()
+                        e1.record(stream)
+                    e1.synchronize()
+                    best = min(best, e0.elapsed_time(e1) * 1e3 / n)
+                del g
+                extra = (N * (K // G) * 4 - 4 * N) if grouped else 0          # group scales and zeros
+                byts = layer_bytes(M, N, K, rk) + extra
+                rows.append({"M": M, "scales": f"group {G}" if grouped else "per channel", "ec": use_ec,
+                             "us": best, "GBps": byts / best / 1e3,
+                             "device_status": spear.spear_get_device_status(ws)})
+    print(json.dumps({"grouped_compare": {"workload": f"decode-qo layer {N}x{K}, EC r={r}, synthetic", "rows": rows}}))
+
+
 def gate_compare(args):
     """Device time per call of the same layer with the scalar gate and with the bottleneck-MLP gate
     (H = 16, random fp32 gate weights), in a chained CUDA graph of calls over rotating weight copies."""
@@ -870,6 +936,9 @@ def main():
     args = parse()
     if args.gate_compare:
         gate_compare(args)
+        return
+    if args.grouped_compare:
+        grouped_compare(args)
         return
     if args.model_sweep:
         model_sweep(args)

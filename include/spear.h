@@ -225,6 +225,44 @@ SPEAR_API spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const voi
                                                const spear_ec* ec, void* y, spear_dtype y_dtype, void* stream);
 
 /*
+ * Group-wise scales (section 3.1: the method sits on GPTQ, AWQ and OmniQuant backends as well as
+ * on RTN).  Every `group` consecutive k of a row have their own binary16 scale and zero-point,
+ * found by the same RTN steps as spear_pack_w4 applied to that group alone:
+ *   What[n,k] = (q[n,k] - z[n, k/group]) * s[n, k/group]
+ *
+ * spear_pack_w4_grouped -- as spear_pack_w4, with scale and zero [N, K/group] (row-major).
+ *   group      even and dividing K; spear_w4ec_gemm_grouped needs a multiple of 128
+ *   packed     [N, K/2], the same layout as spear_pack_w4's
+ * Returns SPEAR_ERR_UNSUPPORTED_SHAPE for a group that is odd or does not divide K.
+ */
+SPEAR_API spear_status spear_pack_w4_grouped(const void* W, spear_dtype w_dtype, int64_t N, int64_t K,
+                                             int64_t group, void* packed, void* scale, void* zero, void* stream);
+
+/*
+ * spear_grouped_workspace_bytes -- workspace of spear_w4ec_gemm_grouped for this shape: the
+ * zeroed control block, plus, with a compensator, u (bf16 [M, rank]) and the fp32 main term
+ * [M, N].  Host only.
+ */
+SPEAR_API spear_status spear_grouped_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group,
+                                                     int32_t rank, size_t* out);
+
+/*
+ * spear_w4ec_gemm_grouped -- y = x What^T + g(x) * ((x A) B) with group-wise scales.
+ *
+ * Arguments as for spear_w4ec_gemm, without a plan, with `group` and the [N, K/group] scale and
+ * zero from spear_pack_w4_grouped.  Requires N % 128 == 0, group a multiple of 128 dividing K, and a
+ * compensator rank of at most 128 (16..128, step 16); the scalar and the MLP gate are both taken.
+ * A weight-streaming tensor-core kernel computes the main term, applying each group's scale to its
+ * 128-code windows.  With a compensator the main term goes to the workspace (fp32) and the
+ * compensator runs beside it on the library's side stream (as SPEAR_PLAN_SEPARATE_EC does for the
+ * prefill kernel), joined by a kernel that adds u B and rounds y once.  Deterministic.
+ */
+SPEAR_API spear_status spear_w4ec_gemm_grouped(const void* x, int64_t M, int64_t N, int64_t K, int64_t group,
+                                               const void* packed, const void* scale, const void* zero,
+                                               const spear_ec* ec, void* y, spear_dtype y_dtype, void* workspace,
+                                               size_t workspace_bytes, void* stream);
+
+/*
  * spear_get_device_status -- read (and optionally clear) the error word that
  * bounded in-kernel waits set when they give up.  Synchronises `stream`.
  * Returns SPEAR_OK, SPEAR_ERR_TIMEOUT, or SPEAR_ERR_CUDA.

@@ -199,3 +199,38 @@ def test_plan_update_and_semifused_workspace():
     assert bytes(q) == before
     with pytest.raises(spear.SpearError):
         spear.spear_plan_update(q2, M, N, K, r)
+
+
+def test_grouped_host_checks():
+    # Group-wise scales: groups of a multiple of 128 dividing K for the layer (any even divisor for
+    # the packer), compensator rank <= 128.  Fake, never-dereferenced addresses throughout.
+    P, lib = ctypes.c_void_p, spear._lib
+    pack = lambda W=0x1000, N=256, K=512, G=128, packed=0x2000, dt=1: lib.spear_pack_w4_grouped(
+        P(W), dt, N, K, G, P(packed), P(0x3000), P(0x4000), None)
+    assert pack(W=0) == INVALID
+    assert pack(G=0) == INVALID
+    assert pack(G=7) == SHAPE
+    assert pack(G=96) == SHAPE            # does not divide 512
+    assert pack(packed=0x2008) == MISALIGNED
+    out = ctypes.c_size_t()
+    ws = lambda M=300, N=512, K=512, G=128, r=0: lib.spear_grouped_workspace_bytes(M, N, K, G, r, ctypes.byref(out))
+    assert ws() == OK and out.value == (128 + 1024) * 1024
+    assert ws(r=16) == OK and out.value == (128 + 1024) * 1024 + (300 * 16 * 2 + 255) // 256 * 256 + 300 * 512 * 4
+    for kw, want in (({"G": 64}, SHAPE), ({"G": 384}, SHAPE), ({"r": 144}, SHAPE), ({"r": 8}, SHAPE),
+                     ({"N": 500}, SHAPE), ({"M": -1}, INVALID)):
+        assert ws(**kw) == want, kw
+    assert lib.spear_grouped_workspace_bytes(1, 512, 512, 128, 0, None) == INVALID
+
+    def gemm(M=4, N=512, K=512, G=128, x=0x1000, y=0x5000, wsp=0x6000, ws_bytes=1 << 30, ec=None):
+        return lib.spear_w4ec_gemm_grouped(P(x), M, N, K, G, P(0x2000), P(0x3000), P(0x4000), ec, P(y), 0, P(wsp),
+                                           ws_bytes, None)
+    assert gemm(x=0) == INVALID
+    assert gemm(wsp=0) == INVALID
+    assert gemm(G=64) == SHAPE
+    assert gemm(x=0x1008) == MISALIGNED
+    assert gemm(ws_bytes=1024) == WS_SMALL
+    assert gemm(M=0) == OK
+    big = spear.spear_ec(0x7000, 0x8000, 0x9000, 0.0, 144)
+    assert gemm(ec=ctypes.byref(big)) == SHAPE
+    e16 = spear.spear_ec(0x7000, 0x8000, 0x9000, 0.0, 16)
+    assert gemm(ec=ctypes.byref(e16), ws_bytes=(128 + 1024) * 1024) == WS_SMALL

@@ -28,7 +28,8 @@ STATUS_NAMES = {0: "SPEAR_OK", 1: "SPEAR_ERR_INVALID_ARG", 2: "SPEAR_ERR_UNSUPPO
                 6: "SPEAR_ERR_TIMEOUT"}
 EXPORTED = ["spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_plan_update", "spear_w4ec_gemm",
             "spear_w4ec_gemm_noalloc", "spear_get_device_status", "spear_status_string", "spear_version",
-            "spear_latency_table", "spear_predict_step_us", "spear_pick_prefill_chunk"]
+            "spear_latency_table", "spear_predict_step_us", "spear_pick_prefill_chunk",
+            "spear_pack_w4_grouped", "spear_grouped_workspace_bytes", "spear_w4ec_gemm_grouped"]
 
 
 class SpearError(RuntimeError):
@@ -78,6 +79,11 @@ def _load():
     lib.spear_w4ec_gemm_noalloc.argtypes = [ctypes.POINTER(spear_plan), P, I64, I64, I64, P, P, P,
                                             ctypes.POINTER(spear_ec), P, ctypes.c_int, P]
     lib.spear_get_device_status.argtypes = [P, ctypes.c_int, P]
+    lib.spear_pack_w4_grouped.argtypes = [P, ctypes.c_int, I64, I64, I64, P, P, P, P]
+    lib.spear_grouped_workspace_bytes.argtypes = [I64, I64, I64, I64, ctypes.c_int32,
+                                                  ctypes.POINTER(ctypes.c_size_t)]
+    lib.spear_w4ec_gemm_grouped.argtypes = [P, I64, I64, I64, I64, P, P, P, ctypes.POINTER(spear_ec), P,
+                                            ctypes.c_int, P, ctypes.c_size_t, P]
     LD, LE = ctypes.POINTER(spear_linear_desc), ctypes.POINTER(spear_latency_entry)
     lib.spear_latency_table.argtypes = [LE, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
     lib.spear_predict_step_us.argtypes = [LD, ctypes.c_int32, I64, ctypes.c_double, LE, ctypes.c_int32,
@@ -90,7 +96,8 @@ def _load():
     lib.spear_version.restype = ctypes.c_int
     for fn in ("spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_plan_update", "spear_w4ec_gemm",
                "spear_w4ec_gemm_noalloc", "spear_get_device_status", "spear_latency_table",
-               "spear_predict_step_us", "spear_pick_prefill_chunk"):
+               "spear_predict_step_us", "spear_pick_prefill_chunk", "spear_pack_w4_grouped",
+               "spear_grouped_workspace_bytes", "spear_w4ec_gemm_grouped"):
         getattr(lib, fn).restype = ctypes.c_int
     return lib
 
@@ -210,6 +217,51 @@ def spear_plan_update(plan: spear_plan, M: int, N: int, K: int, rank: int = 0) -
     """Checks a plan whose fields were changed and recomputes its workspace_bytes (in place)."""
     _check("spear_plan_update", _lib.spear_plan_update(ctypes.byref(plan), M, N, K, rank))
     return plan
+
+
+def spear_pack_w4_grouped(W: torch.Tensor, group: int, stream=None):
+    """Group-wise RTN W4 packing of W [N, K] (fp32 or bf16, on the GPU): packed [N, K/2] uint8,
+    scale and zero [N, K/group] fp16."""
+    _dev(W, "W")
+    if W.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("W must be fp32 or bf16")
+    W = W.contiguous()
+    N, K = W.shape
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    scale = torch.empty((N, max(K // max(group, 1), 1)), dtype=torch.float16, device=W.device)
+    zero = torch.empty_like(scale)
+    dt = SPEAR_BF16 if W.dtype == torch.bfloat16 else SPEAR_FP32
+    _check("spear_pack_w4_grouped", _lib.spear_pack_w4_grouped(_p(W), dt, N, K, group, _p(packed), _p(scale),
+                                                              _p(zero), _stream(stream)))
+    return packed, scale, zero
+
+
+def spear_grouped_workspace_bytes(M: int, N: int, K: int, group: int, rank: int = 0) -> int:
+    out = ctypes.c_size_t()
+    _check("spear_grouped_workspace_bytes", _lib.spear_grouped_workspace_bytes(M, N, K, group, rank, ctypes.byref(out)))
+    return out.value
+
+
+def spear_w4ec_gemm_grouped(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
+                            group: int, ec: Optional[EC] = None, y: Optional[torch.Tensor] = None,
+                            y_dtype=torch.bfloat16, workspace: Optional[torch.Tensor] = None, stream=None):
+    """y = x What^T + g(x) (x A) B with group-wise scales (scale, zero [N, K/group])."""
+    _dev(x, "x")
+    if x.dtype != torch.bfloat16:
+        raise ValueError("x must be bf16")
+    M, K = x.shape
+    N = packed.shape[0]
+    rank = ec.rank if ec is not None else 0
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=x.device)
+    yd = SPEAR_FP32 if y.dtype == torch.float32 else SPEAR_BF16
+    if workspace is None:
+        workspace = alloc_workspace(spear_grouped_workspace_bytes(M, N, K, group, rank), x.device)
+    ec_c = ctypes.byref(ec.as_c()) if ec is not None else None
+    _check("spear_w4ec_gemm_grouped",
+           _lib.spear_w4ec_gemm_grouped(_p(x), M, N, K, group, _p(packed), _p(scale), _p(zero), ec_c, _p(y), yd,
+                                        _p(workspace), workspace.numel(), _stream(stream)))
+    return y
 
 
 def _linears(linears):

@@ -186,11 +186,23 @@ spear_status plan_tc05(int64_t M, int64_t N, int sms, spear_plan* p) {
     return SPEAR_OK;
 }
 
+// Group-wise layer: groups of a multiple of 128 codes dividing K; with a compensator, its EC
+// tiles run on the tcgen05 kernel (rank <= TC05_MAX_RANK).
+spear_status check_grouped_shape(int64_t M, int64_t N, int64_t K, int64_t group, int32_t rank);
+
 // Token count from which the tensor-core kernel replaces the weight-streaming kernel, and the
 // largest compensator rank it takes (one 128-row EC tile per token block).
 constexpr int64_t TC05_MIN_M = 128;
 constexpr int32_t TC05_MAX_RANK = 128;
 bool use_tc05(int64_t M, int32_t rank) { return M >= TC05_MIN_M && rank <= TC05_MAX_RANK; }
+
+spear_status check_grouped_shape(int64_t M, int64_t N, int64_t K, int64_t group, int32_t rank) {
+    spear_status st = check_shape(M, N, K, rank);
+    if (st != SPEAR_OK) return st;
+    if (group <= 0 || group % 128 != 0 || K % group != 0) return SPEAR_ERR_UNSUPPORTED_SHAPE;
+    if (rank > TC05_MAX_RANK) return SPEAR_ERR_UNSUPPORTED_SHAPE;
+    return SPEAR_OK;
+}
 
 spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K, int32_t rank) {
     (void)M;
@@ -395,6 +407,99 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         if (separate && launch_apply(a, s) != cudaSuccess) return SPEAR_ERR_CUDA;
     }
     return SPEAR_OK;
+}
+
+spear_status spear_pack_w4_grouped(const void* W, spear_dtype w_dtype, int64_t N, int64_t K, int64_t group,
+                                   void* packed, void* scale, void* zero, void* stream) {
+    if (!W || !packed || !scale || !zero) return SPEAR_ERR_INVALID_ARG;
+    if (w_dtype != SPEAR_BF16 && w_dtype != SPEAR_FP32) return SPEAR_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0 || group <= 0) return SPEAR_ERR_INVALID_ARG;
+    if (group % 2 != 0 || K % group != 0) return SPEAR_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(W) || !aligned16(packed) || !aligned16(scale) || !aligned16(zero)) return SPEAR_ERR_MISALIGNED;
+    // Each group is quantised as a row of its own: the per-channel packer over W viewed as
+    // [N * K / group, group], whose outputs are laid out as [N, K/2] and [N, K/group].
+    cudaError_t e = launch_pack_w4(W, w_dtype == SPEAR_BF16, N * (K / group), group, packed, scale, zero,
+                                   (cudaStream_t)stream);
+    return e == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
+}
+
+spear_status spear_grouped_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group, int32_t rank,
+                                           size_t* out) {
+    if (!out) return SPEAR_ERR_INVALID_ARG;
+    spear_status st = check_grouped_shape(M, N, K, group, rank);
+    if (st != SPEAR_OK) return st;
+    size_t b = ZEROED_BYTES;
+    if (rank > 0) b += tc05_u_bytes(M, rank) + (size_t)M * N * 4;     // u, then the fp32 main term
+    *out = b;
+    return SPEAR_OK;
+}
+
+spear_status spear_w4ec_gemm_grouped(const void* x, int64_t M, int64_t N, int64_t K, int64_t group,
+                                     const void* packed, const void* scale, const void* zero, const spear_ec* ec,
+                                     void* y, spear_dtype y_dtype, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+    if (!packed || !scale || !zero || !workspace) return SPEAR_ERR_INVALID_ARG;
+    if (M != 0 && (!x || !y)) return SPEAR_ERR_INVALID_ARG;
+    if (y_dtype != SPEAR_BF16 && y_dtype != SPEAR_FP32) return SPEAR_ERR_INVALID_ARG;
+    const int32_t rank = ec ? ec->rank : 0;
+    if (ec && (!ec->A || !ec->B || !ec->w_g)) return SPEAR_ERR_INVALID_ARG;
+    if (ec && isnan(ec->b_g)) return SPEAR_ERR_INVALID_ARG;
+    if (ec && rank == 0) return SPEAR_ERR_UNSUPPORTED_SHAPE;
+    spear_status st = check_grouped_shape(M, N, K, group, rank);
+    if (st != SPEAR_OK) return st;
+    if ((M != 0 && (!aligned16(x) || !aligned16(y))) || !aligned16(packed) || !aligned16(scale) ||
+        !aligned16(zero) || !aligned16(workspace))
+        return SPEAR_ERR_MISALIGNED;
+    if (ec && (!aligned16(ec->A) || !aligned16(ec->B) || !aligned16(ec->w_g))) return SPEAR_ERR_MISALIGNED;
+    st = check_gate_mlp(ec);
+    if (st != SPEAR_OK) return st;
+    size_t need = 0;
+    spear_grouped_workspace_bytes(M, N, K, group, rank, &need);
+    if (workspace_bytes < need) return SPEAR_ERR_WORKSPACE_TOO_SMALL;
+    if (M == 0) return SPEAR_OK;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned char* ws = (unsigned char*)workspace;
+    GroupedArgs ga;
+    ga.x = (const uint16_t*)x;
+    ga.packed = (const uint8_t*)packed;
+    ga.scale = (const __half*)scale;
+    ga.zero = (const __half*)zero;
+    ga.M = M;
+    ga.N = N;
+    ga.K = K;
+    ga.group = group;
+    ga.y = y;
+    ga.y_fp32 = (y_dtype == SPEAR_FP32);
+    ga.ymain = nullptr;
+    if (rank == 0) return launch_w4g_gemm(ga, s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
+
+    // The compensator beside the grouped GEMM, as on the semi-fused prefill path.
+    unsigned* ctrl = (unsigned*)ws;
+    TcArgs t;
+    t.x = (const uint16_t*)x;
+    t.packed = (const uint8_t*)packed;
+    t.scale = (const __half*)scale;
+    t.zero = (const __half*)zero;
+    t.A = (const uint16_t*)ec->A;
+    t.B = (const uint16_t*)ec->B;
+    t.wg = (const uint16_t*)ec->w_g;
+    t.b_g = ec->b_g;
+    t.mlp = gate_mlp_of(ec);
+    t.rank = rank;
+    t.u = (__nv_bfloat16*)(ws + ZEROED_BYTES);
+    t.y = y;
+    t.y_fp32 = (y_dtype == SPEAR_FP32);
+    t.M = M;
+    t.N = N;
+    t.K = K;
+    t.err = ctrl;
+    t.ec_ready = ctrl + TC_FLAGS_WORD;
+    t.ec_consumed = t.ec_ready + TC_BLOCKS_MAX;
+    t.ec_only = 0;
+    ga.ymain = (float*)(ws + ZEROED_BYTES + tc05_u_bytes(M, rank));
+    auto grouped_main = [](const void* ctx, cudaStream_t st) { return launch_w4g_gemm(*(const GroupedArgs*)ctx, st); };
+    return launch_ec_beside(t, grouped_main, &ga, ga.ymain, s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
 }
 
 spear_status spear_get_device_status(void* workspace, int clear, void* stream) {

@@ -105,9 +105,27 @@ struct TcArgs {
 // programmatic dependent of the previous kernel in the stream; priority: 0 or a launch priority.
 cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream, bool pdl = true, int priority = 0);
 
-// Semi-fused prefill: the EC tiles alone on a side stream of the library, beside the main tiles
-// (fp32 main term into ymain [M][N]) on the caller's stream, joined by ec_up_add (y = ymain + u B).
+// The compensator beside a main-term launch: the tcgen05 kernel's EC tiles alone (u = g t) on a
+// side stream of the library, `main` (which writes the fp32 main term to ymain [M][N]) on the
+// caller's stream, joined by ec_up_add (y = ymain + u B).  `ctx` is read during the call only.
+using MainLaunch = cudaError_t (*)(const void* ctx, cudaStream_t stream);
+cudaError_t launch_ec_beside(const TcArgs& a, MainLaunch main, const void* ctx, float* ymain, cudaStream_t stream);
+// Semi-fused prefill: launch_ec_beside with the tcgen05 kernel's main tiles as the main term.
 cudaError_t launch_semifused(const TcArgs& a, int bn, int rows, float* ymain, cudaStream_t stream);
+
+// Group-wise scales: s, z [N, K / group], group a multiple of 128 dividing K.  Writes the main
+// term to ymain (fp32 [M][N]) when it is set, else y.
+struct GroupedArgs {
+    const uint16_t* x;      // bf16 [M, K]
+    const uint8_t* packed;  // [N, K/2]
+    const __half* scale;    // [N, K/group]
+    const __half* zero;     // [N, K/group]
+    int64_t M, N, K, group;
+    float* ymain;
+    void* y;
+    int y_fp32;
+};
+cudaError_t launch_w4g_gemm(const GroupedArgs& a, cudaStream_t stream);
 
 cudaError_t launch_pack_w4(const void* W, bool w_is_bf16, int64_t N, int64_t K, void* packed, void* scale,
                            void* zero, cudaStream_t stream);

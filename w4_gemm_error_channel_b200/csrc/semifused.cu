@@ -164,8 +164,8 @@ static cudaError_t lane_init(SideLane& L) {
     return cudaSuccess;
 }
 
-cudaError_t launch_semifused(const TcArgs& a, int bn, int rows, float* ymain, cudaStream_t stream) {
-    if (a.rank <= 0 || a.u == nullptr || ymain == nullptr) return cudaErrorInvalidValue;
+cudaError_t launch_ec_beside(const TcArgs& a, MainLaunch main, const void* ctx, float* ymain, cudaStream_t stream) {
+    if (a.rank <= 0 || a.u == nullptr || ymain == nullptr || main == nullptr) return cudaErrorInvalidValue;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -178,14 +178,6 @@ cudaError_t launch_semifused(const TcArgs& a, int bn, int rows, float* ymain, cu
     ec.ec_only = 1;
     ec.y = nullptr;
     ec.y_fp32 = 1;
-    TcArgs mn = a;                        // main tiles alone: ymain = s[n] D
-    mn.rank = 0;
-    mn.A = mn.B = mn.wg = nullptr;
-    mn.u = nullptr;
-    mn.mlp = GateMlp{};
-    mn.y = ymain;
-    mn.y_fp32 = 1;
-    mn.ec_only = 0;
 
     // Fork: the side stream starts after all the work already in the caller's stream (the previous
     // call's join read u).  Once forked, the join is always recorded and waited for, so that a
@@ -195,12 +187,41 @@ cudaError_t launch_semifused(const TcArgs& a, int bn, int rows, float* ymain, cu
     cudaError_t first = launch_tc05(ec, 128, 128, L.stream, false, L.priority);
     e = cudaEventRecord(L.join, L.stream);
     if (e != cudaSuccess) return first != cudaSuccess ? first : e;
-    const cudaError_t m = launch_tc05(mn, bn, rows, stream, false, 0);
+    const cudaError_t m = main(ctx, stream);
     if (first == cudaSuccess) first = m;
     e = cudaStreamWaitEvent(stream, L.join, 0);
     if (first == cudaSuccess) first = e;
     if (first != cudaSuccess) return first;
     return launch_ec_up_add(a, ymain, stream);
+}
+
+}  // namespace spear
+
+namespace spear {
+
+// The semi-fused prefill path: the tcgen05 kernel's main tiles alone write the main term.
+struct Tc05Main {
+    TcArgs a;
+    int bn, rows;
+};
+static cudaError_t tc05_main(const void* ctx, cudaStream_t stream) {
+    const Tc05Main* c = static_cast<const Tc05Main*>(ctx);
+    return launch_tc05(c->a, c->bn, c->rows, stream, false, 0);
+}
+
+cudaError_t launch_semifused(const TcArgs& a, int bn, int rows, float* ymain, cudaStream_t stream) {
+    Tc05Main c;
+    c.a = a;                              // main tiles alone, no compensator: ymain = s[n] D
+    c.a.rank = 0;
+    c.a.A = c.a.B = c.a.wg = nullptr;
+    c.a.u = nullptr;
+    c.a.mlp = GateMlp{};
+    c.a.y = ymain;
+    c.a.y_fp32 = 1;
+    c.a.ec_only = 0;
+    c.bn = bn;
+    c.rows = rows;
+    return launch_ec_beside(a, tc05_main, &c, ymain, stream);
 }
 
 }  // namespace spear
