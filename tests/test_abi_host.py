@@ -234,3 +234,34 @@ def test_grouped_host_checks():
     assert gemm(ec=ctypes.byref(big)) == SHAPE
     e16 = spear.spear_ec(0x7000, 0x8000, 0x9000, 0.0, 16)
     assert gemm(ec=ctypes.byref(e16), ws_bytes=(128 + 1024) * 1024) == WS_SMALL
+
+
+def test_plan_update_decode_plans():
+    # Split-K decode plans: the separate EC pass keeps the fp32 main term of one launch (at most
+    # 256 tokens) after the zeroed part; tile and split rules are those of spear_w4ec_gemm.
+    M, N, K, r = 16, 4096, 4096, 64
+    st, p = _plan(M, N, K, r)
+    assert st == OK
+    q = spear.spear_plan.from_buffer_copy(p)
+    q.kernel_id, q.tile_n, q.split_k, q.tile_m, q.flags = 1, 32, 4, 16, 0
+    assert spear._lib.spear_plan_update(ctypes.byref(q), M, N, K, r) == OK
+    fused = q.workspace_bytes
+    assert fused == (128 + 1024) * 1024
+    q.flags = spear.SPEAR_PLAN_SEPARATE_EC
+    assert spear._lib.spear_plan_update(ctypes.byref(q), M, N, K, r) == OK
+    assert q.workspace_bytes == fused + M * N * 4
+    assert spear._lib.spear_plan_update(ctypes.byref(q), 1000, N, K, r) == OK
+    assert q.workspace_bytes == fused + 256 * N * 4
+    for field, val in (("split_k", 3), ("tile_n", 24), ("tile_m", 12), ("flags", 4)):
+        bad = spear.spear_plan.from_buffer_copy(q)
+        setattr(bad, field, val)
+        assert spear._lib.spear_plan_update(ctypes.byref(bad), M, N, K, r) == INVALID, field
+    # tcgen05: 256 weight rows need 128-token tiles and N % 256 == 0; rank at most 128.
+    t = spear.spear_plan.from_buffer_copy(q)
+    t.kernel_id, t.tile_n, t.split_k, t.tile_m, t.flags = 2, 256, 1, 128, 0
+    assert spear._lib.spear_plan_update(ctypes.byref(t), 2048, N, K, r) == OK
+    assert spear._lib.spear_plan_update(ctypes.byref(t), 2048, 4224, K, r) == INVALID
+    t.tile_m = 256
+    assert spear._lib.spear_plan_update(ctypes.byref(t), 2048, N, K, r) == INVALID
+    t.tile_n, t.tile_m = 128, 256
+    assert spear._lib.spear_plan_update(ctypes.byref(t), 2048, N, K, 144) == INVALID

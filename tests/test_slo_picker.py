@@ -109,3 +109,63 @@ def test_errors():
     # decode tokens + chunk never exceed 65536 tokens.
     c, _ = spear.spear_pick_prefill_chunk(ONE, 65500, 4096, 1e9, granule=16, lut=LINE)
     assert c == 32
+
+
+# ----------------------------------------------------------------------------- properties
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+def _py_T(samples, M):
+    """The documented reading of a latency table, restated: nondecreasing samples (larger time for
+    a repeated M, then the running maximum), linear interpolation, flat below, proportional above."""
+    if M <= 0:
+        return 0.0
+    by_m = {}
+    for m, us in samples:
+        by_m[m] = max(by_m.get(m, 0.0), us)
+    pts = sorted(by_m.items())
+    run, mono = 0.0, []
+    for m, us in pts:
+        run = max(run, us)
+        mono.append((m, run))
+    if M <= mono[0][0]:
+        return mono[0][1]
+    if M >= mono[-1][0]:
+        return mono[-1][1] * M / mono[-1][0]
+    for (m0, t0), (m1, t1) in zip(mono, mono[1:]):
+        if m0 <= M <= m1:
+            return t0 + (t1 - t0) * (M - m0) / (m1 - m0)
+
+
+_sample = st.tuples(st.integers(1, 8192), st.floats(0.5, 5000.0, allow_nan=False))
+_shape = st.tuples(st.sampled_from([(256, 512), (1024, 256), (2048, 2048)]), st.booleans(),
+                   st.lists(_sample, min_size=1, max_size=6), st.integers(0, 5))
+
+
+@settings(max_examples=80, deadline=None)
+@given(shapes=st.lists(_shape, min_size=1, max_size=4, unique_by=lambda s: (s[0], s[1])),
+       D=st.integers(0, 512), cap=st.integers(0, 9000), granule=st.sampled_from([1, 16, 64, 128, 1000]),
+       slo=st.floats(1.0, 1e5, allow_nan=False), fixed=st.floats(0.0, 500.0, allow_nan=False))
+def test_picker_properties(shapes, D, cap, granule, slo, fixed):
+    lut, lin = [], []
+    for (N, K), has_ec, samples, count in shapes:
+        lut += [(m, N, K, int(has_ec), us) for (m, us) in samples]
+        lin.append((N, K, 16 if has_ec else 0, count))
+    step = lambda M: fixed + sum(c * _py_T([(m, us) for (m, n, k, e, us) in lut if (n, k, e) == (N, K, int(r > 0))], M)
+                                 for (N, K, r, c) in lin)
+    for M in (0, 1, D, D + 7, 4096, 65536):
+        got = spear.spear_predict_step_us(lin, M, fixed_us=fixed, lut=lut)
+        assert math.isclose(got, step(M), rel_tol=1e-9, abs_tol=1e-9), M
+    chunk, pred = spear.spear_pick_prefill_chunk(lin, D, cap, slo, granule=granule, fixed_us=fixed, lut=lut)
+    room = min(cap, 65536 - D)
+    assert chunk % granule == 0 and 0 <= chunk <= room
+    assert math.isclose(pred, step(D + chunk), rel_tol=1e-9, abs_tol=1e-9)
+    if step(D) <= slo:
+        assert pred <= slo
+        if chunk + granule <= room:
+            assert step(D + chunk + granule) > slo
+    else:
+        assert chunk == 0
+    a, b = sorted((D, D + chunk + 3))
+    assert spear.spear_predict_step_us(lin, a, fixed_us=fixed, lut=lut) <= \
+        spear.spear_predict_step_us(lin, b, fixed_us=fixed, lut=lut) + 1e-9

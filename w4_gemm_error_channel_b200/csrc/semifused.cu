@@ -10,7 +10,8 @@
 //   caller's stream, after both                     ec_up_add_kernel:                 y = ymain + u B
 //
 // When the caller captures its stream into a CUDA graph, the first two launches become parallel
-// branches and the third joins them.  The arithmetic is the fused path's (the same bf16 u, the same
+// branches and the third joins them.  launch_ec_beside is the fork/join with any main-term launch;
+// the group-wise-scale layer (grouped.cu) uses it too.  The arithmetic is the fused path's (the same bf16 u, the same
 // fp32 main term); only the last sum takes two fp32 roundings (s[n] D, then + u B) where the fused
 // epilogue takes one multiply-add, before the single rounding to y's type.
 #include <mutex>
