@@ -35,6 +35,10 @@
  * Packing: byte b of row n holds q[n,2b] in bits 0..3 and q[n,2b+1] in bits 4..7.
  * s and z are stored as IEEE binary16 bit patterns (z is an exact integer).
  *
+ * Also here: the group-wise variant (scale and zero-point per group of G consecutive k of a row,
+ * the per-channel steps applied to each group; oracle_w4ec_gemm_grouped) and the pages'
+ * bottleneck-MLP gate (oracle_w4ec_gemm_mlp).
+ *
  * Everything after quantisation runs in fp64, sums in ascending index order.
  *
  * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -fopenmp -shared -fPIC.
