@@ -527,7 +527,7 @@ def _sweep_shape(torch, spear, L, batches):
         base = spear.spear_gemm_plan(M, N, K, r)
         # Room for the tcgen05 kernel's u buffer (bf16 [M, r]) and the fp32 main term of the
         # separate EC pass ([min(M, 256), N]) or of the semi-fused prefill path ([M, N]).
-        ws = spear.alloc_workspace(base.workspace_bytes + (M * r * 2 + 255) // 256 * 256 + M * N * 4)
+        ws = spear.alloc_workspace(base.workspace_bytes + (M * r * 2 + 255) // 256 * 256 + M * N * 4 + (8 << 20))
         # (kernel, tile_n, split_k, flags[, tile_m]): every split-K decode tiling, fused and with the
         # separate EC pass, and the tcgen05 kernel with 128- or 256-token tiles, fused and
         # semi-fused (flags 1).
@@ -535,15 +535,20 @@ def _sweep_shape(torch, spear, L, batches):
                                            for split in (1, 2, 4, 8) for fl in (0, 1)]
         for fl in ((0, 1) if M >= 128 else (0,)):
             candidates += [(2, 128, 1, fl, 128)] + ([(2, 128, 1, fl, 256)] if M >= 256 else [])
+        # The stream-K kernel (kernel 3) up to 64 tokens: token tile, K codes per stage, and the ring
+        # mode (flags 2: one CTA per SM with a deep ring).
+        if M <= 64:
+            bn = 16 if M <= 16 else (32 if M <= 32 else 64)
+            candidates += [(3, 128, kc, fl, bn) for kc in (128, 256) for fl in (0, 2) if K % kc == 0]
         for cand in candidates:
                 kernel_id, tile_n, split, fl = cand[:4]
                 tc_tile_m = cand[4] if len(cand) > 4 else None
                 for use_ec in (True, False):
-                    if fl and not use_ec:
+                    if (fl & spear.SPEAR_PLAN_SEPARATE_EC) and not use_ec:
                         continue
                     plan = spear.spear_plan.from_buffer_copy(base)
                     plan.kernel_id, plan.tile_n, plan.split_k, plan.flags = kernel_id, tile_n, split, fl
-                    if kernel_id == 2:
+                    if kernel_id in (2, 3):
                         plan.tile_m = tc_tile_m
                     elif base.kernel_id == 2:
                         plan.tile_m = 8 if M <= 8 else (16 if M <= 16 else 32)
@@ -558,6 +563,15 @@ def _sweep_shape(torch, spear, L, batches):
                             call(0)
                         stream.synchronize()
                     except spear.SpearError:
+                        continue
+                    desc = (f"M={M} N={N} K={K} ec={int(use_ec)} kernel={kernel_id} tile_n={tile_n} split_k={split} "
+                            f"tile_m={plan.tile_m} flags={fl}")
+                    err = spear.spear_get_device_status(ws, clear=True, stream=stream)
+                    if err != spear.SPEAR_OK:
+                        # A bounded in-kernel wait gave up: report it and do not time this plan.
+                        print(f"sweep: {desc}: device status {err}, skipped", file=sys.stderr, flush=True)
+                        ws.zero_()
+                        torch.cuda.synchronize()
                         continue
                     g = torch.cuda.CUDAGraph()
                     with torch.cuda.stream(stream):
@@ -574,6 +588,7 @@ def _sweep_shape(torch, spear, L, batches):
                         e1.synchronize()
                         best = min(best, e0.elapsed_time(e1) * 1e3 / n_calls)
                     del g
+                    print(f"sweep: {desc}: {best:.2f} us", file=sys.stderr, flush=True)
                     rows.append({"M": M, "N": N, "K": K, "rank": r if use_ec else 0, "kernel": kernel_id, "flags": fl,
                                  "tile_n": tile_n, "tile_m": plan.tile_m,
                                  "split_k": split, "us": best,

@@ -63,7 +63,14 @@ typedef enum {
     SPEAR_KERNEL_AUTO = 0,      /* let spear_gemm_plan decide */
     SPEAR_KERNEL_SPLITK = 1,    /* decode: split-K weight-streaming kernel (mma.sync on registers); EC
                                    CTAs of the same launch reduce x A through int64 accumulators */
-    SPEAR_KERNEL_TC05 = 2       /* prefill: TMA + tcgen05/TMEM kernel, EC applied in its epilogue */
+    SPEAR_KERNEL_TC05 = 2,      /* prefill: TMA + tcgen05/TMEM kernel, EC applied in its epilogue */
+    SPEAR_KERNEL_STREAM = 3     /* decode and small batches (M <= 64): persistent stream-K TMA + tcgen05
+                                   kernel; every SM streams an equal share of the weight tiles' K chunks,
+                                   partial tiles meet through the workspace in a fixed order, and the
+                                   compensator is fused (its x A split over the CTAs, u B on the tensor
+                                   cores).  Plan fields: tile_n = 128 (weight rows per tile), tile_m =
+                                   16, 32 or 64 (token tile, >= M), split_k = K codes per pipeline stage
+                                   (128 or 256, dividing K).  The scalar gate only. */
 } spear_kernel;
 
 /* spear_plan.flags bits. */
@@ -79,7 +86,12 @@ enum {
      * third kernel adds u B and rounds y.  The call forks and joins through events, so a CUDA
      * graph captured from the caller's stream holds the two as parallel branches (a static DAG).
      * Concurrent calls from several host threads are ordered by a lock around the enqueue. */
-    SPEAR_PLAN_SEPARATE_EC = 1
+    SPEAR_PLAN_SEPARATE_EC = 1,
+    /* SPEAR_KERNEL_STREAM only: one CTA per SM with a deep weight ring (up to 227 KB of shared
+     * memory, 512 TMEM columns) instead of a ring small enough for two CTAs per SM.  The deep ring
+     * keeps more weight bytes in flight (large layers); the small one lets the next call's CTAs
+     * start their weight stream on the same SMs while this call finishes (small layers). */
+    SPEAR_PLAN_DEEP_RING = 2
 };
 
 /* Error compensator of one layer.  Pass NULL for a layer without EC (section
@@ -108,8 +120,9 @@ typedef struct {
  * SPEAR_ERR_INVALID_ARG. */
 typedef struct {
     int32_t kernel_id;        /* spear_kernel */
-    int32_t tile_n;           /* weight rows per CTA */
-    int32_t split_k;          /* number of K slices (1 = none), reduced in a thread-block cluster */
+    int32_t tile_n;           /* weight rows per CTA (per tile for SPEAR_KERNEL_STREAM) */
+    int32_t split_k;          /* number of K slices (1 = none), reduced in a thread-block cluster;
+                                 SPEAR_KERNEL_STREAM: K codes per pipeline stage */
     int32_t tile_m;           /* token rows per CTA (or per launch chunk) */
     int32_t flags;            /* SPEAR_PLAN_* bits; 0 = none */
     int32_t reserved;
@@ -212,17 +225,28 @@ SPEAR_API spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, in
  *   select SPEAR_KERNEL_SPLITK.
  *   Limits: 1 <= M <= 64 (larger M returns SPEAR_ERR_UNSUPPORTED_SHAPE), rank 0 or 16..256, the
  *   scalar gate only (ec->gate_w1 != NULL returns SPEAR_ERR_INVALID_ARG).
+ *   plan == NULL plans the split-K decode kernel for the shape (never another kernel).
  *   The first call on a device looks up that device's scratch address (once per device, with the
- *   device current); make that first call before any stream capture.  Every call first clears the
- *   part of the scratch it uses, then launches the fused decode kernel.
+ *   device current); make that first call before any stream capture.  The array starts zeroed
+ *   and each completed call leaves its counters and accumulators zeroed again, so a call clears
+ *   nothing before its launch.
  *   All calls share the one array and it keeps the last call's contents: calls that can overlap
  *   on the GPU (different streams, or different host threads) race and must be serialised by the
- *   caller.  Errors from bounded in-kernel waits are not reported by this call; run the same
- *   problem through spear_w4ec_gemm and spear_get_device_status to diagnose one.
+ *   caller.  Timeouts of bounded in-kernel waits are read (and the array reset after one) with
+ *   spear_noalloc_get_device_status.
  */
 SPEAR_API spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const void* x, int64_t M, int64_t N,
                                                int64_t K, const void* packed, const void* scale, const void* zero,
                                                const spear_ec* ec, void* y, spear_dtype y_dtype, void* stream);
+
+/*
+ * spear_noalloc_get_device_status -- the error word of spear_w4ec_gemm_noalloc's array (the
+ * timeouts of its bounded in-kernel waits), as spear_get_device_status reads a workspace's.  With
+ * clear != 0 and a nonzero word, the whole array is zeroed, so that the next call starts clean.
+ * Synchronises `stream`; order it after the calls it should observe.  Allocates nothing.
+ * Returns SPEAR_OK, SPEAR_ERR_TIMEOUT, or SPEAR_ERR_CUDA.
+ */
+SPEAR_API spear_status spear_noalloc_get_device_status(int clear, void* stream);
 
 /*
  * Group-wise scales (section 3.1: the method sits on GPTQ, AWQ and OmniQuant backends as well as

@@ -1,0 +1,265 @@
+"""The small-batch stream-K kernel (SPEAR_KERNEL_STREAM) against the CPU oracle, through the C ABI.
+
+Every token tile (16, 32, 64), pipeline-stage width (64, 128, 256 codes) and ring mode (two CTAs
+per SM, or one with a deep ring) is run with explicit plans; the tolerance is the one of
+tests/gpu_helpers.py.  The tiles that straddle CTAs meet in a fixed order, so repeated calls are
+bit-identical, and a compensator whose gate is exactly 0 gives the plain layer bit for bit.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synthetic import config_layers, make_layer
+from gpu_helpers import check_close, host_f64, to_dev, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import w4_gemm_error_channel_b200 as spear
+else:
+    spear = None
+
+ZEROED = (128 + 1024) * 1024          # control block + EC accumulators: zero at rest
+
+
+def stream_plan(M, N, K, rank, bn, kc, deep):
+    p = spear.spear_plan()
+    p.kernel_id, p.tile_n, p.tile_m, p.split_k = spear.SPEAR_KERNEL_STREAM, 128, bn, kc
+    p.flags = spear.SPEAR_PLAN_DEEP_RING if deep else 0
+    return spear.spear_plan_update(p, M, N, K, rank)
+
+
+class Dev:
+    def __init__(self, L):
+        self.L = L
+        self.packed, self.scale, self.zero = spear.spear_pack_w4(to_dev(L.W))
+        self.ec = None
+        if L.rank > 0:
+            self.ec = spear.EC(to_dev_bf16(L.A_bits), to_dev_bf16(L.B_bits), to_dev_bf16(L.wg_bits), L.b_g)
+        self.xd = {}
+
+    def x(self, M):
+        if M not in self.xd:
+            self.xd[M] = to_dev_bf16(self.L.x(M))
+        return self.xd[M]
+
+    def run(self, M, plan, ws, y_dtype=torch.bfloat16, ec="same", y=None, stream=None):
+        e = self.ec if ec == "same" else ec
+        return spear.spear_w4ec_gemm(self.x(M), self.packed, self.scale, self.zero, e, y=y, y_dtype=y_dtype,
+                                     plan=plan, workspace=ws, stream=stream)
+
+    def ref(self, M, rows=None, ec=True):
+        L = self.L
+        x = L.x(M) if rows is None else L.x(M)[rows]
+        p, s, z = oracle.pack_w4(L.W)
+        if ec and L.rank > 0:
+            return oracle.w4ec_gemm(x, p, s, z, L.A_bits, L.B_bits, L.wg_bits, L.b_g)
+        return oracle.w4ec_gemm(x, p, s, z)
+
+
+@functools.lru_cache(maxsize=None)
+def dev(idx, li=0, layer=None):
+    layers = (layer,) if layer is not None else None
+    return Dev(config_layers(idx, layers=layers)[li])
+
+
+def tilings(M, K, ec_rank):
+    out = []
+    for bn in (16, 32, 64):
+        if M > bn:
+            continue
+        for kc in (128, 256):
+            if K % kc:
+                continue
+            for deep in (False, True):
+                out.append((bn, kc, deep))
+    return out
+
+
+def ok_status(ws):
+    assert spear.spear_get_device_status(ws) == 0, "a bounded wait timed out"
+    assert int(ws[:ZEROED].count_nonzero().item()) == 0, "control words or accumulators not re-armed"
+
+
+def _configurable(M, L, bn, kc, deep):
+    try:
+        return stream_plan(M, L.N, L.K, L.rank, bn, kc, deep)
+    except spear.SpearError:
+        return None
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_tiny_every_tiling(M):
+    d = dev(0)
+    L = d.L
+    ref = d.ref(M)
+    ref_plain = d.ref(M, ec=False)
+    for bn, kc, deep in tilings(M, L.K, L.rank):
+        plan = _configurable(M, L, bn, kc, deep)
+        if plan is None:
+            continue
+        ws = spear.alloc_workspace(plan.workspace_bytes)
+        what = f"tiny M={M} bn={bn} kc={kc} deep={deep}"
+        check_close(host_f64(d.run(M, plan, ws)), ref, True, what)
+        check_close(host_f64(d.run(M, plan, ws, y_dtype=torch.float32)), ref, False, what + " fp32")
+        plain = stream_plan(M, L.N, L.K, 0, bn, kc, deep)
+        check_close(host_f64(d.run(M, plain, ws, ec=None)), ref_plain, True, what + " no EC")
+        ok_status(ws)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_qo(M):
+    d = dev(1)
+    L = d.L
+    ref = d.ref(M)
+    for bn, kc, deep in [(16, 128, False), (16, 256, False), (16, 256, True), (32, 128, False), (64, 128, True)]:
+        if M > bn:
+            continue
+        plan = stream_plan(M, L.N, L.K, L.rank, bn, kc, deep)
+        ws = spear.alloc_workspace(plan.workspace_bytes)
+        what = f"decode-qo M={M} bn={bn} kc={kc} deep={deep}"
+        check_close(host_f64(d.run(M, plan, ws)), ref, True, what)
+        check_close(host_f64(d.run(M, plan, ws, y_dtype=torch.float32)), ref, False, what + " fp32")
+        ok_status(ws)
+
+
+@pytest.mark.parametrize("M", [1, 8, 32, 64])
+def test_decode_mlp_sampled_rows(M):
+    d = dev(2)
+    L = d.L
+    rows = np.arange(M) if M <= 8 else np.array([0, 3, M // 2, M - 1])
+    ref = d.ref(M, rows=rows)
+    bn = 16 if M <= 16 else (32 if M <= 32 else 64)
+    for kc, deep in [(256, True), (128, False), (128, True)]:
+        plan = _configurable(M, L, bn, kc, deep)
+        if plan is None:
+            continue
+        ws = spear.alloc_workspace(plan.workspace_bytes)
+        y = host_f64(d.run(M, plan, ws))
+        check_close(y[rows], ref, True, f"decode-mlp M={M} kc={kc} deep={deep}")
+        assert np.isfinite(y).all()
+        ok_status(ws)
+
+
+@pytest.mark.parametrize("li", [0, 1, 2, 3])
+@pytest.mark.parametrize("layer", [0, 2])           # layer 0 carries a compensator, layer 2 does not
+def test_sweep_linears(layer, li):
+    d = dev(4, li=li, layer=layer)
+    L = d.L
+    for M in (1, 16):
+        ref = d.ref(M)
+        plan = stream_plan(M, L.N, L.K, L.rank, 16, 128, False)
+        ws = spear.alloc_workspace(plan.workspace_bytes)
+        check_close(host_f64(d.run(M, plan, ws)), ref, True, f"sweep L{layer}.{li} M={M}")
+        ok_status(ws)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 7, 9, 15, 16, 17, 31, 33, 47, 63, 64])
+@pytest.mark.parametrize("r", [0, 16, 48, 256])
+def test_ragged_shapes(M, r):
+    # N = 384: three tiles; K = 640 = 5 stages of 128 codes, so tiles straddle CTAs unevenly.
+    L = make_layer("stream-ragged", 91 + r, 64, 384, 640, r, outlier_frac=0.02, outlier_scale=10.0, b_g=0.5)
+    d = Dev(L)
+    ref = d.ref(M)
+    bn = 16 if M <= 16 else (32 if M <= 32 else 64)
+    for deep in (False, True):
+        plan = _configurable(M, L, bn, 128, deep)
+        if plan is None:
+            continue
+        ws = spear.alloc_workspace(plan.workspace_bytes)
+        check_close(host_f64(d.run(M, plan, ws)), ref, True, f"ragged M={M} r={r} deep={deep}")
+        ok_status(ws)
+
+
+def test_gate_off_is_bitwise_plain_and_deterministic():
+    d = dev(1)
+    L = d.L
+    off = spear.EC(d.ec.A, d.ec.B, d.ec.w_g, float("-inf"))
+    for M, bn, kc in ((1, 16, 128), (16, 16, 256), (16, 32, 256)):
+        plan = stream_plan(M, L.N, L.K, L.rank, bn, kc, False)
+        plain = stream_plan(M, L.N, L.K, 0, bn, kc, False)
+        ws = spear.alloc_workspace(plan.workspace_bytes)
+        y_plain = d.run(M, plain, ws, ec=None, y_dtype=torch.float32)
+        y_off = d.run(M, plan, ws, ec=off, y_dtype=torch.float32)
+        assert torch.equal(y_plain, y_off)
+        y1, y2 = d.run(M, plan, ws), d.run(M, plan, ws)
+        assert torch.equal(y1, y2)
+        ok_status(ws)
+
+
+def test_chained_calls_in_one_stream():
+    # Back-to-back calls on one stream overlap through programmatic dependent launch: each call's
+    # weight stream starts while the previous one finishes.  Alternate two layers and two batch
+    # sizes on one workspace, then check every output.
+    d1, d0 = dev(1), dev(0)
+    stream = torch.cuda.Stream()
+    plans = {}
+    for d in (d1, d0):
+        for M in (1, 16):
+            # decode-qo: 64-code stages with the deep ring at M = 1 (a small CTA that must still hold
+            # its SM alone), 128-code stages with two CTAs per SM at M = 16
+            deep = d is d1 and M == 1
+            plans[(d.L.name, M)] = stream_plan(M, d.L.N, d.L.K, d.L.rank, 16, 128 if (d is d0 or deep) else 256, deep)
+    ws = spear.alloc_workspace(max(p.workspace_bytes for p in plans.values()))
+    seq = [(d1, 16), (d1, 16), (d0, 1), (d1, 1), (d0, 16), (d1, 16)] * 3
+    outs = []
+    with torch.cuda.stream(stream):
+        for d, M in seq:
+            outs.append(d.run(M, plans[(d.L.name, M)], ws, stream=stream))
+    stream.synchronize()
+    refs = {}
+    for (d, M), y in zip(seq, outs):
+        key = (d.L.name, M)
+        if key not in refs:
+            refs[key] = d.ref(M)
+        check_close(host_f64(y), refs[key], True, f"chained {key}")
+    ok_status(ws)
+
+
+def test_graph_replay():
+    d = dev(1)
+    L = d.L
+    plan = stream_plan(16, L.N, L.K, L.rank, 16, 128, False)
+    ws = spear.alloc_workspace(plan.workspace_bytes)
+    x = d.x(16)
+    y = torch.empty((16, L.N), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        d.run(16, plan, ws, y=y, stream=stream)          # warm-up outside the capture
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(4):
+            spear.spear_w4ec_gemm(x, d.packed, d.scale, d.zero, d.ec, y=y, plan=plan, workspace=ws, stream=stream)
+    y.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    check_close(host_f64(y), d.ref(16), True, "graph replay")
+    ok_status(ws)
+
+
+def test_rejects_bad_stream_plans():
+    d = dev(0)
+    L = d.L
+    plan = stream_plan(4, L.N, L.K, L.rank, 16, 128, False)
+    bad = spear.spear_plan.from_buffer_copy(plan)
+    bad.tile_m = 8                                       # not a token tile of this kernel
+    with pytest.raises(spear.SpearError):
+        spear.spear_plan_update(bad, 4, L.N, L.K, L.rank)
+    bad = spear.spear_plan.from_buffer_copy(plan)
+    bad.split_k = 64                                     # one sub-chunk per stage: not taken
+    with pytest.raises(spear.SpearError):
+        spear.spear_plan_update(bad, 4, L.N, L.K, L.rank)
+    with pytest.raises(spear.SpearError):                # more tokens than the tile
+        spear.spear_plan_update(spear.spear_plan.from_buffer_copy(plan), 17, L.N, L.K, L.rank)
+    H = 4
+    mlp = spear.EC(d.ec.A, d.ec.B, d.ec.w_g, 0.0,
+                   gate_w1=torch.zeros((H, L.rank), device="cuda"), gate_b1=torch.zeros(H, device="cuda"),
+                   gate_w2=torch.zeros((L.rank, H), device="cuda"), gate_b2=torch.zeros(L.rank, device="cuda"))
+    ws = spear.alloc_workspace(plan.workspace_bytes)
+    with pytest.raises(spear.SpearError):               # the MLP gate is not taken by this kernel
+        d.run(4, plan, ws, ec=mlp)

@@ -21,13 +21,13 @@ LIB_PATH = os.path.join(_PKG, "libspear.so")
 
 SPEAR_OK = 0
 SPEAR_BF16, SPEAR_FP32 = 0, 1
-SPEAR_KERNEL_AUTO, SPEAR_KERNEL_SPLITK, SPEAR_KERNEL_TC05 = 0, 1, 2
-SPEAR_PLAN_SEPARATE_EC = 1
+SPEAR_KERNEL_AUTO, SPEAR_KERNEL_SPLITK, SPEAR_KERNEL_TC05, SPEAR_KERNEL_STREAM = 0, 1, 2, 3
+SPEAR_PLAN_SEPARATE_EC, SPEAR_PLAN_DEEP_RING = 1, 2
 STATUS_NAMES = {0: "SPEAR_OK", 1: "SPEAR_ERR_INVALID_ARG", 2: "SPEAR_ERR_UNSUPPORTED_SHAPE",
                 3: "SPEAR_ERR_MISALIGNED", 4: "SPEAR_ERR_WORKSPACE_TOO_SMALL", 5: "SPEAR_ERR_CUDA",
                 6: "SPEAR_ERR_TIMEOUT"}
 EXPORTED = ["spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_plan_update", "spear_w4ec_gemm",
-            "spear_w4ec_gemm_noalloc", "spear_get_device_status", "spear_status_string", "spear_version",
+            "spear_w4ec_gemm_noalloc", "spear_noalloc_get_device_status", "spear_get_device_status", "spear_status_string", "spear_version",
             "spear_latency_table", "spear_predict_step_us", "spear_pick_prefill_chunk",
             "spear_pack_w4_grouped", "spear_grouped_workspace_bytes", "spear_w4ec_gemm_grouped"]
 
@@ -79,6 +79,7 @@ def _load():
     lib.spear_w4ec_gemm_noalloc.argtypes = [ctypes.POINTER(spear_plan), P, I64, I64, I64, P, P, P,
                                             ctypes.POINTER(spear_ec), P, ctypes.c_int, P]
     lib.spear_get_device_status.argtypes = [P, ctypes.c_int, P]
+    lib.spear_noalloc_get_device_status.argtypes = [ctypes.c_int, P]
     lib.spear_pack_w4_grouped.argtypes = [P, ctypes.c_int, I64, I64, I64, P, P, P, P]
     lib.spear_grouped_workspace_bytes.argtypes = [I64, I64, I64, I64, ctypes.c_int32,
                                                   ctypes.POINTER(ctypes.c_size_t)]
@@ -95,7 +96,8 @@ def _load():
     lib.spear_status_string.restype = ctypes.c_char_p
     lib.spear_version.restype = ctypes.c_int
     for fn in ("spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_plan_update", "spear_w4ec_gemm",
-               "spear_w4ec_gemm_noalloc", "spear_get_device_status", "spear_latency_table",
+               "spear_w4ec_gemm_noalloc", "spear_noalloc_get_device_status", "spear_get_device_status",
+               "spear_latency_table",
                "spear_predict_step_us", "spear_pick_prefill_chunk", "spear_pack_w4_grouped",
                "spear_grouped_workspace_bytes", "spear_w4ec_gemm_grouped"):
         getattr(lib, fn).restype = ctypes.c_int
@@ -343,19 +345,22 @@ def spear_w4ec_gemm(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, 
 
 
 def spear_w4ec_gemm_noalloc(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
-                            ec: Optional[EC] = None, y: Optional[torch.Tensor] = None, y_dtype=torch.bfloat16,
-                            plan: Optional[spear_plan] = None, stream=None):
+                            y: torch.Tensor, ec: Optional[EC] = None, plan: Optional[spear_plan] = None,
+                            stream=None):
     """The layer for up to 64 tokens with the library's own device scratch (no workspace).
 
-    For callers that cannot allocate device memory; calls sharing the scratch must not overlap.
+    For callers that cannot allocate device memory: y [M, N] (bf16, or fp32 for checks) is the
+    caller's, and neither this wrapper nor the C call allocates anything.  Calls sharing the
+    library's scratch must not overlap on the GPU.
     """
     _dev(x, "x")
+    _dev(y, "y")
     if x.dtype != torch.bfloat16:
         raise ValueError("x must be bf16")
     M, K = x.shape
     N = packed.shape[0]
-    if y is None:
-        y = torch.empty((M, N), dtype=y_dtype, device=x.device)
+    if y.dtype not in (torch.bfloat16, torch.float32) or tuple(y.shape) != (M, N):
+        raise ValueError("y must be a contiguous bf16 or fp32 [M, N] tensor")
     yd = SPEAR_FP32 if y.dtype == torch.float32 else SPEAR_BF16
     ec_c = ctypes.byref(ec.as_c()) if ec is not None else None
     plan_c = ctypes.byref(plan) if plan is not None else None
@@ -432,6 +437,11 @@ class W4ECLayer:
 
 def spear_get_device_status(workspace: torch.Tensor, clear: bool = True, stream=None) -> int:
     return int(_lib.spear_get_device_status(_p(workspace), int(clear), _stream(stream)))
+
+
+def spear_noalloc_get_device_status(clear: bool = True, stream=None) -> int:
+    """Error word of spear_w4ec_gemm_noalloc's library-owned array (SPEAR_OK or SPEAR_ERR_TIMEOUT)."""
+    return int(_lib.spear_noalloc_get_device_status(int(clear), _stream(stream)))
 
 
 def loaded_library_path() -> str:

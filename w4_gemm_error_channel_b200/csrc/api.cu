@@ -77,8 +77,13 @@ size_t tc05_u_bytes(int64_t M, int32_t rank) { return ((size_t)M * rank * 2 + 25
 
 // Workspace: the zeroed prefix (control block + EC accumulators); split-K partial sums meet in
 // distributed shared memory.  The prefill kernel with a compensator also keeps u (bf16 [M][r]).
-size_t workspace_bytes_for(const spear_plan& p, int64_t M, int64_t N_for_ws, int32_t rank) {
+size_t workspace_bytes_for(const spear_plan& p, int64_t M, int64_t N_for_ws, int64_t K, int32_t rank, int sms) {
     size_t b = ZEROED_BYTES;
+    if (p.kernel_id == SPEAR_KERNEL_STREAM) {
+        // fp32 partial sums of the tiles that straddle two CTAs: [grid][tile_m][128].
+        const int grid = p.split_k > 0 && K % p.split_k == 0 ? stream_grid(N_for_ws, K, p.split_k, sms) : 0;
+        return b + (size_t)grid * p.tile_m * 128 * 4;
+    }
     if (p.kernel_id == SPEAR_KERNEL_TC05 && rank > 0) b += tc05_u_bytes(M, rank);
     if (p.kernel_id == SPEAR_KERNEL_TC05 && (p.flags & SPEAR_PLAN_SEPARATE_EC) && rank > 0)
         b += (size_t)M * N_for_ws * 4;                                              // fp32 main term
@@ -103,7 +108,10 @@ const MeasuredPlan kMeasured[] = {
 #include "plan_table.inc"
 };
 
-bool lookup_measured(int64_t M, int64_t N, int64_t K, int has_ec, int sms, spear_plan* p) {
+spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K, int32_t rank);
+
+bool lookup_measured(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spear_plan* p) {
+    const int has_ec = rank > 0 ? 1 : 0;
     const int nb = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
     const MeasuredPlan* best = nullptr;
     for (const MeasuredPlan& e : kMeasured) {
@@ -114,6 +122,19 @@ bool lookup_measured(int64_t M, int64_t N, int64_t K, int has_ec, int sms, spear
         if (!best || std::llabs(e.M - M) < std::llabs(best->M - M)) best = &e;
     }
     if (!best) return false;
+    if (best->kernel_id == SPEAR_KERNEL_STREAM) {
+        // The measured stage width and ring mode; the token tile must hold M.
+        const int bn = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+        if (M > 64 || K % best->split_k != 0) return false;
+        p->kernel_id = SPEAR_KERNEL_STREAM;
+        p->tile_n = 128;
+        p->split_k = best->split_k;
+        p->tile_m = best->tile_m > bn ? best->tile_m : bn;
+        p->flags = best->flags & SPEAR_PLAN_DEEP_RING;
+        p->reserved = 0;
+        if (validate_plan(*p, M, N, K, rank) != SPEAR_OK) return false;
+        return true;
+    }
     if (best->kernel_id == SPEAR_KERNEL_TC05) {
         if (plan_tc05(M, N, sms, p) != SPEAR_OK) return false;
         if (best->tile_m == 128 || best->tile_m == 256) p->tile_m = best->tile_m;   // the measured width
@@ -128,8 +149,15 @@ bool lookup_measured(int64_t M, int64_t N, int64_t K, int has_ec, int sms, spear
     return true;
 }
 
+spear_status plan_decode_rules(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spear_plan* p);
 spear_status plan_decode(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spear_plan* p) {
-    if (lookup_measured(M, N, K, rank > 0 ? 1 : 0, sms, p)) return SPEAR_OK;
+    if (lookup_measured(M, N, K, rank, sms, p)) return SPEAR_OK;
+    return plan_decode_rules(M, N, K, rank, sms, p);
+}
+
+// The split-K decode kernel's tiling from the cost model alone.
+spear_status plan_decode_rules(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spear_plan* p) {
+    (void)rank;
     const int nb = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
     const int64_t tm = 8 * nb;
     const int64_t ml = M < LAUNCH_TOKENS_MAX ? M : LAUNCH_TOKENS_MAX;
@@ -205,7 +233,21 @@ spear_status check_grouped_shape(int64_t M, int64_t N, int64_t K, int64_t group,
 }
 
 spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K, int32_t rank) {
-    (void)M;
+    if (p.kernel_id == SPEAR_KERNEL_STREAM) {
+        if (p.flags & ~SPEAR_PLAN_DEEP_RING) return SPEAR_ERR_INVALID_ARG;
+        if (p.tile_n != 128 || !(p.tile_m == 16 || p.tile_m == 32 || p.tile_m == 64) || M > p.tile_m)
+            return SPEAR_ERR_INVALID_ARG;
+        if (!(p.split_k == 128 || p.split_k == 256) || K % p.split_k != 0) return SPEAR_ERR_INVALID_ARG;
+        // The tiling must fit the ring mode's shared memory and TMEM (checked as the launch will).
+        StreamArgs a = {};
+        a.M = M > 0 ? M : 1;
+        a.N = N;
+        a.K = K;
+        a.rank = rank;
+        a.grid = stream_grid(N, K, p.split_k, device_sms(-1));
+        if (!stream_configure(a, p.tile_m, p.split_k, (p.flags & SPEAR_PLAN_DEEP_RING) != 0)) return SPEAR_ERR_INVALID_ARG;
+        return SPEAR_OK;
+    }
     if (p.kernel_id == SPEAR_KERNEL_TC05) {
         if (rank > TC05_MAX_RANK || (p.flags & ~SPEAR_PLAN_SEPARATE_EC)) return SPEAR_ERR_INVALID_ARG;
         if ((M + p.tile_m - 1) / p.tile_m > (int64_t)TC_BLOCKS_MAX) return SPEAR_ERR_INVALID_ARG;
@@ -232,6 +274,25 @@ spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K,
 }
 
 }  // namespace
+
+namespace spear {
+// A fused split-K decode plan (SPEAR_KERNEL_SPLITK, no separate EC pass): the measured table's
+// entry for this shape when it is one, else the cost model.  Used where only that kernel can run.
+spear_status plan_split_k_decode(int64_t M, int64_t N, int64_t K, int32_t rank, spear_plan* out) {
+    spear_status st = check_shape(M, N, K, rank);
+    if (st != SPEAR_OK) return st;
+    const int sms = device_sms(-1);
+    spear_plan p = {};
+    if (!lookup_measured(M, N, K, rank, sms, &p) || p.kernel_id != SPEAR_KERNEL_SPLITK ||
+        (p.flags & SPEAR_PLAN_SEPARATE_EC)) {
+        st = plan_decode_rules(M, N, K, rank, sms, &p);
+        if (st != SPEAR_OK) return st;
+    }
+    p.workspace_bytes = workspace_bytes_for(p, M, N, K, rank, sms);
+    *out = p;
+    return SPEAR_OK;
+}
+}  // namespace spear
 
 extern "C" {
 
@@ -279,11 +340,11 @@ spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int 
     const int sms = device_sms(device);
     spear_plan p = {};
     // A measured plan for this shape (either kernel) first, then the rules.
-    if (lookup_measured(M > 0 ? M : 1, N, K, rank > 0 ? 1 : 0, sms, &p)) st = SPEAR_OK;
+    if (lookup_measured(M > 0 ? M : 1, N, K, rank, sms, &p)) st = SPEAR_OK;
     else if (use_tc05(M, rank)) st = plan_tc05(M, N, sms, &p);
     else st = plan_decode(M > 0 ? M : 1, N, K, rank, sms, &p);
     if (st != SPEAR_OK) return st;
-    p.workspace_bytes = workspace_bytes_for(p, M, N, rank);
+    p.workspace_bytes = workspace_bytes_for(p, M, N, K, rank, sms);
     *out = p;
     return SPEAR_OK;
 }
@@ -294,7 +355,7 @@ spear_status spear_plan_update(spear_plan* plan, int64_t M, int64_t N, int64_t K
     if (st != SPEAR_OK) return st;
     st = validate_plan(*plan, M, N, K, rank);
     if (st != SPEAR_OK) return st;
-    plan->workspace_bytes = workspace_bytes_for(*plan, M, N, rank);
+    plan->workspace_bytes = workspace_bytes_for(*plan, M, N, K, rank, device_sms(-1));
     return SPEAR_OK;
 }
 
@@ -320,18 +381,24 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
     if (M == 0) return SPEAR_OK;
 
     const int sms = device_sms(-1);
+    const bool mlp_gate = ec && ec->gate_w1;
     spear_plan p;
     if (plan) {
         p = *plan;
+        if (mlp_gate && p.kernel_id == SPEAR_KERNEL_STREAM) return SPEAR_ERR_INVALID_ARG;   // scalar gate only
     } else {
-        if (lookup_measured(M, N, K, rank > 0 ? 1 : 0, sms, &p)) st = SPEAR_OK;
+        if (lookup_measured(M, N, K, rank, sms, &p)) st = SPEAR_OK;
         else if (use_tc05(M, rank)) st = plan_tc05(M, N, sms, &p);
         else st = plan_decode(M, N, K, rank, sms, &p);
+        if (st != SPEAR_OK) return st;
+        // The stream kernel takes the scalar gate only: the bottleneck-MLP gate runs on the
+        // split-K decode kernel.
+        if (mlp_gate && p.kernel_id == SPEAR_KERNEL_STREAM) st = plan_decode_rules(M, N, K, rank, sms, &p);
         if (st != SPEAR_OK) return st;
     }
     st = validate_plan(p, M, N, K, rank);
     if (st != SPEAR_OK) return st;
-    if (workspace_bytes < workspace_bytes_for(p, M, N, rank)) return SPEAR_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace_bytes < workspace_bytes_for(p, M, N, K, rank, sms)) return SPEAR_ERR_WORKSPACE_TOO_SMALL;
 
     cudaStream_t s = (cudaStream_t)stream;
     unsigned char* ws = (unsigned char*)workspace;
@@ -364,6 +431,32 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         else
             e = launch_tc05(t, p.tile_m, p.tile_n, s);
         return e == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
+    }
+    if (p.kernel_id == SPEAR_KERNEL_STREAM) {
+        StreamArgs a = {};
+        a.x = (const uint16_t*)x;
+        a.packed = (const uint8_t*)packed;
+        a.scale = (const __half*)scale;
+        a.zero = (const __half*)zero;
+        a.A = ec ? (const uint16_t*)ec->A : nullptr;
+        a.B = ec ? (const uint16_t*)ec->B : nullptr;
+        a.wg = ec ? (const uint16_t*)ec->w_g : nullptr;
+        a.b_g = ec ? ec->b_g : 0.0f;
+        a.rank = rank;
+        a.y = y;
+        a.y_fp32 = (y_dtype == SPEAR_FP32);
+        a.M = M;
+        a.N = N;
+        a.K = K;
+        a.grid = stream_grid(N, K, p.split_k, sms);
+        if (!stream_configure(a, p.tile_m, p.split_k, (p.flags & SPEAR_PLAN_DEEP_RING) != 0))
+            return SPEAR_ERR_INVALID_ARG;
+        a.tacc = (long long*)(ws + CTRL_BYTES);
+        a.err = ctrl;
+        a.flags = ctrl + STREAM_FLAGS_WORD;
+        a.ec_readers = ctrl + STREAM_FLAGS_WORD + STREAM_GRID_MAX;
+        a.partial = (float*)(ws + ZEROED_BYTES);
+        return launch_stream(a, p.tile_m, s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
     }
     const int nb = nb_for_tile_m(p.tile_m);
     const int g = p.tile_n / 16;

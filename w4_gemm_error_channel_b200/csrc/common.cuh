@@ -93,6 +93,12 @@ SPEAR_DEVI uint4 ldg_u4(const void* p) {
     return v;
 }
 
+SPEAR_DEVI uint32_t ldg_u32_nc(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 // ---------------------------------------------------------------------------------------------
 // Programmatic dependent launch controls (no-ops when the grid was launched without PDL).
 // ---------------------------------------------------------------------------------------------

@@ -792,14 +792,11 @@ size_t apply_dyn_smem_bytes(int rank, int gate_hidden) {
 
 cudaError_t launch_apply(const DecodeArgs& a, cudaStream_t stream) {
     const size_t dyn = apply_dyn_smem_bytes(a.rank, a.mlp.w1 ? a.mlp.hidden : 0);
-    static size_t opted[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dyn > 48 * 1024 && dev >= 0 && dev < 64 && dyn > opted[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(w4ec_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
-        if (e != cudaSuccess) return e;
-        opted[dev] = dyn;
-    }
+    // The limit is raised to this launch's size when it is below (thread-safe, per device).
+    static std::mutex mu;
+    static size_t opted[kMaxDevices] = {0};
+    cudaError_t oe = opt_in_smem_at_least((const void*)w4ec_apply_kernel, dyn, mu, opted);
+    if (oe != cudaSuccess) return oe;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.N / AP_ROWS));
     cfg.blockDim = dim3(AP_ROWS);
@@ -839,16 +836,11 @@ static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     static_assert(WPW * G <= 8, "weight registers");
     const unsigned grid = (unsigned)(a.ec_ctas + a.row_tiles * a.split * a.mchunks);
     const size_t dyn = decode_dyn_smem_bytes(NB, G, a.ec_jr, a.rank, a.mlp.w1 ? a.mlp.hidden : 0);
-    // Static plus dynamic shared memory above 48 KB needs the opt-in attribute (per device).
-    static size_t opted[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dyn > 0 && dev >= 0 && dev < 64 && dyn > opted[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(w4ec_decode_kernel<NB, G, WPW>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
-        if (e != cudaSuccess) return e;
-        opted[dev] = dyn;
-    }
+    // Static plus dynamic shared memory above 48 KB needs the opt-in attribute (once per device).
+    static std::mutex mu;
+    static size_t opted[kMaxDevices] = {0};
+    cudaError_t oe = opt_in_smem_at_least((const void*)w4ec_decode_kernel<NB, G, WPW>, dyn, mu, opted);
+    if (oe != cudaSuccess) return oe;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(DK_THREADS);

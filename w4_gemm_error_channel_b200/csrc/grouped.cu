@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(GW_THREADS) w4g_gemm_kernel(GroupedArgs a) {
 template <int NB, int RG>
 static cudaError_t launch_w4g_t(const GroupedArgs& a, cudaStream_t stream) {
     const dim3 grid((unsigned)(a.N / (16 * RG)), (unsigned)((a.M + 8 * NB - 1) / (8 * NB)));
+    cudaGetLastError();   // report this launch only, not an earlier call's error
     w4g_gemm_kernel<NB, RG><<<grid, GW_THREADS, 0, stream>>>(a);
     return cudaGetLastError();
 }

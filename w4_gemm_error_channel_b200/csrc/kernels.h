@@ -1,12 +1,31 @@
 // kernels.h -- internal launch interface between the C ABI (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
+#include "../../include/spear.h"
+
 namespace spear {
+
+// Host helpers shared by the kernels' launchers (tc05.cu).
+constexpr int kMaxDevices = 64;
+// 2-D tensor map over a row-major [rows][cols] array of `elem`-byte elements, box {box_cols, box_rows}.
+bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem, uint64_t cols,
+                 uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
+// Raise `func`'s dynamic shared-memory limit to `bytes` once per device (thread-safe); `once` and
+// `status` are per-function arrays of kMaxDevices entries.
+cudaError_t opt_in_smem(const void* func, size_t bytes, std::once_flag* once, cudaError_t* status);
+// For kernels whose dynamic size varies per launch (and that may also use static shared memory):
+// raise the limit to `bytes` if it is below, under `mu`; opted[] holds the limit set per device.
+cudaError_t opt_in_smem_at_least(const void* func, size_t bytes, std::mutex& mu, size_t* opted);
+// Largest dynamic shared memory of a block on sm_100.
+constexpr size_t SMEM_OPTIN_MAX = 227 * 1024;
 
 // Zeroed part of every workspace: it must start zeroed and every call leaves it zeroed again
 // (unless a bounded wait timed out).
@@ -100,6 +119,46 @@ struct TcArgs {
     GateMlp mlp;            // bottleneck-MLP gate (w1 == null: the scalar gate)
     int ec_only;            // 1: launch the EC tiles alone (u only, no ready flags); 0: the whole layer
 };
+
+// Small-batch stream-K kernel (stream.cu).  The host fills the problem fields and `grid`, then
+// stream_configure() fills the tiling, shared-memory layout and compensator slicing.
+constexpr size_t STREAM_GRID_MAX = 1024;                   // CTAs (one partial-sum flag each)
+constexpr size_t STREAM_FLAGS_WORD = TC_FLAGS_WORD + 2 * TC_BLOCKS_MAX;
+static_assert(STREAM_FLAGS_WORD + STREAM_GRID_MAX + 1 <= CTRL_BYTES / 4, "control block");
+struct StreamArgs {
+    const uint16_t* x;      // bf16 [M, K]
+    const uint8_t* packed;  // [N, K/2]
+    const __half* scale;    // [N]
+    const __half* zero;     // [N]
+    const uint16_t* A;      // bf16 [K, r]   (rank == 0: no compensator)
+    const uint16_t* B;      // bf16 [r, N]
+    const uint16_t* wg;     // bf16 [K]
+    float b_g;
+    int rank;
+    void* y;
+    int y_fp32;
+    int64_t M, N, K;
+    int grid;               // CTAs (<= SMs, <= units)
+    // filled by stream_configure
+    int kc, nch, ntiles, units;     // K codes per unit, units per tile, tiles, units in all
+    int nst, na;                    // shared-memory stages, TMEM sub-chunk slots
+    int jb, nbu;                    // B rows per B unit, B units per finalised tile
+    int stage_bytes, off_u, off_a, off_wg, off_g, off_bar, smem_bytes;
+    uint32_t tmem_cols;
+    int ec_kr, ec_slices;           // rows of A per compensator slice, slices (<= grid)
+    int finalizers;                 // CTAs that finalise at least one tile
+    // workspace
+    long long* tacc;        // [M][r + 1] int64 fixed-point accumulators (zeroed part)
+    unsigned* err;          // error word
+    unsigned* flags;        // [grid] partial-sum ready flags (zeroed part)
+    unsigned* ec_readers;   // CTAs that have read the accumulators (zeroed part)
+    float* partial;         // [grid][BN][128] fp32 partial sums
+};
+int stream_grid(int64_t N, int64_t K, int kc, int sms);
+// A fused split-K decode plan for this shape (api.cu).
+spear_status plan_split_k_decode(int64_t M, int64_t N, int64_t K, int32_t rank, spear_plan* out);
+bool stream_configure(StreamArgs& a, int bn, int kc, bool deep);
+cudaError_t launch_stream(const StreamArgs& a, int bn, cudaStream_t stream);
 
 // bn = tokens per tile; rows = weight rows per tile (128, or 256 with bn = 128).  pdl: launch as a
 // programmatic dependent of the previous kernel in the stream; priority: 0 or a launch priority.

@@ -73,11 +73,14 @@ extern "C" spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const vo
         return SPEAR_ERR_MISALIGNED;
     if (ec && (!aligned16(ec->A) || !aligned16(ec->B) || !aligned16(ec->w_g))) return SPEAR_ERR_MISALIGNED;
 
+    // Without a plan, the split-K decode kernel's own plan for this shape (the dispatcher may
+    // prefer another kernel, which needs a workspace).
     spear_plan p;
     if (plan) {
         p = *plan;
-    } else if (spear_gemm_plan(M, N, K, rank, -1, &p) != SPEAR_OK) {
-        return SPEAR_ERR_INVALID_ARG;
+    } else {
+        const spear_status st = plan_split_k_decode(M, N, K, rank, &p);
+        if (st != SPEAR_OK) return st;
     }
     // Only the weight-streaming decode kernel runs here.
     if (p.kernel_id != SPEAR_KERNEL_SPLITK || p.flags != 0) return SPEAR_ERR_INVALID_ARG;
@@ -92,10 +95,10 @@ extern "C" spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const vo
     unsigned char* scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess || scratch == nullptr) return SPEAR_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
-    // The kernel re-arms its counters and accumulators, but a call that stopped on an error would
-    // leave them set: start every call from zero.
-    const size_t used = NOALLOC_CTRL_BYTES + (rank > 0 ? (size_t)M * (rank + 1) * 8 : 0);
-    if (cudaMemsetAsync(scratch, 0, used, s) != cudaSuccess) return SPEAR_ERR_CUDA;
+    // The array starts zeroed and every completed call leaves its counters and accumulators
+    // zeroed again, so nothing is cleared here (a clear would also sit between the previous
+    // kernel and this one and stop their overlap).  After a call that stopped on a timed-out
+    // wait, spear_noalloc_get_device_status(clear = 1) zeroes the array.
 
     unsigned* ctrl = reinterpret_cast<unsigned*>(scratch);
     DecodeArgs a;
@@ -128,4 +131,19 @@ extern "C" spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const vo
     a.ymain = nullptr;                                    // the compensator stays fused here
     a.mlp = GateMlp{};                                    // the scalar gate
     return launch_decode(a, nb, p.tile_n / 16, wpw_of(ksl), s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
+}
+
+extern "C" spear_status spear_noalloc_get_device_status(int clear, void* stream) {
+    unsigned char* scratch = nullptr;
+    if (scratch_address(&scratch) != cudaSuccess || scratch == nullptr) return SPEAR_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned word = 0;
+    if (cudaMemcpyAsync(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess) return SPEAR_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SPEAR_ERR_CUDA;
+    if (clear && word != 0) {
+        // A call that gave up may have left counters and accumulators set: zero the whole array.
+        if (cudaMemsetAsync(scratch, 0, NOALLOC_SCRATCH_BYTES, s) != cudaSuccess) return SPEAR_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return SPEAR_ERR_CUDA;
+    }
+    return word == 0 ? SPEAR_OK : SPEAR_ERR_TIMEOUT;
 }

@@ -155,6 +155,7 @@ cudaError_t launch_pack_w4(const void* W, bool w_is_bf16, int64_t N, int64_t K, 
                            void* zero, cudaStream_t stream) {
     const int rows_per_block = 8;
     const dim3 grid((unsigned)((N + rows_per_block - 1) / rows_per_block));
+    cudaGetLastError();   // report this launch only, not an earlier call's error
     if (w_is_bf16)
         pack_w4_kernel<uint16_t><<<grid, 256, 0, stream>>>((const uint16_t*)W, N, K, (uint8_t*)packed,
                                                            (__half*)scale, (__half*)zero);
@@ -168,6 +169,7 @@ cudaError_t launch_unpack_w4(const void* packed, const void* zero, int64_t N, in
                              void* qz_out, cudaStream_t stream) {
     const int64_t items = (K % 8 == 0) ? N * (K / 8) : N * (K / 2);
     const dim3 grid((unsigned)((items + 255) / 256));
+    cudaGetLastError();   // report this launch only, not an earlier call's error
     unpack_w4_kernel<<<grid, 256, 0, stream>>>((const uint8_t*)packed, (const __half*)zero, N, K,
                                                (uint8_t*)q_out, (uint16_t*)qz_out);
     return cudaGetLastError();

@@ -110,17 +110,12 @@ __global__ void __launch_bounds__(UA_THREADS) ec_up_add_kernel(const uint16_t* _
 
 static cudaError_t launch_ec_up_add(const TcArgs& a, const float* ymain, cudaStream_t stream) {
     if (a.rank < 16 || a.rank > UA_RANK_MAX || a.rank % 16 != 0 || a.N % UA_BN != 0) return cudaErrorInvalidValue;
-    static bool opted[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t opt_status[kMaxDevices];
+    cudaError_t e = opt_in_smem((const void*)ec_up_add_kernel, up_add_smem_bytes(UA_RANK_MAX), once, opt_status);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && !opted[dev]) {
-        e = cudaFuncSetAttribute(ec_up_add_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)up_add_smem_bytes(UA_RANK_MAX));
-        if (e != cudaSuccess) return e;
-        opted[dev] = true;
-    }
     const dim3 grid((unsigned)(a.N / UA_BN), (unsigned)((a.M + UA_BM - 1) / UA_BM));
+    cudaGetLastError();   // report this launch only, not an earlier call's error
     ec_up_add_kernel<<<grid, UA_THREADS, up_add_smem_bytes(a.rank), stream>>>(
         reinterpret_cast<const uint16_t*>(a.u), a.B, ymain, a.y, a.y_fp32, a.M, a.N, a.rank);
     return cudaGetLastError();

@@ -26,10 +26,10 @@
 // the u tile and the B slice (MN-major, from [r, N]) by TMA and accumulates E[n, m] = sum_j
 // B[j, n] u[m, j] into TMEM; the epilogue writes y = s[n] D + E.
 // Every mbarrier and flag wait is bounded: on timeout the kernel records an error bit and stops.
-#include <cuda.h>
+#include <mutex>
 
-#include "common.cuh"
 #include "kernels.h"
+#include "tcgen05.cuh"
 
 namespace spear {
 
@@ -38,126 +38,6 @@ constexpr int TC_BM = 128;               // weight rows per tile (MMA M)
 constexpr int TC_BK = 64;                // K codes per stage
 constexpr uint32_t WAIT_LIMIT = 1u << 24;
 
-// ---------------------------------------------------------------------------------------------
-// PTX wrappers
-// ---------------------------------------------------------------------------------------------
-SPEAR_DEVI uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-SPEAR_DEVI void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-SPEAR_DEVI void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-SPEAR_DEVI void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-// Bounded wait for the phase with the given parity.  Returns false after WAIT_LIMIT polls.
-SPEAR_DEVI bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    const uint32_t a = smem_u32(bar);
-    for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
-        uint32_t done;
-        asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-                     : "=r"(done) : "r"(a), "r"(parity) : "memory");
-        if (done) return true;
-    }
-    return false;
-}
-
-SPEAR_DEVI void tma_load_2d(void* dst, const CUtensorMap* map, int32_t c0, int32_t c1, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar)) : "memory");
-}
-
-// Shared memory -> global tile store (no multicast); coordinates are never negative here.
-SPEAR_DEVI void tma_store_2d(const CUtensorMap* map, const void* src, int32_t c0, int32_t c1) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
-                 ::"l"(map), "r"(smem_u32(src)), "r"(c0), "r"(c1) : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-SPEAR_DEVI void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-
-SPEAR_DEVI void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-SPEAR_DEVI void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-SPEAR_DEVI void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 bytes apart.
-SPEAR_DEVI uint64_t smem_desc_k_sw128(const void* base) {
-    const uint64_t addr = smem_u32(base);
-    uint64_t d = 0;
-    d |= (addr >> 4) & 0x3FFFull;            // start address (16-byte units)
-    d |= 1ull << 16;                         // leading byte offset (unused for swizzled K-major)
-    d |= (uint64_t)(1024 >> 4) << 32;        // stride byte offset: 8 rows x 128 bytes
-    d |= 1ull << 46;                         // descriptor version (sm_100)
-    d |= 2ull << 61;                         // layout: 128-byte swizzle
-    return d;
-}
-
-// Instruction descriptor: kind::f16 with bf16 A and B (both K-major), fp32 accumulator.
-constexpr uint32_t idesc_bf16_f32(int M, int N) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-SPEAR_DEVI void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
-}
-// A operand from TMEM (128 lanes = rows, 32-bit columns holding bf16 pairs k = 2c, 2c + 1).
-SPEAR_DEVI void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
-}
-SPEAR_DEVI void tmem_st32(uint32_t taddr, const uint32_t v[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
-          "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
-          "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-        : "memory");
-}
-SPEAR_DEVI void mma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 ::"r"(smem_u32(bar)) : "memory");
-}
-
-SPEAR_DEVI void tmem_ld16(uint32_t taddr, float v[16]) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Shared-memory matrix descriptor: MN-major, 128-byte swizzle.  The MN extent is split in groups
-// of 64 elements `lbo_bytes` apart; K rows are 128 bytes apart, 8-row groups 1024 bytes apart.
-SPEAR_DEVI uint64_t smem_desc_mn_sw128(const void* base, uint32_t lbo_bytes) {
-    const uint64_t addr = smem_u32(base);
-    uint64_t d = 0;
-    d |= (addr >> 4) & 0x3FFFull;
-    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
-    d |= (uint64_t)(1024 >> 4) << 32;
-    d |= 1ull << 46;
-    d |= 2ull << 61;
-    return d;
-}
-constexpr uint32_t IDESC_A_MN = 1u << 15;   // A operand MN-major
-
-SPEAR_DEVI unsigned ld_acquire_gpu(const unsigned* p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 SPEAR_DEVI void named_bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }   // warps 2-5
 
 // ---------------------------------------------------------------------------------------------
@@ -535,23 +415,24 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once per process (thread-safe).
 static EncodeTiledFn encode_fn() {
+    static std::once_flag once;
     static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    std::call_once(once, []() {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
             fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+        else
+            cudaGetLastError();
+    });
     return fn;
 }
 
-// 2-D tensor map over a row-major [rows][cols] array of `elem` bytes per element.
-static bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem, uint64_t cols,
-                        uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem, uint64_t cols,
+                 uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {cols, rows};
@@ -560,6 +441,30 @@ static bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t opt_in_smem_at_least(const void* func, size_t bytes, std::mutex& mu, size_t* opted) {
+    if (bytes == 0) return cudaSuccess;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (bytes <= opted[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) opted[dev] = bytes;
+    return e;
+}
+
+cudaError_t opt_in_smem(const void* func, size_t bytes, std::once_flag* once, cudaError_t* status) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [&]() {
+        status[dev] = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    });
+    return status[dev];
 }
 
 template <int BN, int STAGES, int SUB>
@@ -599,15 +504,10 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream, bool pdl, i
     } else {
         ma = mx; mb = mx; mu = mx; mg = mx;      // unused
     }
-    static bool opted[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !opted[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(w4_tc05_kernel<BN, STAGES, SUB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             L::TOTAL);
-        if (e != cudaSuccess) return e;
-        opted[dev] = true;
-    }
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t opt_status[kMaxDevices];
+    cudaError_t oe = opt_in_smem((const void*)w4_tc05_kernel<BN, STAGES, SUB>, L::TOTAL, once, opt_status);
+    if (oe != cudaSuccess) return oe;
     const unsigned mblocks = (unsigned)((a.M + BN - 1) / BN);
     const unsigned eblocks = (unsigned)((a.M + TC_EB - 1) / TC_EB);
     const unsigned tiles = a.ec_only ? eblocks : (unsigned)(a.N / (TC_BM * SUB)) * mblocks + (has_ec ? eblocks : 0u);
