@@ -540,6 +540,10 @@ def _sweep_shape(torch, spear, L, batches):
         if M <= 64:
             bn = 16 if M <= 16 else (32 if M <= 32 else 64)
             candidates += [(3, 128, kc, fl, bn) for kc in (128, 256) for fl in (0, 2) if K % kc == 0]
+            # The register-path stream kernel (kernel 4): 8-token tiles from M <= 8, 64 only deep.
+            bn_rk = 8 if M <= 8 else bn
+            candidates += [(4, 128, kc, fl, bn_rk) for kc in (128, 256) for fl in (0, 2)
+                           if K % kc == 0 and (bn_rk < 64 or fl == 2) and (r <= 128)]
         for cand in candidates:
                 kernel_id, tile_n, split, fl = cand[:4]
                 tc_tile_m = cand[4] if len(cand) > 4 else None
@@ -548,7 +552,7 @@ def _sweep_shape(torch, spear, L, batches):
                         continue
                     plan = spear.spear_plan.from_buffer_copy(base)
                     plan.kernel_id, plan.tile_n, plan.split_k, plan.flags = kernel_id, tile_n, split, fl
-                    if kernel_id in (2, 3):
+                    if kernel_id in (2, 3, 4):
                         plan.tile_m = tc_tile_m
                     elif base.kernel_id == 2:
                         plan.tile_m = 8 if M <= 8 else (16 if M <= 16 else 32)

@@ -64,13 +64,18 @@ typedef enum {
     SPEAR_KERNEL_SPLITK = 1,    /* decode: split-K weight-streaming kernel (mma.sync on registers); EC
                                    CTAs of the same launch reduce x A through int64 accumulators */
     SPEAR_KERNEL_TC05 = 2,      /* prefill: TMA + tcgen05/TMEM kernel, EC applied in its epilogue */
-    SPEAR_KERNEL_STREAM = 3     /* decode and small batches (M <= 64): persistent stream-K TMA + tcgen05
+    SPEAR_KERNEL_STREAM = 3,    /* decode and small batches (M <= 64): persistent stream-K TMA + tcgen05
                                    kernel; every SM streams an equal share of the weight tiles' K chunks,
                                    partial tiles meet through the workspace in a fixed order, and the
                                    compensator is fused (its x A split over the CTAs, u B on the tensor
                                    cores).  Plan fields: tile_n = 128 (weight rows per tile), tile_m =
                                    16, 32 or 64 (token tile, >= M), split_k = K codes per pipeline stage
                                    (128 or 256, dividing K).  The scalar gate only. */
+    SPEAR_KERNEL_STREAM_RK = 4  /* decode (M <= 64): the same stream-K schedule, workspace and fused
+                                   compensator as SPEAR_KERNEL_STREAM, with the int4 codes converted
+                                   into registers and fed to mma.sync (no TMEM staging).  tile_n = 128,
+                                   tile_m = 8, 16, 32 or 64 (>= M; 64 needs SPEAR_PLAN_DEEP_RING),
+                                   split_k = 128 or 256 (dividing K), rank <= 128, scalar gate only. */
 } spear_kernel;
 
 /* spear_plan.flags bits. */
@@ -87,7 +92,7 @@ enum {
      * graph captured from the caller's stream holds the two as parallel branches (a static DAG).
      * Concurrent calls from several host threads are ordered by a lock around the enqueue. */
     SPEAR_PLAN_SEPARATE_EC = 1,
-    /* SPEAR_KERNEL_STREAM only: one CTA per SM with a deep weight ring (up to 227 KB of shared
+    /* SPEAR_KERNEL_STREAM and _STREAM_RK: one CTA per SM with a deep weight ring (up to 227 KB of shared
      * memory, 512 TMEM columns) instead of a ring small enough for two CTAs per SM.  The deep ring
      * keeps more weight bytes in flight (large layers); the small one lets the next call's CTAs
      * start their weight stream on the same SMs while this call finishes (small layers). */

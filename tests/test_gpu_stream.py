@@ -25,9 +25,13 @@ else:
 ZEROED = (128 + 1024) * 1024          # control block + EC accumulators: zero at rest
 
 
-def stream_plan(M, N, K, rank, bn, kc, deep):
+KERNELS = ["tc", "rk"]                 # tcgen05 (converted weights in TMEM) and register (mma.sync) paths
+
+
+def stream_plan(M, N, K, rank, bn, kc, deep, kernel="tc"):
     p = spear.spear_plan()
-    p.kernel_id, p.tile_n, p.tile_m, p.split_k = spear.SPEAR_KERNEL_STREAM, 128, bn, kc
+    kid = spear.SPEAR_KERNEL_STREAM if kernel == "tc" else spear.SPEAR_KERNEL_STREAM_RK
+    p.kernel_id, p.tile_n, p.tile_m, p.split_k = kid, 128, bn, kc
     p.flags = spear.SPEAR_PLAN_DEEP_RING if deep else 0
     return spear.spear_plan_update(p, M, N, K, rank)
 
@@ -66,9 +70,9 @@ def dev(idx, li=0, layer=None):
     return Dev(config_layers(idx, layers=layers)[li])
 
 
-def tilings(M, K, ec_rank):
+def tilings(M, K, ec_rank, kernel="tc"):
     out = []
-    for bn in (16, 32, 64):
+    for bn in ((16, 32, 64) if kernel == "tc" else (8, 16, 32, 64)):
         if M > bn:
             continue
         for kc in (128, 256):
@@ -84,103 +88,112 @@ def ok_status(ws):
     assert int(ws[:ZEROED].count_nonzero().item()) == 0, "control words or accumulators not re-armed"
 
 
-def _configurable(M, L, bn, kc, deep):
+def _configurable(M, L, bn, kc, deep, kernel="tc"):
     try:
-        return stream_plan(M, L.N, L.K, L.rank, bn, kc, deep)
+        return stream_plan(M, L.N, L.K, L.rank, bn, kc, deep, kernel)
     except spear.SpearError:
         return None
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("M", [1, 4])
-def test_tiny_every_tiling(M):
+def test_tiny_every_tiling(M, kernel):
     d = dev(0)
     L = d.L
     ref = d.ref(M)
     ref_plain = d.ref(M, ec=False)
-    for bn, kc, deep in tilings(M, L.K, L.rank):
-        plan = _configurable(M, L, bn, kc, deep)
+    for bn, kc, deep in tilings(M, L.K, L.rank, kernel):
+        plan = _configurable(M, L, bn, kc, deep, kernel)
         if plan is None:
             continue
         ws = spear.alloc_workspace(plan.workspace_bytes)
-        what = f"tiny M={M} bn={bn} kc={kc} deep={deep}"
+        what = f"tiny {kernel} M={M} bn={bn} kc={kc} deep={deep}"
         check_close(host_f64(d.run(M, plan, ws)), ref, True, what)
         check_close(host_f64(d.run(M, plan, ws, y_dtype=torch.float32)), ref, False, what + " fp32")
-        plain = stream_plan(M, L.N, L.K, 0, bn, kc, deep)
+        plain = stream_plan(M, L.N, L.K, 0, bn, kc, deep, kernel)
         check_close(host_f64(d.run(M, plain, ws, ec=None)), ref_plain, True, what + " no EC")
         ok_status(ws)
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("M", [1, 4, 16])
-def test_decode_qo(M):
+def test_decode_qo(M, kernel):
     d = dev(1)
     L = d.L
     ref = d.ref(M)
-    for bn, kc, deep in [(16, 128, False), (16, 256, False), (16, 256, True), (32, 128, False), (64, 128, True)]:
+    tiles = [(16, 128, False), (16, 256, False), (16, 256, True), (32, 128, False), (64, 128, True)]
+    if kernel == "rk":
+        tiles += [(8, 128, False), (8, 256, False), (8, 256, True)]
+    for bn, kc, deep in tiles:
         if M > bn:
             continue
-        plan = stream_plan(M, L.N, L.K, L.rank, bn, kc, deep)
+        plan = stream_plan(M, L.N, L.K, L.rank, bn, kc, deep, kernel)
         ws = spear.alloc_workspace(plan.workspace_bytes)
-        what = f"decode-qo M={M} bn={bn} kc={kc} deep={deep}"
+        what = f"decode-qo {kernel} M={M} bn={bn} kc={kc} deep={deep}"
         check_close(host_f64(d.run(M, plan, ws)), ref, True, what)
         check_close(host_f64(d.run(M, plan, ws, y_dtype=torch.float32)), ref, False, what + " fp32")
         ok_status(ws)
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("M", [1, 8, 32, 64])
-def test_decode_mlp_sampled_rows(M):
+def test_decode_mlp_sampled_rows(M, kernel):
     d = dev(2)
     L = d.L
     rows = np.arange(M) if M <= 8 else np.array([0, 3, M // 2, M - 1])
     ref = d.ref(M, rows=rows)
-    bn = 16 if M <= 16 else (32 if M <= 32 else 64)
+    bn = (8 if kernel == "rk" and M <= 8 else 16) if M <= 16 else (32 if M <= 32 else 64)
     for kc, deep in [(256, True), (128, False), (128, True)]:
-        plan = _configurable(M, L, bn, kc, deep)
+        plan = _configurable(M, L, bn, kc, deep, kernel)
         if plan is None:
             continue
         ws = spear.alloc_workspace(plan.workspace_bytes)
         y = host_f64(d.run(M, plan, ws))
-        check_close(y[rows], ref, True, f"decode-mlp M={M} kc={kc} deep={deep}")
+        check_close(y[rows], ref, True, f"decode-mlp {kernel} M={M} kc={kc} deep={deep}")
         assert np.isfinite(y).all()
         ok_status(ws)
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("li", [0, 1, 2, 3])
 @pytest.mark.parametrize("layer", [0, 2])           # layer 0 carries a compensator, layer 2 does not
-def test_sweep_linears(layer, li):
+def test_sweep_linears(layer, li, kernel):
     d = dev(4, li=li, layer=layer)
     L = d.L
     for M in (1, 16):
         ref = d.ref(M)
-        plan = stream_plan(M, L.N, L.K, L.rank, 16, 128, False)
+        plan = stream_plan(M, L.N, L.K, L.rank, 16, 128, False, kernel)
         ws = spear.alloc_workspace(plan.workspace_bytes)
-        check_close(host_f64(d.run(M, plan, ws)), ref, True, f"sweep L{layer}.{li} M={M}")
+        check_close(host_f64(d.run(M, plan, ws)), ref, True, f"sweep {kernel} L{layer}.{li} M={M}")
         ok_status(ws)
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("M", [1, 2, 3, 7, 9, 15, 16, 17, 31, 33, 47, 63, 64])
-@pytest.mark.parametrize("r", [0, 16, 48, 256])
-def test_ragged_shapes(M, r):
+@pytest.mark.parametrize("r", [0, 16, 48, 128, 256])
+def test_ragged_shapes(M, r, kernel):
     # N = 384: three tiles; K = 640 = 5 stages of 128 codes, so tiles straddle CTAs unevenly.
     L = make_layer("stream-ragged", 91 + r, 64, 384, 640, r, outlier_frac=0.02, outlier_scale=10.0, b_g=0.5)
     d = Dev(L)
     ref = d.ref(M)
-    bn = 16 if M <= 16 else (32 if M <= 32 else 64)
+    bn = (8 if kernel == "rk" and M <= 8 else 16) if M <= 16 else (32 if M <= 32 else 64)
     for deep in (False, True):
-        plan = _configurable(M, L, bn, 128, deep)
+        plan = _configurable(M, L, bn, 128, deep, kernel)
         if plan is None:
             continue
         ws = spear.alloc_workspace(plan.workspace_bytes)
-        check_close(host_f64(d.run(M, plan, ws)), ref, True, f"ragged M={M} r={r} deep={deep}")
+        check_close(host_f64(d.run(M, plan, ws)), ref, True, f"ragged {kernel} M={M} r={r} deep={deep}")
         ok_status(ws)
 
 
-def test_gate_off_is_bitwise_plain_and_deterministic():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_gate_off_is_bitwise_plain_and_deterministic(kernel):
     d = dev(1)
     L = d.L
     off = spear.EC(d.ec.A, d.ec.B, d.ec.w_g, float("-inf"))
-    for M, bn, kc in ((1, 16, 128), (16, 16, 256), (16, 32, 256)):
-        plan = stream_plan(M, L.N, L.K, L.rank, bn, kc, False)
-        plain = stream_plan(M, L.N, L.K, 0, bn, kc, False)
+    for M, bn, kc in ((1, 16, 128), (16, 16, 256), (16, 32, 128)):
+        plan = stream_plan(M, L.N, L.K, L.rank, bn, kc, False, kernel)
+        plain = stream_plan(M, L.N, L.K, 0, bn, kc, False, kernel)
         ws = spear.alloc_workspace(plan.workspace_bytes)
         y_plain = d.run(M, plain, ws, ec=None, y_dtype=torch.float32)
         y_off = d.run(M, plan, ws, ec=off, y_dtype=torch.float32)
@@ -190,7 +203,8 @@ def test_gate_off_is_bitwise_plain_and_deterministic():
         ok_status(ws)
 
 
-def test_chained_calls_in_one_stream():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_chained_calls_in_one_stream(kernel):
     # Back-to-back calls on one stream overlap through programmatic dependent launch: each call's
     # weight stream starts while the previous one finishes.  Alternate two layers and two batch
     # sizes on one workspace, then check every output.
@@ -202,7 +216,8 @@ def test_chained_calls_in_one_stream():
             # decode-qo: 64-code stages with the deep ring at M = 1 (a small CTA that must still hold
             # its SM alone), 128-code stages with two CTAs per SM at M = 16
             deep = d is d1 and M == 1
-            plans[(d.L.name, M)] = stream_plan(M, d.L.N, d.L.K, d.L.rank, 16, 128 if (d is d0 or deep) else 256, deep)
+            plans[(d.L.name, M)] = stream_plan(M, d.L.N, d.L.K, d.L.rank, 16, 128 if (d is d0 or deep) else 256, deep,
+                                               kernel)
     ws = spear.alloc_workspace(max(p.workspace_bytes for p in plans.values()))
     seq = [(d1, 16), (d1, 16), (d0, 1), (d1, 1), (d0, 16), (d1, 16)] * 3
     outs = []
@@ -219,10 +234,11 @@ def test_chained_calls_in_one_stream():
     ok_status(ws)
 
 
-def test_graph_replay():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_graph_replay(kernel):
     d = dev(1)
     L = d.L
-    plan = stream_plan(16, L.N, L.K, L.rank, 16, 128, False)
+    plan = stream_plan(16, L.N, L.K, L.rank, 16, 128, False, kernel)
     ws = spear.alloc_workspace(plan.workspace_bytes)
     x = d.x(16)
     y = torch.empty((16, L.N), dtype=torch.bfloat16, device="cuda")
@@ -256,6 +272,12 @@ def test_rejects_bad_stream_plans():
         spear.spear_plan_update(bad, 4, L.N, L.K, L.rank)
     with pytest.raises(spear.SpearError):                # more tokens than the tile
         spear.spear_plan_update(spear.spear_plan.from_buffer_copy(plan), 17, L.N, L.K, L.rank)
+    # The register path: 64 tokens only with the deep ring, ranks up to 128.
+    with pytest.raises(spear.SpearError):
+        stream_plan(64, L.N, L.K, L.rank, 64, 128, False, "rk")
+    stream_plan(64, L.N, L.K, L.rank, 64, 128, True, "rk")
+    with pytest.raises(spear.SpearError):
+        stream_plan(4, L.N, L.K, 256, 8, 128, False, "rk")
     H = 4
     mlp = spear.EC(d.ec.A, d.ec.B, d.ec.w_g, 0.0,
                    gate_w1=torch.zeros((H, L.rank), device="cuda"), gate_b1=torch.zeros(H, device="cuda"),

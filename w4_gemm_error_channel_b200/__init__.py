@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_PKG, "libspear.so")
 
 SPEAR_OK = 0
 SPEAR_BF16, SPEAR_FP32 = 0, 1
-SPEAR_KERNEL_AUTO, SPEAR_KERNEL_SPLITK, SPEAR_KERNEL_TC05, SPEAR_KERNEL_STREAM = 0, 1, 2, 3
+SPEAR_KERNEL_AUTO, SPEAR_KERNEL_SPLITK, SPEAR_KERNEL_TC05, SPEAR_KERNEL_STREAM, SPEAR_KERNEL_STREAM_RK = 0, 1, 2, 3, 4
 SPEAR_PLAN_SEPARATE_EC, SPEAR_PLAN_DEEP_RING = 1, 2
 STATUS_NAMES = {0: "SPEAR_OK", 1: "SPEAR_ERR_INVALID_ARG", 2: "SPEAR_ERR_UNSUPPORTED_SHAPE",
                 3: "SPEAR_ERR_MISALIGNED", 4: "SPEAR_ERR_WORKSPACE_TOO_SMALL", 5: "SPEAR_ERR_CUDA",

@@ -79,7 +79,7 @@ size_t tc05_u_bytes(int64_t M, int32_t rank) { return ((size_t)M * rank * 2 + 25
 // distributed shared memory.  The prefill kernel with a compensator also keeps u (bf16 [M][r]).
 size_t workspace_bytes_for(const spear_plan& p, int64_t M, int64_t N_for_ws, int64_t K, int32_t rank, int sms) {
     size_t b = ZEROED_BYTES;
-    if (p.kernel_id == SPEAR_KERNEL_STREAM) {
+    if (p.kernel_id == SPEAR_KERNEL_STREAM || p.kernel_id == SPEAR_KERNEL_STREAM_RK) {
         // fp32 partial sums of the tiles that straddle two CTAs: [grid][tile_m][128].
         const int grid = p.split_k > 0 && K % p.split_k == 0 ? stream_grid(N_for_ws, K, p.split_k, sms) : 0;
         return b + (size_t)grid * p.tile_m * 128 * 4;
@@ -122,11 +122,11 @@ bool lookup_measured(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spe
         if (!best || std::llabs(e.M - M) < std::llabs(best->M - M)) best = &e;
     }
     if (!best) return false;
-    if (best->kernel_id == SPEAR_KERNEL_STREAM) {
+    if (best->kernel_id == SPEAR_KERNEL_STREAM || best->kernel_id == SPEAR_KERNEL_STREAM_RK) {
         // The measured stage width and ring mode; the token tile must hold M.
-        const int bn = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+        const int bn = (best->kernel_id == SPEAR_KERNEL_STREAM_RK && M <= 8) ? 8 : M <= 16 ? 16 : (M <= 32 ? 32 : 64);
         if (M > 64 || K % best->split_k != 0) return false;
-        p->kernel_id = SPEAR_KERNEL_STREAM;
+        p->kernel_id = best->kernel_id;
         p->tile_n = 128;
         p->split_k = best->split_k;
         p->tile_m = best->tile_m > bn ? best->tile_m : bn;
@@ -233,6 +233,20 @@ spear_status check_grouped_shape(int64_t M, int64_t N, int64_t K, int64_t group,
 }
 
 spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K, int32_t rank) {
+    if (p.kernel_id == SPEAR_KERNEL_STREAM_RK) {
+        if (p.flags & ~SPEAR_PLAN_DEEP_RING) return SPEAR_ERR_INVALID_ARG;
+        if (p.tile_n != 128 || !(p.tile_m == 8 || p.tile_m == 16 || p.tile_m == 32 || p.tile_m == 64) || M > p.tile_m)
+            return SPEAR_ERR_INVALID_ARG;
+        if (!(p.split_k == 128 || p.split_k == 256) || K % p.split_k != 0) return SPEAR_ERR_INVALID_ARG;
+        StreamArgs a = {};
+        a.M = M > 0 ? M : 1;
+        a.N = N;
+        a.K = K;
+        a.rank = rank;
+        a.grid = stream_grid(N, K, p.split_k, device_sms(-1));
+        if (!stream_rk_configure(a, p.tile_m, p.split_k, (p.flags & SPEAR_PLAN_DEEP_RING) != 0)) return SPEAR_ERR_INVALID_ARG;
+        return SPEAR_OK;
+    }
     if (p.kernel_id == SPEAR_KERNEL_STREAM) {
         if (p.flags & ~SPEAR_PLAN_DEEP_RING) return SPEAR_ERR_INVALID_ARG;
         if (p.tile_n != 128 || !(p.tile_m == 16 || p.tile_m == 32 || p.tile_m == 64) || M > p.tile_m)
@@ -385,7 +399,8 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
     spear_plan p;
     if (plan) {
         p = *plan;
-        if (mlp_gate && p.kernel_id == SPEAR_KERNEL_STREAM) return SPEAR_ERR_INVALID_ARG;   // scalar gate only
+        if (mlp_gate && (p.kernel_id == SPEAR_KERNEL_STREAM || p.kernel_id == SPEAR_KERNEL_STREAM_RK))
+            return SPEAR_ERR_INVALID_ARG;   // scalar gate only
     } else {
         if (lookup_measured(M, N, K, rank, sms, &p)) st = SPEAR_OK;
         else if (use_tc05(M, rank)) st = plan_tc05(M, N, sms, &p);
@@ -393,7 +408,8 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         if (st != SPEAR_OK) return st;
         // The stream kernel takes the scalar gate only: the bottleneck-MLP gate runs on the
         // split-K decode kernel.
-        if (mlp_gate && p.kernel_id == SPEAR_KERNEL_STREAM) st = plan_decode_rules(M, N, K, rank, sms, &p);
+        if (mlp_gate && (p.kernel_id == SPEAR_KERNEL_STREAM || p.kernel_id == SPEAR_KERNEL_STREAM_RK))
+            st = plan_decode_rules(M, N, K, rank, sms, &p);
         if (st != SPEAR_OK) return st;
     }
     st = validate_plan(p, M, N, K, rank);
@@ -432,7 +448,8 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
             e = launch_tc05(t, p.tile_m, p.tile_n, s);
         return e == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
     }
-    if (p.kernel_id == SPEAR_KERNEL_STREAM) {
+    if (p.kernel_id == SPEAR_KERNEL_STREAM || p.kernel_id == SPEAR_KERNEL_STREAM_RK) {
+        const bool rk = p.kernel_id == SPEAR_KERNEL_STREAM_RK;
         StreamArgs a = {};
         a.x = (const uint16_t*)x;
         a.packed = (const uint8_t*)packed;
@@ -449,14 +466,16 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         a.N = N;
         a.K = K;
         a.grid = stream_grid(N, K, p.split_k, sms);
-        if (!stream_configure(a, p.tile_m, p.split_k, (p.flags & SPEAR_PLAN_DEEP_RING) != 0))
+        const bool deep = (p.flags & SPEAR_PLAN_DEEP_RING) != 0;
+        if (!(rk ? stream_rk_configure(a, p.tile_m, p.split_k, deep) : stream_configure(a, p.tile_m, p.split_k, deep)))
             return SPEAR_ERR_INVALID_ARG;
         a.tacc = (long long*)(ws + CTRL_BYTES);
         a.err = ctrl;
         a.flags = ctrl + STREAM_FLAGS_WORD;
         a.ec_readers = ctrl + STREAM_FLAGS_WORD + STREAM_GRID_MAX;
         a.partial = (float*)(ws + ZEROED_BYTES);
-        return launch_stream(a, p.tile_m, s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
+        const cudaError_t e = rk ? launch_stream_rk(a, p.tile_m, s) : launch_stream(a, p.tile_m, s);
+        return e == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
     }
     const int nb = nb_for_tile_m(p.tile_m);
     const int g = p.tile_n / 16;

@@ -18,6 +18,9 @@ constexpr int kMaxDevices = 64;
 // 2-D tensor map over a row-major [rows][cols] array of `elem`-byte elements, box {box_cols, box_rows}.
 bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem, uint64_t cols,
                  uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
+// 3-D tensor map: dims[0] innermost, strides of dims 1 and 2 in bytes.
+bool make_map_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, const uint64_t dims[3],
+                 const uint64_t strides_bytes[2], const uint32_t box[3], CUtensorMapSwizzle swz);
 // Raise `func`'s dynamic shared-memory limit to `bytes` once per device (thread-safe); `once` and
 // `status` are per-function arrays of kMaxDevices entries.
 cudaError_t opt_in_smem(const void* func, size_t bytes, std::once_flag* once, cudaError_t* status);
@@ -144,6 +147,7 @@ struct StreamArgs {
     int nst, na;                    // shared-memory stages, TMEM sub-chunk slots
     int jb, nbu;                    // B rows per B unit, B units per finalised tile
     int stage_bytes, off_u, off_a, off_wg, off_g, off_bar, smem_bytes;
+    int off_b, off_red, nfin;       // register path: B-slice buffer, K-half exchange buffer, finalised EC tiles
     uint32_t tmem_cols;
     int ec_kr, ec_slices;           // rows of A per compensator slice, slices (<= grid)
     int finalizers;                 // CTAs that finalise at least one tile
@@ -155,6 +159,10 @@ struct StreamArgs {
     float* partial;         // [grid][BN][128] fp32 partial sums
 };
 int stream_grid(int64_t N, int64_t K, int kc, int sms);
+// The register-path variant (stream_rk.cu): same schedule and workspace, converted weights in
+// registers feeding mma.sync.  bn = 8, 16, 32 or 64 tokens; kc = 128 or 256; rank <= 128.
+bool stream_rk_configure(StreamArgs& a, int bn, int kc, bool deep);
+cudaError_t launch_stream_rk(const StreamArgs& a, int bn, cudaStream_t stream);
 // A fused split-K decode plan for this shape (api.cu).
 spear_status plan_split_k_decode(int64_t M, int64_t N, int64_t K, int32_t rank, spear_plan* out);
 bool stream_configure(StreamArgs& a, int bn, int kc, bool deep);

@@ -1,0 +1,609 @@
+// stream_rk.cu -- the register-path stream-K kernel for decode batches (up to 64 tokens).
+//
+// SPEAR (Post-Quantization Error-Adaptive Recovery), technical summary section 2.2A: decode is
+// bound by the weight stream and the compensator is fused into the low-bit GEMM.  The layer is
+//
+//   y[m,n] = s[n] * sum_k x[m,k] (q[n,k] - z[n])  +  sum_j u[m,j] B[j,n],
+//   u[m,j] = g[m] t[m,j],  t = x A,  g = sigmoid(x w_g + b_g).
+//
+// Same work split as the tcgen05 stream kernel (stream.cu): 128-row weight tiles cut into K chunks
+// of KC codes, the chunks spread evenly over a persistent grid (stream-K), segments processed
+// last-first, partial tiles handed to the finalising CTA through the workspace in CTA order, and
+// the compensator's x A sliced over the CTAs into exact fixed-point accumulators.  What differs is
+// where the int4 -> bf16 conversion goes: into registers, straight into mma.sync m16n8k16.  At
+// decode sizes a tcgen05 MMA over 128 rows x 16 codes costs about the same whatever the token
+// count, so staging converted weights for it caps the stream; the register path has no staging and
+// leaves the issue slots to the conversion.  Per CTA, 10 warps:
+//   warp 0      TMA producer: per K chunk and 128-code window, the packed tile as two boxes, even
+//               weight rows and odd ones, 64 bytes per row.  The odd box starts one row pair early
+//               (65 rows; before the first tile it reads zeros), so that odd row 2p + 1 sits 64
+//               bytes past even row 2p in the 128-byte bank window and a quarter-warp's loads of
+//               rows 2p and 2p + 1 never collide, while every box stays 128-byte aligned as tensor
+//               copies require.  Then the bf16 x tile (64-code boxes, 128-byte swizzle).  The first
+//               stages' weights go before the wait on the previous kernel, x after it.  For each
+//               finalised tile with a compensator, B[:, tile] into a buffer of its own.
+//   warps 1-8   compute: warp w takes 16 * KC/128 weight rows and one 128-code window of each
+//               chunk (KC = 256: four row quarters x two K halves, exchanged once per segment in a
+//               fixed order).  Lane (g, t) holds 32 codes of rows g and g + 8 per row group; codes
+//               become exact bf16 (q - z) pairs (k, k + 4) and x is loaded with the same pairing.
+//               Then the segment's epilogue: partial sum out, or finalisation with the lower CTAs'
+//               partial sums, the compensator term E[n, m] = sum_j B[j, n] u[m, j] on mma.sync (B
+//               from shared memory by ldmatrix.trans, u split into bf16 hi + lo), y = s[n] D + E.
+//   warp 9      the compensator's slice of x A.  In a CTA that finalises a tile, the compute warps
+//               read the accumulators and form u (fp32) together at its first finalisation.
+// Every wait is bounded in time; on timeout a bit of the error word is set and the site recorded.
+#include "kernels.h"
+#include "stream_common.cuh"
+
+namespace spear {
+
+constexpr int RK_THREADS = 320;
+constexpr int RK_COMPUTE_WARPS = 8;
+
+
+// Weight part of a stage with NWIN 128-code windows: even boxes (64 rows x 64 B) at window * 4096,
+// odd boxes (65 rows x 64 B, 128-byte padded) at NWIN * 4096 + window * 4224.
+constexpr int RK_EVEN_BOX = 64 * 64;
+constexpr int RK_ODD_BOX = 65 * 64;
+constexpr int RK_ODD_PITCH = 4224;                 // RK_ODD_BOX rounded up to 128 bytes
+constexpr int rk_w_bytes(int nwin) { return (nwin * RK_EVEN_BOX + (nwin - 1) * RK_ODD_PITCH + RK_ODD_BOX + 1023) / 1024 * 1024; }
+// Offset of the 64 bytes of weight row `row` (0..127) in window `win` of a stage.
+SPEAR_DEVI uint32_t rk_row_off(uint32_t row, uint32_t win, uint32_t nwin) {
+    return (row & 1u) ? nwin * RK_EVEN_BOX + win * RK_ODD_PITCH + ((row >> 1) + 1u) * 64u
+                      : win * RK_EVEN_BOX + (row >> 1) * 64u;
+}
+
+SPEAR_DEVI void named_bar_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }   // warps 1-8
+SPEAR_DEVI uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+
+// All 256 compute threads: wait (bounded) until every accumulator word holds all slices, then
+// u[m][j] = sigmoid(p[m] + b_g) t[m][j] (fp32) for m < rows (zero past M) into ubuf [rows][ustride].
+// Each thread reads its words in batches of RK_UB independent loads.
+constexpr int RK_UB = 8;
+SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc, float* gs, float* ubuf, int ustride,
+                             int rows) {
+    const int tid = (int)threadIdx.x - 32;           // compute threads are 32 .. 287
+    const int r = a.rank, rs = r + 1;
+    const unsigned long long want = (unsigned long long)a.ec_slices;
+    // pass 0: the gate words (column r); pass 1: t.
+    for (int pass = 0; pass < 2; ++pass) {
+        const int total = pass == 0 ? rows : rows * r;
+        for (int base = 0; base < total; base += 256 * RK_UB) {
+            unsigned long long v[RK_UB];
+            int idx[RK_UB];
+#pragma unroll
+            for (int q = 0; q < RK_UB; ++q) {
+                const int e = base + tid + 256 * q;
+                idx[q] = e < total ? e : -1;
+            }
+            const uint64_t t0 = globaltimer_ns();
+            for (uint32_t it = 0;; ++it) {
+                bool done = true;
+#pragma unroll
+                for (int q = 0; q < RK_UB; ++q) {
+                    const int e = idx[q];
+                    const int m = pass == 0 ? e : e / r, j = pass == 0 ? r : e % r;
+                    v[q] = (e >= 0 && m < a.M) ? ld_relaxed_u64(tacc + (int64_t)m * rs + j) : want;
+                }
+#pragma unroll
+                for (int q = 0; q < RK_UB; ++q) done = done && ((v[q] & 0xFFull) == want);
+                if (done) break;
+                if (globaltimer_ns() - t0 > SK_WAIT_NS) {
+                    sk_fail(a.err, SK_ERR_FLAG, SITE_EC_TACC, base);
+                    break;
+                }
+                __nanosleep(64);
+            }
+#pragma unroll
+            for (int q = 0; q < RK_UB; ++q) {
+                const int e = idx[q];
+                if (e < 0) continue;
+                const int m = pass == 0 ? e : e / r, j = pass == 0 ? r : e % r;
+                const float val = m < a.M ? __ll2float_rn((long long)v[q] >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) : 0.0f;
+                if (pass == 0) gs[m] = m < a.M ? 1.0f / (1.0f + expf(-(val + a.b_g))) : 0.0f;
+                else ubuf[m * ustride + j] = val * gs[m];
+            }
+        }
+        named_bar_compute();
+    }
+}
+
+template <int NB, int KC>
+__global__ void __launch_bounds__(RK_THREADS, (NB <= 4 ? 2 : 1))
+w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_we, const __grid_constant__ CUtensorMap tmap_wo,
+                    const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_b,
+                    const StreamArgs a) {
+    constexpr int BN = 8 * NB;                // token tile
+    constexpr int PITCH = KC / 2;             // bytes per weight row per chunk
+    constexpr int NWIN = KC / 128;            // 128-code windows per chunk
+    constexpr int RG = KC / 128;              // 16-row groups per compute warp
+    constexpr int WB = rk_w_bytes(NWIN);      // weight part of a stage; x follows
+    constexpr int XBOX = BN * 128;            // one 64-code x box
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int NST = a.nst;
+    uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + a.off_bar);    // weights landed
+    uint64_t* xfull = wfull + NST;                                        // x landed
+    uint64_t* sempty = xfull + NST;                                       // stage consumed (8 warps)
+    uint64_t* bfull = sempty + NST;                                       // B slice landed
+    uint64_t* bempty = bfull + 1;                                         // B slice consumed (8 warps)
+    uint64_t* ec_bar = bempty + 1;                                        // A and w_g slices landed
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x;
+    const int u0 = sk_u0(a, c), u1 = sk_u0(a, c + 1);
+    const int nseg = u0 < u1 ? (u1 - 1) / a.nch - u0 / a.nch + 1 : 0;
+    const bool has_ec = a.rank > 0;
+    unsigned char* stages = smem;
+    unsigned char* bbuf = smem + a.off_b;                 // B[:, tile]: two [r][64] boxes, 128-byte swizzle
+    float* ubuf = reinterpret_cast<float*>(smem + a.off_u);   // u fp32 [BN][r + 4]
+    const int ustride = a.rank + 4;
+    uint16_t* As = reinterpret_cast<uint16_t*>(smem + a.off_a);
+    uint16_t* wgs = reinterpret_cast<uint16_t*>(smem + a.off_wg);
+    float* red = reinterpret_cast<float*>(smem + a.off_red);  // K-half exchange [4][2][32][4 NB]
+    const bool has_slice = has_ec && c < a.ec_slices;
+    const int64_t ec_k0 = (int64_t)c * a.ec_kr;
+    const int ec_rows = has_slice ? (int)imin64(a.ec_kr, a.K - ec_k0) : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&wfull[s], 1);
+            mbar_init(&xfull[s], 1);
+            mbar_init(&sempty[s], RK_COMPUTE_WARPS);
+        }
+        mbar_init(bfull, 1);
+        mbar_init(bempty, RK_COMPUTE_WARPS);
+        mbar_init(ec_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    // The next kernel in the stream may be scheduled now; its own wait still covers this grid.
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            bool ok = true;
+            int issued_w = 0, issued_x = 0, bnext = 0;
+            auto issue_w = [&](int sq, int tile, int kci) {
+                const int s = sq % NST;
+                unsigned char* st = stages + (size_t)s * a.stage_bytes;
+                mbar_arrive_expect_tx(&wfull[s], (uint32_t)(NWIN * (RK_EVEN_BOX + RK_ODD_BOX)));
+                for (int w = 0; w < NWIN; ++w) {
+                    tma_load_3d(st + w * RK_EVEN_BOX, &tmap_we, kci * PITCH + 64 * w, 0, tile * 64, &wfull[s]);
+                    tma_load_3d(st + NWIN * RK_EVEN_BOX + w * RK_ODD_PITCH, &tmap_wo, kci * PITCH + 64 * w, 1,
+                                tile * 64 - 1, &wfull[s]);
+                }
+                issued_w = sq + 1;
+            };
+            auto issue_x = [&](int sq, int kci) {
+                const int s = sq % NST;
+                unsigned char* xs = stages + (size_t)s * a.stage_bytes + WB;
+                mbar_arrive_expect_tx(&xfull[s], (uint32_t)((KC / 64) * XBOX));
+                for (int b = 0; b < KC / 64; ++b) tma_load_2d(xs + b * XBOX, &tmap_x, kci * KC + 64 * b, 0, &xfull[s]);
+                issued_x = sq + 1;
+            };
+            // B slice of the fe-th finalised tile (processing order).
+            auto fin_tile = [&](int fe) {
+                int k = 0;
+                for (int i = 0; i < nseg; ++i) {
+                    const SkSeg sg = sk_seg(a, u0, u1, i);
+                    if (sg.fin && k++ == fe) return sg.tile;
+                }
+                return 0;
+            };
+            auto issue_b = [&](int fe) {
+                const int tile = fin_tile(fe);
+                mbar_arrive_expect_tx(bfull, (uint32_t)(2 * a.rank * 128));
+                tma_load_2d(bbuf, &tmap_b, tile * 128, 0, bfull);
+                tma_load_2d(bbuf + a.rank * 128, &tmap_b, tile * 128 + 64, 0, bfull);
+            };
+            int nfin = 0;                     // finalised tiles of this CTA (each needs its B slice)
+            if (has_ec)
+                for (int i = 0; i < nseg; ++i) nfin += sk_seg(a, u0, u1, i).fin ? 1 : 0;
+            // Weights of the first stages and the first B slice before the wait; x after it.
+            int seq = 0;
+            for (int i = 0; i < nseg && seq < NST; ++i) {
+                const SkSeg sg = sk_seg(a, u0, u1, i);
+                for (int kci = sg.kb; kci < sg.ke && seq < NST; ++kci, ++seq) issue_w(seq, sg.tile, kci);
+            }
+            if (nfin > 0) issue_b(bnext++);
+            pdl_wait_primary();
+            seq = 0;
+            for (int i = 0; i < nseg && ok; ++i) {
+                const SkSeg sg = sk_seg(a, u0, u1, i);
+                for (int kci = sg.kb; kci < sg.ke && ok; ++kci, ++seq) {
+                    if (seq < NST) {
+                        issue_x(seq, kci);
+                        continue;
+                    }
+                    // Wait for the stage to be consumed; meanwhile load the next B slice as soon as
+                    // the previous one is released (an epilogue may be waiting for it).
+                    const int s = seq % NST;
+                    const uint32_t ph = ((seq / NST) - 1) & 1;
+                    const uint64_t t0 = globaltimer_ns();
+                    for (uint32_t it = 0;; ++it) {
+                        if (mbar_try(&sempty[s], ph)) break;
+                        if (bnext < nfin && mbar_try(bempty, (bnext - 1) & 1)) issue_b(bnext++);
+                        if ((it & 63) == 63 && globaltimer_ns() - t0 > SK_WAIT_NS) {
+                            sk_fail(a.err, SK_ERR_MBAR, SITE_PROD_SEMPTY, seq);
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!ok) break;
+                    issue_w(seq, sg.tile, kci);
+                    issue_x(seq, kci);
+                }
+            }
+            while (ok && bnext < nfin) {
+                if (!mbar_wait_ns(bempty, (bnext - 1) & 1, SK_WAIT_NS)) {
+                    sk_fail(a.err, SK_ERR_MBAR, SITE_PROD_SEMPTY, -1);
+                    break;
+                }
+                issue_b(bnext++);
+            }
+            // Never leave with copies in flight: wait (bounded) for the last load of every stage.
+            for (int s = 0; s < NST; ++s) {
+                if (s < issued_w) {
+                    const int last = s + (issued_w - 1 - s) / NST * NST;
+                    if (!mbar_wait_ns(&wfull[s], (last / NST) & 1, SK_WAIT_NS)) sk_fail(a.err, SK_ERR_MBAR, SITE_EXIT, last);
+                }
+                if (s < issued_x) {
+                    const int last = s + (issued_x - 1 - s) / NST * NST;
+                    if (!mbar_wait_ns(&xfull[s], (last / NST) & 1, SK_WAIT_NS)) sk_fail(a.err, SK_ERR_MBAR, SITE_EXIT, last);
+                }
+            }
+            if (bnext > 0 && !mbar_wait_ns(bfull, (bnext - 1) & 1, SK_WAIT_NS)) sk_fail(a.err, SK_ERR_MBAR, SITE_EXIT, -2);
+        }
+    } else if (warp <= RK_COMPUTE_WARPS) {
+        // ---------------- compute warps ----------------
+        const int cw = warp - 1;
+        const int g = lane >> 2, t = lane & 3;
+        const int win = KC == 256 ? cw >> 2 : 0;              // 128-code window of each chunk
+        const int rgb = KC == 256 ? 2 * (cw & 3) : cw;         // first 16-row group of this warp
+        // Every wait below depends on x, which follows the previous kernel: wait for it first.
+        pdl_wait_primary();
+        bool ok = true;
+        int seq = 0, fe = 0;
+        bool u_seen = false;
+        for (int i = 0; i < nseg; ++i) {
+            const SkSeg sg = sk_seg(a, u0, u1, i);
+            uint32_t zb[RG][2];
+#pragma unroll
+            for (int j = 0; j < RG; ++j)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    zb[j][h] = zero_bias_bf16x2((uint32_t)__half2float(a.zero[(int64_t)sg.tile * 128 + 16 * (rgb + j) + g + 8 * h]));
+            float acc[RG][NB][4];
+#pragma unroll
+            for (int j = 0; j < RG; ++j)
+#pragma unroll
+                for (int b = 0; b < NB; ++b) acc[j][b][0] = acc[j][b][1] = acc[j][b][2] = acc[j][b][3] = 0.0f;
+
+            for (int kci = sg.kb; kci < sg.ke; ++kci, ++seq) {
+                const int s = seq % NST;
+                const uint32_t ph = (seq / NST) & 1;
+                if (ok && !(mbar_wait_ns(&wfull[s], ph, SK_WAIT_NS) && mbar_wait_ns(&xfull[s], ph, SK_WAIT_NS))) {
+                    sk_fail(a.err, SK_ERR_MBAR, SITE_CVT_WFULL, seq);
+                    ok = false;
+                }
+                const unsigned char* st = stages + (size_t)s * a.stage_bytes;
+                const unsigned char* xs = st + WB;
+                // 16 bytes (32 codes: window codes 32t .. 32t + 31) of rows g and g + 8 per row group.
+                uint4 wa[RG], wb[RG];
+#pragma unroll
+                for (int j = 0; j < RG; ++j) {
+                    const uint32_t r0 = (uint32_t)(16 * (rgb + j) + g);
+                    wa[j] = lds128(st + rk_row_off(r0, win, NWIN) + 16 * t);
+                    wb[j] = lds128(st + rk_row_off(r0 + 8, win, NWIN) + 16 * t);
+                }
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    // x codes 128 win + 32 t + 8 w .. + 7 of every token: box 2 win + t / 2, chunk
+                    // 4 (t % 2) + w, 128-byte swizzle on the token row.
+                    uint32_t xb[NB][4];
+#pragma unroll
+                    for (int b = 0; b < NB; ++b) {
+                        const uint32_t m = (uint32_t)(8 * b + g);
+                        const uint32_t chunk = (uint32_t)(4 * (t & 1) + w);
+                        const uint4 v = lds128(xs + (2 * win + (t >> 1)) * XBOX + m * 128 + ((chunk ^ (m & 7)) << 4));
+                        xb[b][0] = prmt(v.x, v.z, 0x5410u);   // (x0, x4)
+                        xb[b][1] = prmt(v.x, v.z, 0x7632u);   // (x1, x5)
+                        xb[b][2] = prmt(v.y, v.w, 0x5410u);   // (x2, x6)
+                        xb[b][3] = prmt(v.y, v.w, 0x7632u);   // (x3, x7)
+                    }
+#pragma unroll
+                    for (int j = 0; j < RG; ++j) {
+                        const uint32_t qa = w == 0 ? wa[j].x : w == 1 ? wa[j].y : w == 2 ? wa[j].z : wa[j].w;
+                        const uint32_t qb = w == 0 ? wb[j].x : w == 1 ? wb[j].y : w == 2 ? wb[j].z : wb[j].w;
+                        uint32_t ra[4], rb[4];
+                        cvt_w4_pairs_i_i4(qa, zb[j][0], ra);
+                        cvt_w4_pairs_i_i4(qb, zb[j][1], rb);
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint32_t af[4] = {ra[2 * hh], rb[2 * hh], ra[2 * hh + 1], rb[2 * hh + 1]};
+#pragma unroll
+                            for (int b = 0; b < NB; ++b) mma_bf16_16816(acc[j][b], af, xb[b][2 * hh], xb[b][2 * hh + 1]);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sempty[s]);
+            }
+
+            // ---- this warp's final sums for one 16-row group (KC = 256: K halves exchanged) ----
+            float fin[NB][4];
+            int rgf = rgb;
+            if constexpr (KC == 256) {
+                const int qd = cw & 3, h = cw >> 2;
+                float* give = red + ((qd * 2 + (1 - h)) * 32 + lane) * (4 * NB);   // the row group handed over
+                if (h == 0) {
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+                        *reinterpret_cast<float4*>(give + 4 * b) = make_float4(acc[1][b][0], acc[1][b][1], acc[1][b][2], acc[1][b][3]);
+                } else {
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+                        *reinterpret_cast<float4*>(give + 4 * b) = make_float4(acc[0][b][0], acc[0][b][1], acc[0][b][2], acc[0][b][3]);
+                }
+                named_bar_compute();
+                const float* take = red + ((qd * 2 + h) * 32 + lane) * (4 * NB);
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    const float4 o = *reinterpret_cast<const float4*>(take + 4 * b);
+                    // Fixed order: window 0's sum, then window 1's.
+                    if (h == 0) {
+                        fin[b][0] = acc[0][b][0] + o.x; fin[b][1] = acc[0][b][1] + o.y;
+                        fin[b][2] = acc[0][b][2] + o.z; fin[b][3] = acc[0][b][3] + o.w;
+                    } else {
+                        fin[b][0] = o.x + acc[1][b][0]; fin[b][1] = o.y + acc[1][b][1];
+                        fin[b][2] = o.z + acc[1][b][2]; fin[b][3] = o.w + acc[1][b][3];
+                    }
+                }
+                rgf = rgb + h;
+                named_bar_compute();              // the exchange buffer is free again
+            } else {
+#pragma unroll
+                for (int b = 0; b < NB; ++b)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) fin[b][q] = acc[0][b][q];
+            }
+
+            // ---- epilogue: rows 16 rgf + g (+ 8) of the tile; tokens 8 b + 2 t (+ 1) ----
+            const int row0 = 16 * rgf + g;
+            float* own = a.partial + (size_t)c * BN * 128;
+            if (!sg.fin) {
+                // Partial sum of a tile that a higher CTA finalises: [BN][128] fp32, then the flag.
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    const int m = 8 * b + 2 * t;
+                    __stcg(own + m * 128 + row0, fin[b][0]);
+                    __stcg(own + (m + 1) * 128 + row0, fin[b][1]);
+                    __stcg(own + m * 128 + row0 + 8, fin[b][2]);
+                    __stcg(own + (m + 1) * 128 + row0 + 8, fin[b][3]);
+                }
+                __threadfence();
+                named_bar_compute();
+                if (cw == 0 && lane == 0) st_release_gpu(a.flags + c, 1u);
+                continue;
+            }
+            const int c_lo = sg.kb > 0 ? sk_cta_of(a, sg.tile * a.nch) : c;
+            if (c_lo < c) {
+                // Lower CTAs computed the tile's first chunks: add their partial sums in CTA order,
+                // then this CTA's own.
+                if (cw == 0 && lane == 0) {
+                    for (int cc = c_lo; cc < c; ++cc) {
+                        unsigned v;
+                        if (!poll_until<unsigned>(ld_acquire_gpu, a.flags + cc, [](unsigned w) { return w != 0u; }, v))
+                            sk_fail(a.err, SK_ERR_FLAG, SITE_EPI_FLAG, cc);
+                    }
+                }
+                named_bar_compute();
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    const int m = 8 * b + 2 * t;
+                    float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+                    for (int cc = c_lo; cc < c; ++cc) {
+                        const float* pp = a.partial + (size_t)cc * BN * 128;
+                        const float q0 = __ldcg(pp + m * 128 + row0), q1 = __ldcg(pp + (m + 1) * 128 + row0);
+                        const float q2 = __ldcg(pp + m * 128 + row0 + 8), q3 = __ldcg(pp + (m + 1) * 128 + row0 + 8);
+                        if (cc == c_lo) { p0 = q0; p1 = q1; p2 = q2; p3 = q3; }
+                        else { p0 += q0; p1 += q1; p2 += q2; p3 += q3; }
+                    }
+                    fin[b][0] = p0 + fin[b][0]; fin[b][1] = p1 + fin[b][1];
+                    fin[b][2] = p2 + fin[b][2]; fin[b][3] = p3 + fin[b][3];
+                }
+                named_bar_compute();
+                if (cw == 0 && lane == 0)
+                    for (int cc = c_lo; cc < c; ++cc) a.flags[cc] = 0u;   // re-armed for the next call
+            }
+            float e[NB][4];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) e[b][0] = e[b][1] = e[b][2] = e[b][3] = 0.0f;
+            if (has_ec) {
+                if (!u_seen) {
+                    // u for every token, read by all 256 compute threads in batches of independent
+                    // loads (one dependent round trip per batch, not per word).
+                    rk_compute_u(a, reinterpret_cast<const unsigned long long*>(a.tacc),
+                                 reinterpret_cast<float*>(smem + a.off_g), ubuf, ustride, BN);
+                    if (cw == 0) ec_retire(a, reinterpret_cast<unsigned long long*>(a.tacc));
+                    u_seen = true;
+                }
+                // E[n, m] = sum_j B[j, n] u[m, j]: B^T fragments by ldmatrix.trans from the B buffer
+                // ([j][64] boxes, 128-byte swizzle), u as bf16 hi + lo parts.
+                if (ok && !mbar_wait_ns(bfull, fe & 1, SK_WAIT_NS)) {
+                    sk_fail(a.err, SK_ERR_MBAR, SITE_MMA_BUNIT, fe);
+                    ok = false;
+                }
+                const int mat = lane >> 3, rr = lane & 7;
+                const int nb = 16 * rgf + (mat & 1) * 8;                 // first row of this lane's 8x8 matrix
+                const unsigned char* bbox = bbuf + (nb >> 6) * (a.rank * 128);
+                for (int j0 = 0; j0 < a.rank; j0 += 16) {
+                    const int jr = j0 + (mat >> 1) * 8 + rr;
+                    uint32_t af[4];
+                    ldsm_x4_trans(af, bbox + jr * 128 + (((((nb & 63) >> 3) ^ (jr & 7)) & 7) << 4));
+#pragma unroll
+                    for (int b = 0; b < NB; ++b) {
+                        const float* ur = ubuf + (8 * b + g) * ustride + j0 + 2 * t;
+                        const float2 u01 = *reinterpret_cast<const float2*>(ur);
+                        const float2 u89 = *reinterpret_cast<const float2*>(ur + 8);
+                        const __nv_bfloat162 h0 = __floats2bfloat162_rn(u01.x, u01.y);
+                        const __nv_bfloat162 h1 = __floats2bfloat162_rn(u89.x, u89.y);
+                        const __nv_bfloat162 l0 = __floats2bfloat162_rn(u01.x - __low2float(h0), u01.y - __high2float(h0));
+                        const __nv_bfloat162 l1 = __floats2bfloat162_rn(u89.x - __low2float(h1), u89.y - __high2float(h1));
+                        mma_bf16_16816(e[b], af, *reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+                        mma_bf16_16816(e[b], af, *reinterpret_cast<const uint32_t*>(&l0), *reinterpret_cast<const uint32_t*>(&l1));
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bempty);
+                ++fe;
+            }
+            const int64_t n_lo = (int64_t)sg.tile * 128 + row0;
+            const float s_lo = __half2float(a.scale[n_lo]), s_hi = __half2float(a.scale[n_lo + 8]);
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                const int64_t m = 8 * b + 2 * t;
+                const float y00 = fmaf(s_lo, fin[b][0], e[b][0]), y01 = fmaf(s_lo, fin[b][1], e[b][1]);
+                const float y10 = fmaf(s_hi, fin[b][2], e[b][2]), y11 = fmaf(s_hi, fin[b][3], e[b][3]);
+                if (a.y_fp32) {
+                    float* y = reinterpret_cast<float*>(a.y);
+                    if (m < a.M) { y[m * a.N + n_lo] = y00; y[m * a.N + n_lo + 8] = y10; }
+                    if (m + 1 < a.M) { y[(m + 1) * a.N + n_lo] = y01; y[(m + 1) * a.N + n_lo + 8] = y11; }
+                } else {
+                    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.y);
+                    if (m < a.M) { y[m * a.N + n_lo] = __float2bfloat16_rn(y00); y[m * a.N + n_lo + 8] = __float2bfloat16_rn(y10); }
+                    if (m + 1 < a.M) {
+                        y[(m + 1) * a.N + n_lo] = __float2bfloat16_rn(y01);
+                        y[(m + 1) * a.N + n_lo + 8] = __float2bfloat16_rn(y11);
+                    }
+                }
+            }
+        }
+    } else {
+        // ---------------- compensator (warp 9) ----------------
+        if (has_slice && lane == 0) {
+            const uint32_t abytes = (uint32_t)(ec_rows * a.rank * 2), gbytes = (uint32_t)(ec_rows * 2);
+            mbar_arrive_expect_tx(ec_bar, abytes + gbytes);
+            bulk_load(As, a.A + ec_k0 * a.rank, abytes, ec_bar);
+            bulk_load(wgs, a.wg + ec_k0, gbytes, ec_bar);
+        }
+        pdl_wait_primary();
+        unsigned long long* tacc = reinterpret_cast<unsigned long long*>(a.tacc);
+        if (has_slice) {
+            if (mbar_wait_ns(ec_bar, 0, SK_WAIT_NS))
+                ec_slice(a, As, wgs, ec_k0, ec_rows, tacc);
+            else if (lane == 0)
+                sk_fail(a.err, SK_ERR_MBAR, SITE_EC_BAR, 0);
+        }
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------------------------
+static int rk_align(int v, int a) { return (v + a - 1) / a * a; }
+
+bool stream_rk_configure(StreamArgs& a, int bn, int kc, bool deep) {
+    if (!(bn == 8 || bn == 16 || bn == 32 || bn == 64) || !(kc == 128 || kc == 256)) return false;
+    if (a.K % kc != 0 || a.N % 128 != 0 || a.M < 1 || a.M > bn || a.rank > 128) return false;
+    if (bn == 64 && !deep) return false;             // 64 tokens need the registers of one CTA per SM
+    a.kc = kc;
+    a.nch = (int)(a.K / kc);
+    a.ntiles = (int)(a.N / 128);
+    a.units = a.ntiles * a.nch;
+    if (a.grid < 1 || a.grid > a.units || a.grid > (int)STREAM_GRID_MAX) return false;
+    a.stage_bytes = rk_align(rk_w_bytes(kc / 128) + (kc / 64) * bn * 128, 1024);
+    a.jb = a.nbu = 0;
+    a.ec_kr = a.ec_slices = 0;
+    int b_bytes = 0, u_bytes = 0, a_bytes = 0, wg_bytes = 0, g_bytes = 0;
+    if (a.rank > 0) {
+        const int64_t per = (a.K + a.grid - 1) / a.grid;
+        a.ec_kr = (int)((per + 31) / 32 * 32);
+        a.ec_slices = (int)((a.K + a.ec_kr - 1) / a.ec_kr);
+        if (a.ec_slices > a.grid || a.ec_slices > 255) return false;
+        b_bytes = 2 * a.rank * 128;
+        u_bytes = rk_align(bn * (a.rank + 4) * 4, 128);
+        a_bytes = rk_align(a.ec_kr * a.rank * 2, 128);
+        wg_bytes = rk_align(a.ec_kr * 2, 128);
+        g_bytes = rk_align(bn * 4, 128);
+    }
+    const int red_bytes = kc == 256 ? 4 * 2 * 32 * 4 * (bn / 8) * 4 : 0;
+    const int bar_bytes = 8 * (3 * 16 + 4) + 16;
+    const int fixed = b_bytes + u_bytes + a_bytes + wg_bytes + g_bytes + red_bytes + bar_bytes + 1024;
+    const int budget = deep ? (int)SMEM_OPTIN_MAX : 110 * 1024;
+    int nst = (budget - fixed) / a.stage_bytes;
+    if (nst > 16) nst = 16;
+    if (nst < 2) return false;
+    a.nst = nst;
+    a.na = 0;
+    a.tmem_cols = 0;
+    a.off_b = nst * a.stage_bytes;                    // 1024-aligned (stages are)
+    a.off_u = a.off_b + rk_align(b_bytes, 1024);
+    a.off_a = a.off_u + u_bytes;
+    a.off_wg = a.off_a + a_bytes;
+    a.off_g = a.off_wg + wg_bytes;
+    a.off_red = a.off_g + g_bytes;
+    a.off_bar = a.off_red + red_bytes;
+    a.smem_bytes = a.off_bar + bar_bytes + 1024;
+    if (a.smem_bytes > (int)SMEM_OPTIN_MAX) return false;
+    // The deep ring keeps one CTA per SM: reserve more than half of the SM's shared memory.
+    if (deep && a.smem_bytes < 116 * 1024) a.smem_bytes = 116 * 1024;
+    a.finalizers = 0;
+    for (int cc = 0; cc < a.grid; ++cc) {
+        const int v0 = (int)((int64_t)a.units * cc / a.grid), v1 = (int)((int64_t)a.units * (cc + 1) / a.grid);
+        if (v0 < v1 && (v1 % a.nch == 0 || (v1 - 1) / a.nch > v0 / a.nch)) ++a.finalizers;
+    }
+    a.nfin = 0;        // counted per CTA on the device
+    return true;
+}
+
+template <int NB, int KC>
+static cudaError_t launch_rk_t(const StreamArgs& a, cudaStream_t stream) {
+    CUtensorMap mwe, mwo, mx, mb;
+    // Packed weights [N][K/2] viewed as [N/2 row pairs][2][K/2]: boxes of 64 bytes of one row
+    // parity, 64 pairs (even rows) or 65 pairs (odd rows, starting one pair early).
+    const uint64_t wdims[3] = {(uint64_t)(a.K / 2), 2, (uint64_t)(a.N / 2)};
+    const uint64_t wstr[2] = {(uint64_t)(a.K / 2), (uint64_t)a.K};
+    const uint32_t ebox[3] = {64, 1, 64}, obox[3] = {64, 1, 65};
+    if (!make_map_3d(&mwe, a.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, wdims, wstr, ebox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map_3d(&mwo, a.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, wdims, wstr, obox, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    if (!make_map_2d(&mx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.K, (uint64_t)a.M, 64, 8 * NB,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (a.rank > 0) {
+        if (!make_map_2d(&mb, a.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.N, (uint64_t)a.rank, 64,
+                         (uint32_t)a.rank, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    } else {
+        mb = mx;   // unused
+    }
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t opt_status[kMaxDevices];
+    cudaError_t oe = opt_in_smem((const void*)w4_stream_rk_kernel<NB, KC>, SMEM_OPTIN_MAX, once, opt_status);
+    if (oe != cudaSuccess) return oe;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)a.grid);
+    cfg.blockDim = dim3(RK_THREADS);
+    cfg.dynamicSmemBytes = (size_t)a.smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, w4_stream_rk_kernel<NB, KC>, mwe, mwo, mx, mb, a);
+}
+
+cudaError_t launch_stream_rk(const StreamArgs& a, int bn, cudaStream_t stream) {
+#define SPEAR_RK(NB_)                                                                   \
+    if (bn == 8 * NB_) return a.kc == 256 ? launch_rk_t<NB_, 256>(a, stream) : launch_rk_t<NB_, 128>(a, stream);
+    SPEAR_RK(1) SPEAR_RK(2) SPEAR_RK(4) SPEAR_RK(8)
+#undef SPEAR_RK
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace spear
