@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--once", type=int, default=0, metavar="M",
                     help="run 5 layer calls of the workload with M tokens and exit (for profilers)")
     ap.add_argument("--no-ec", action="store_true", help="with --once: the plain W4 layer")
+    ap.add_argument("--plan", default="", metavar="KERNEL,TILE_N,TILE_M,SPLIT_K,FLAGS",
+                    help="with --once: this plan (checked by spear_plan_update) instead of the planner's")
     ap.add_argument("--model-sweep", action="store_true",
                     help="the 16-layer sweep workload (hidden 2048, MLP 8192, EC r=32 on layers 0, 1, 7, 15): "
                          "all 64 linears of one pass per batch size, with the dispatcher's plans")
@@ -518,6 +520,14 @@ def _sweep_shape(torch, spear, L, batches):
     per_set = layer_bytes(max(batches), N, K, r)
     copies = max(2, int(np.ceil(2 * L2_BYTES / per_set)) + 1)
     sets = make_device_layer(torch, spear, L, copies)
+    tiled = []
+
+    def tiled_sets():
+        # The same weight sets with the codes in tile order (made on first use).
+        if not tiled and L.N % 128 == 0 and L.K % 128 == 0:
+            tiled.extend((spear.spear_tile_w4(p),) + tuple(rest) for p, *rest in sets)
+            torch.cuda.synchronize()
+        return tiled
     dev = torch.device("cuda")
     stream = torch.cuda.Stream()
     rows = []
@@ -542,7 +552,8 @@ def _sweep_shape(torch, spear, L, batches):
             candidates += [(3, 128, kc, fl, bn) for kc in (128, 256) for fl in (0, 2) if K % kc == 0]
             # The register-path stream kernel (kernel 4): 8-token tiles from M <= 8, 64 only deep.
             bn_rk = 8 if M <= 8 else bn
-            candidates += [(4, 128, kc, fl, bn_rk) for kc in (128, 256) for fl in (0, 2)
+            # (codes in the tile order of spear_tile_w4: flag 4)
+            candidates += [(4, 128, kc, fl | 4, bn_rk) for kc in (128, 256) for fl in (0, 2)
                            if K % kc == 0 and (bn_rk < 64 or fl == 2) and (r <= 128)]
         for cand in candidates:
                 kernel_id, tile_n, split, fl = cand[:4]
@@ -558,8 +569,10 @@ def _sweep_shape(torch, spear, L, batches):
                         plan.tile_m = 8 if M <= 8 else (16 if M <= 16 else 32)
                     n_calls = 64
 
+                    src = tiled_sets() if fl & spear.SPEAR_PLAN_W4_TILES else sets
+
                     def call(i):
-                        p, sc, z, A, B, wg = sets[i % copies]
+                        p, sc, z, A, B, wg = src[i % copies]
                         ec = spear.EC(A, B, wg, L.b_g) if use_ec else None
                         spear.spear_w4ec_gemm(x, p, sc, z, ec, y=y, workspace=ws, plan=plan, stream=stream)
                     try:
@@ -597,7 +610,7 @@ def _sweep_shape(torch, spear, L, batches):
                                  "tile_n": tile_n, "tile_m": plan.tile_m,
                                  "split_k": split, "us": best,
                                  "GBps": layer_bytes(M, N, K, r if use_ec else 0) / best / 1e3})
-    del sets
+    del sets, tiled
     torch.cuda.empty_cache()
     return rows
 
@@ -615,9 +628,15 @@ def run_once(args):
     bf = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
     ec = None if args.no_ec else spear.EC(bf(L.A_bits), bf(L.B_bits), bf(L.wg_bits), L.b_g)
     x = bf(L.x(M))
-    plan = spear.spear_gemm_plan(M, L.N, L.K, 0 if args.no_ec else L.rank)
+    rank = 0 if args.no_ec else L.rank
+    plan = spear.spear_gemm_plan(M, L.N, L.K, rank)
+    if args.plan:
+        plan.kernel_id, plan.tile_n, plan.tile_m, plan.split_k, plan.flags = (int(v) for v in args.plan.split(","))
+        plan = spear.spear_plan_update(plan, M, L.N, L.K, rank)
     ws = spear.alloc_workspace(plan.workspace_bytes)
     y = torch.empty((M, L.N), dtype=torch.bfloat16, device="cuda")
+    if plan.flags & spear.SPEAR_PLAN_W4_TILES:
+        packed = spear.spear_tile_w4(packed)
     for _ in range(5):
         spear.spear_w4ec_gemm(x, packed, scale, zero, ec, y=y, workspace=ws, plan=plan)
     torch.cuda.synchronize()

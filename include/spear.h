@@ -73,9 +73,11 @@ typedef enum {
                                    (128 or 256, dividing K).  The scalar gate only. */
     SPEAR_KERNEL_STREAM_RK = 4  /* decode (M <= 64): the same stream-K schedule, workspace and fused
                                    compensator as SPEAR_KERNEL_STREAM, with the int4 codes converted
-                                   into registers and fed to mma.sync (no TMEM staging).  tile_n = 128,
-                                   tile_m = 8, 16, 32 or 64 (>= M; 64 needs SPEAR_PLAN_DEEP_RING),
-                                   split_k = 128 or 256 (dividing K), rank <= 128, scalar gate only. */
+                                   into registers and fed to mma.sync (no TMEM staging).  Reads the
+                                   codes in the tile order of spear_tile_w4 (plan flag
+                                   SPEAR_PLAN_W4_TILES, required).  tile_n = 128, tile_m = 8, 16, 32
+                                   or 64 (>= M; 64 needs SPEAR_PLAN_DEEP_RING), split_k = 128 or 256
+                                   (dividing K), rank <= 128, scalar gate only. */
 } spear_kernel;
 
 /* spear_plan.flags bits. */
@@ -96,7 +98,10 @@ enum {
      * memory, 512 TMEM columns) instead of a ring small enough for two CTAs per SM.  The deep ring
      * keeps more weight bytes in flight (large layers); the small one lets the next call's CTAs
      * start their weight stream on the same SMs while this call finishes (small layers). */
-    SPEAR_PLAN_DEEP_RING = 2
+    SPEAR_PLAN_DEEP_RING = 2,
+    /* `packed` holds the codes in the tile order written by spear_tile_w4, not spear_pack_w4's
+     * row order.  Required by SPEAR_KERNEL_STREAM_RK and rejected by every other kernel. */
+    SPEAR_PLAN_W4_TILES = 4
 };
 
 /* Error compensator of one layer.  Pass NULL for a layer without EC (section
@@ -168,6 +173,23 @@ SPEAR_API spear_status spear_debug_unpack_w4(const void* packed, const void* zer
                                    void* q_out, void* qz_out, void* stream);
 
 /*
+ * spear_tile_w4 -- copy packed codes (spear_pack_w4's row order) into the tile order that
+ * SPEAR_KERNEL_STREAM_RK streams (section 2.2A: decode is bound by the weight stream, so the codes
+ * are laid out for it once, at load time).
+ *
+ *   packed  device, uint8 [N, K/2] (layout of spear_pack_w4)
+ *   tiled   device, N * K / 2 bytes, 16-byte aligned, not overlapping `packed`
+ *
+ * Tile order: blocks of 128 rows x 128 codes (8192 bytes); block (T, B) holds rows 128T ..
+ * 128T + 127 and codes 128B .. 128B + 127 and starts at byte (T * K/128 + B) * 8192.  Inside a
+ * block, row r's 64 bytes start at r * 64 as 16 little-endian 32-bit words; word i holds codes
+ * 8i .. 8i + 7 of the block row, code 8i + j in bits 4p .. 4p + 3 with p = (j / 2) + 4 (j % 2)
+ * (codes 2i' and 2i' + 1 sit in nibbles i' and i' + 4).  The scales and zero-points are unchanged.
+ * Requires N % 128 == 0 and K % 128 == 0.  A pure permutation of the 4-bit codes: bit-exact.
+ */
+SPEAR_API spear_status spear_tile_w4(const void* packed, int64_t N, int64_t K, void* tiled, void* stream);
+
+/*
  * spear_gemm_plan -- host-only choice of kernel and tiling for one
  * (M, N, K, rank) problem (section 2.2A: the phase decides between the fused
  * epilogue and a separate EC kernel; section 2.2C: decisions come from
@@ -177,6 +199,15 @@ SPEAR_API spear_status spear_debug_unpack_w4(const void* packed, const void* zer
  */
 SPEAR_API spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int device,
                              spear_plan* out);
+
+/*
+ * spear_gemm_plan_tiled -- as spear_gemm_plan, for codes in spear_tile_w4's tile order: a
+ * SPEAR_KERNEL_STREAM_RK plan (flags include SPEAR_PLAN_W4_TILES).  Requires M <= 64,
+ * N % 128 == 0, K % 128 == 0 and rank <= 128; SPEAR_ERR_UNSUPPORTED_SHAPE otherwise (such
+ * problems need the row-order codes).  The plan serves the scalar gate only.
+ */
+SPEAR_API spear_status spear_gemm_plan_tiled(int64_t M, int64_t N, int64_t K, int32_t rank, int device,
+                                   spear_plan* out);
 
 /*
  * spear_plan_update -- check a plan whose fields the caller has changed (kernel, tiling, flags)
@@ -195,7 +226,8 @@ SPEAR_API spear_status spear_plan_update(spear_plan* plan, int64_t M, int64_t N,
  *
  *   plan       host, from spear_gemm_plan, or NULL (planned on the fly)
  *   x          device, bf16 [M, K]
- *   packed, scale, zero   from spear_pack_w4 for W [N, K]
+ *   packed, scale, zero   from spear_pack_w4 for W [N, K]; with SPEAR_PLAN_W4_TILES in the
+ *              plan's flags, packed from spear_tile_w4 (a NULL plan means row order)
  *   ec         host struct with device pointers, or NULL for a plain W4 layer
  *   y          device, [M, N], bf16 (y_dtype = SPEAR_BF16, one rounding at the
  *              end) or fp32 (SPEAR_FP32, unrounded: a test/debug output)

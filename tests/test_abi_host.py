@@ -265,3 +265,31 @@ def test_plan_update_decode_plans():
     assert spear._lib.spear_plan_update(ctypes.byref(t), 2048, N, K, r) == INVALID
     t.tile_n, t.tile_m = 128, 256
     assert spear._lib.spear_plan_update(ctypes.byref(t), 2048, N, K, 144) == INVALID
+
+
+def test_tiled_plan_and_tile_order_argument_checks():
+    # Plans for codes in the tile order: the register-path stream kernel, flagged as such.
+    p = spear.spear_plan()
+    for M in (1, 8, 16, 32, 64):
+        assert spear._lib.spear_gemm_plan_tiled(M, 4096, 4096, 64, -1, ctypes.byref(p)) == OK
+        assert p.kernel_id == spear.SPEAR_KERNEL_STREAM_RK and p.flags & spear.SPEAR_PLAN_W4_TILES
+        assert p.tile_m >= M and 4096 % p.split_k == 0
+    for M, N, K, r in ((65, 4096, 4096, 64), (1, 4160, 4096, 64), (1, 4096, 4032, 64), (1, 4096, 4096, 144)):
+        assert spear._lib.spear_gemm_plan_tiled(M, N, K, r, -1, ctypes.byref(p)) == SHAPE, (M, N, K, r)
+    # Without the flag the register path is refused; the row-order kernels refuse the flag.
+    assert spear._lib.spear_gemm_plan_tiled(4, 4096, 4096, 64, -1, ctypes.byref(p)) == OK
+    q = spear.spear_plan.from_buffer_copy(p)
+    q.flags &= ~spear.SPEAR_PLAN_W4_TILES
+    assert spear._lib.spear_plan_update(ctypes.byref(q), 4, 4096, 4096, 64) == INVALID
+    st, rows = _plan(4, 4096, 4096, 64)
+    assert st == OK and not rows.flags & spear.SPEAR_PLAN_W4_TILES
+    assert rows.kernel_id != spear.SPEAR_KERNEL_STREAM_RK           # row-order planning never picks it
+    rows.flags |= spear.SPEAR_PLAN_W4_TILES
+    assert spear._lib.spear_plan_update(ctypes.byref(rows), 4, 4096, 4096, 64) == INVALID
+    # spear_tile_w4 checks its arguments before touching the device.
+    tile = spear._lib.spear_tile_w4
+    assert tile(None, 128, 128, ctypes.c_void_p(4096), None) == INVALID
+    assert tile(ctypes.c_void_p(4096), 100, 128, ctypes.c_void_p(1 << 20), None) == SHAPE
+    assert tile(ctypes.c_void_p(4096), 128, 192, ctypes.c_void_p(1 << 20), None) == SHAPE
+    assert tile(ctypes.c_void_p(4104), 128, 128, ctypes.c_void_p(1 << 20), None) == MISALIGNED
+    assert tile(ctypes.c_void_p(4096), 128, 128, ctypes.c_void_p(4096 + 16), None) == INVALID   # overlap

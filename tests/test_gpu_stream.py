@@ -1,7 +1,8 @@
-"""The small-batch stream-K kernel (SPEAR_KERNEL_STREAM) against the CPU oracle, through the C ABI.
+"""The small-batch stream-K kernels (SPEAR_KERNEL_STREAM, and SPEAR_KERNEL_STREAM_RK on codes in the
+tile order of spear_tile_w4) against the CPU oracle, through the C ABI.
 
-Every token tile (16, 32, 64), pipeline-stage width (64, 128, 256 codes) and ring mode (two CTAs
-per SM, or one with a deep ring) is run with explicit plans; the tolerance is the one of
+Every token tile (8 to 64), pipeline-stage width (128, 256 codes) and ring mode (two CTAs per SM,
+or one with a deep ring) is run with explicit plans; the tolerance is the one of
 tests/gpu_helpers.py.  The tiles that straddle CTAs meet in a fixed order, so repeated calls are
 bit-identical, and a compensator whose gate is exactly 0 gives the plain layer bit for bit.
 """
@@ -32,7 +33,7 @@ def stream_plan(M, N, K, rank, bn, kc, deep, kernel="tc"):
     p = spear.spear_plan()
     kid = spear.SPEAR_KERNEL_STREAM if kernel == "tc" else spear.SPEAR_KERNEL_STREAM_RK
     p.kernel_id, p.tile_n, p.tile_m, p.split_k = kid, 128, bn, kc
-    p.flags = spear.SPEAR_PLAN_DEEP_RING if deep else 0
+    p.flags = (spear.SPEAR_PLAN_DEEP_RING if deep else 0) | (spear.SPEAR_PLAN_W4_TILES if kernel == "rk" else 0)
     return spear.spear_plan_update(p, M, N, K, rank)
 
 
@@ -40,6 +41,7 @@ class Dev:
     def __init__(self, L):
         self.L = L
         self.packed, self.scale, self.zero = spear.spear_pack_w4(to_dev(L.W))
+        self._tiled = None
         self.ec = None
         if L.rank > 0:
             self.ec = spear.EC(to_dev_bf16(L.A_bits), to_dev_bf16(L.B_bits), to_dev_bf16(L.wg_bits), L.b_g)
@@ -50,9 +52,16 @@ class Dev:
             self.xd[M] = to_dev_bf16(self.L.x(M))
         return self.xd[M]
 
+    @property
+    def tiled(self):
+        if self._tiled is None:
+            self._tiled = spear.spear_tile_w4(self.packed)
+        return self._tiled
+
     def run(self, M, plan, ws, y_dtype=torch.bfloat16, ec="same", y=None, stream=None):
         e = self.ec if ec == "same" else ec
-        return spear.spear_w4ec_gemm(self.x(M), self.packed, self.scale, self.zero, e, y=y, y_dtype=y_dtype,
+        codes = self.tiled if plan is not None and plan.flags & spear.SPEAR_PLAN_W4_TILES else self.packed
+        return spear.spear_w4ec_gemm(self.x(M), codes, self.scale, self.zero, e, y=y, y_dtype=y_dtype,
                                      plan=plan, workspace=ws, stream=stream)
 
     def ref(self, M, rows=None, ec=True):
@@ -249,7 +258,8 @@ def test_graph_replay(kernel):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         for _ in range(4):
-            spear.spear_w4ec_gemm(x, d.packed, d.scale, d.zero, d.ec, y=y, plan=plan, workspace=ws, stream=stream)
+            spear.spear_w4ec_gemm(x, d.tiled if kernel == "rk" else d.packed, d.scale, d.zero, d.ec, y=y, plan=plan,
+                                  workspace=ws, stream=stream)
     y.zero_()
     for _ in range(3):
         g.replay()
@@ -278,6 +288,16 @@ def test_rejects_bad_stream_plans():
     stream_plan(64, L.N, L.K, L.rank, 64, 128, True, "rk")
     with pytest.raises(spear.SpearError):
         stream_plan(4, L.N, L.K, 256, 8, 128, False, "rk")
+    # Tile-order codes: required by the register path, refused by the others.
+    rk = stream_plan(4, L.N, L.K, L.rank, 8, 128, False, "rk")
+    bad = spear.spear_plan.from_buffer_copy(rk)
+    bad.flags &= ~spear.SPEAR_PLAN_W4_TILES
+    with pytest.raises(spear.SpearError):
+        spear.spear_plan_update(bad, 4, L.N, L.K, L.rank)
+    bad = spear.spear_plan.from_buffer_copy(plan)
+    bad.flags |= spear.SPEAR_PLAN_W4_TILES
+    with pytest.raises(spear.SpearError):
+        spear.spear_plan_update(bad, 4, L.N, L.K, L.rank)
     H = 4
     mlp = spear.EC(d.ec.A, d.ec.B, d.ec.w_g, 0.0,
                    gate_w1=torch.zeros((H, L.rank), device="cuda"), gate_b1=torch.zeros(H, device="cuda"),
@@ -285,3 +305,39 @@ def test_rejects_bad_stream_plans():
     ws = spear.alloc_workspace(plan.workspace_bytes)
     with pytest.raises(spear.SpearError):               # the MLP gate is not taken by this kernel
         d.run(4, plan, ws, ec=mlp)
+
+
+def _tile_order_numpy(packed, N, K):
+    """The tile order restated on the host: 128 x 128-code blocks, row r's 64 bytes at r * 64,
+    code 8i + j of a block row in nibble (j // 2) + 4 (j % 2) of word i."""
+    words = np.ascontiguousarray(packed).view(np.uint32).reshape(N, K // 8)
+    codes = np.stack([(words >> (4 * j)) & 0xF for j in range(8)], axis=-1)        # [N, K/8, 8]
+    out_words = np.zeros_like(words)
+    for j in range(8):
+        out_words |= codes[..., j] << np.uint32(4 * (j // 2 + 4 * (j % 2)))
+    blocks = out_words.reshape(N // 128, 128, K // 128, 16).transpose(0, 2, 1, 3)   # [T][B][r][i]
+    return np.ascontiguousarray(blocks).reshape(-1).view(np.uint8)
+
+
+@pytest.mark.parametrize("N,K", [(128, 128), (256, 640), (4096, 4096)])
+def test_tile_w4_is_the_documented_permutation(N, K):
+    rng = np.random.default_rng(N + K)
+    packed = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    pd = torch.from_numpy(packed).cuda()
+    tiled = spear.spear_tile_w4(pd)
+    torch.cuda.synchronize()
+    got = tiled.cpu().numpy().reshape(-1)
+    assert np.array_equal(got, _tile_order_numpy(packed, N, K))
+    with pytest.raises(spear.SpearError):                 # K not a multiple of 128
+        spear.spear_tile_w4(pd[:, : (K // 2) - 32].contiguous())
+
+
+@pytest.mark.parametrize("M", [1, 8, 16, 32, 64])
+def test_tiled_planner_runs(M):
+    d = dev(1)
+    L = d.L
+    plan = spear.spear_gemm_plan_tiled(M, L.N, L.K, L.rank)
+    assert plan.kernel_id == spear.SPEAR_KERNEL_STREAM_RK and plan.flags & spear.SPEAR_PLAN_W4_TILES
+    ws = spear.alloc_workspace(plan.workspace_bytes)
+    check_close(host_f64(d.run(M, plan, ws)), d.ref(M), True, f"tiled planner M={M}")
+    ok_status(ws)

@@ -22,11 +22,12 @@ LIB_PATH = os.path.join(_PKG, "libspear.so")
 SPEAR_OK = 0
 SPEAR_BF16, SPEAR_FP32 = 0, 1
 SPEAR_KERNEL_AUTO, SPEAR_KERNEL_SPLITK, SPEAR_KERNEL_TC05, SPEAR_KERNEL_STREAM, SPEAR_KERNEL_STREAM_RK = 0, 1, 2, 3, 4
-SPEAR_PLAN_SEPARATE_EC, SPEAR_PLAN_DEEP_RING = 1, 2
+SPEAR_PLAN_SEPARATE_EC, SPEAR_PLAN_DEEP_RING, SPEAR_PLAN_W4_TILES = 1, 2, 4
 STATUS_NAMES = {0: "SPEAR_OK", 1: "SPEAR_ERR_INVALID_ARG", 2: "SPEAR_ERR_UNSUPPORTED_SHAPE",
                 3: "SPEAR_ERR_MISALIGNED", 4: "SPEAR_ERR_WORKSPACE_TOO_SMALL", 5: "SPEAR_ERR_CUDA",
                 6: "SPEAR_ERR_TIMEOUT"}
-EXPORTED = ["spear_pack_w4", "spear_debug_unpack_w4", "spear_gemm_plan", "spear_plan_update", "spear_w4ec_gemm",
+EXPORTED = ["spear_pack_w4", "spear_debug_unpack_w4", "spear_tile_w4", "spear_gemm_plan", "spear_gemm_plan_tiled",
+            "spear_plan_update", "spear_w4ec_gemm",
             "spear_w4ec_gemm_noalloc", "spear_noalloc_get_device_status", "spear_get_device_status", "spear_status_string", "spear_version",
             "spear_latency_table", "spear_predict_step_us", "spear_pick_prefill_chunk",
             "spear_pack_w4_grouped", "spear_grouped_workspace_bytes", "spear_w4ec_gemm_grouped"]
@@ -72,7 +73,9 @@ def _load():
     P, I64 = ctypes.c_void_p, ctypes.c_int64
     lib.spear_pack_w4.argtypes = [P, ctypes.c_int, I64, I64, P, P, P, P]
     lib.spear_debug_unpack_w4.argtypes = [P, P, I64, I64, P, P, P]
+    lib.spear_tile_w4.argtypes = [P, I64, I64, P, P]
     lib.spear_gemm_plan.argtypes = [I64, I64, I64, ctypes.c_int32, ctypes.c_int, ctypes.POINTER(spear_plan)]
+    lib.spear_gemm_plan_tiled.argtypes = [I64, I64, I64, ctypes.c_int32, ctypes.c_int, ctypes.POINTER(spear_plan)]
     lib.spear_plan_update.argtypes = [ctypes.POINTER(spear_plan), I64, I64, I64, ctypes.c_int32]
     lib.spear_w4ec_gemm.argtypes = [ctypes.POINTER(spear_plan), P, I64, I64, I64, P, P, P,
                                     ctypes.POINTER(spear_ec), P, ctypes.c_int, P, ctypes.c_size_t, P]
@@ -213,6 +216,23 @@ def spear_gemm_plan(M: int, N: int, K: int, rank: int = 0, device: int = -1) -> 
     plan = spear_plan()
     _check("spear_gemm_plan", _lib.spear_gemm_plan(M, N, K, rank, device, ctypes.byref(plan)))
     return plan
+
+
+def spear_gemm_plan_tiled(M: int, N: int, K: int, rank: int = 0, device: int = -1) -> spear_plan:
+    """Plan for codes in spear_tile_w4's tile order (the register-path stream kernel, M <= 64)."""
+    plan = spear_plan()
+    _check("spear_gemm_plan_tiled", _lib.spear_gemm_plan_tiled(M, N, K, rank, device, ctypes.byref(plan)))
+    return plan
+
+
+def spear_tile_w4(packed: torch.Tensor, tiled=None, stream=None) -> torch.Tensor:
+    """Codes of spear_pack_w4 (u8 [N, K/2]) in the tile order of the register-path stream kernel
+    (u8 [N, K/2] storage holding the reordered bytes)."""
+    _dev(packed, "packed")
+    N, half = packed.shape
+    tiled = torch.empty_like(packed) if tiled is None else tiled
+    _check("spear_tile_w4", _lib.spear_tile_w4(_p(packed), N, 2 * half, _p(tiled), _stream(stream)))
+    return tiled
 
 
 def spear_plan_update(plan: spear_plan, M: int, N: int, K: int, rank: int = 0) -> spear_plan:

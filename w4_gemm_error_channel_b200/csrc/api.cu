@@ -81,7 +81,7 @@ size_t workspace_bytes_for(const spear_plan& p, int64_t M, int64_t N_for_ws, int
     size_t b = ZEROED_BYTES;
     if (p.kernel_id == SPEAR_KERNEL_STREAM || p.kernel_id == SPEAR_KERNEL_STREAM_RK) {
         // fp32 partial sums of the tiles that straddle two CTAs: [grid][tile_m][128].
-        const int grid = p.split_k > 0 && K % p.split_k == 0 ? stream_grid(N_for_ws, K, p.split_k, sms) : 0;
+        const int grid = p.split_k > 0 && K % p.split_k == 0 ? stream_grid(N_for_ws, K, p.split_k, sms, (p.flags & SPEAR_PLAN_DEEP_RING) != 0) : 0;
         return b + (size_t)grid * p.tile_m * 128 * 4;
     }
     if (p.kernel_id == SPEAR_KERNEL_TC05 && rank > 0) b += tc05_u_bytes(M, rank);
@@ -110,12 +110,15 @@ const MeasuredPlan kMeasured[] = {
 
 spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K, int32_t rank);
 
-bool lookup_measured(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spear_plan* p) {
+// tiles: only the register-path stream kernel's entries (codes in tile order); otherwise every
+// other kernel's.
+bool lookup_measured(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spear_plan* p, bool tiles = false) {
     const int has_ec = rank > 0 ? 1 : 0;
     const int nb = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
     const MeasuredPlan* best = nullptr;
     for (const MeasuredPlan& e : kMeasured) {
         const int enb = e.M <= 8 ? 1 : (e.M <= 16 ? 2 : 4);
+        if ((e.kernel_id == SPEAR_KERNEL_STREAM_RK) != tiles) continue;
         if (e.N != N || e.K != K || e.has_ec != has_ec || enb != nb) continue;
         if (e.M > 2 * M || 2 * e.M < M) continue;        // measured within a factor of two of M
         // Same token-tile size; prefer the measured batch closest to M.
@@ -130,7 +133,7 @@ bool lookup_measured(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spe
         p->tile_n = 128;
         p->split_k = best->split_k;
         p->tile_m = best->tile_m > bn ? best->tile_m : bn;
-        p->flags = best->flags & SPEAR_PLAN_DEEP_RING;
+        p->flags = (best->flags & SPEAR_PLAN_DEEP_RING) | (tiles ? SPEAR_PLAN_W4_TILES : 0);
         p->reserved = 0;
         if (validate_plan(*p, M, N, K, rank) != SPEAR_OK) return false;
         return true;
@@ -234,7 +237,9 @@ spear_status check_grouped_shape(int64_t M, int64_t N, int64_t K, int64_t group,
 
 spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K, int32_t rank) {
     if (p.kernel_id == SPEAR_KERNEL_STREAM_RK) {
-        if (p.flags & ~SPEAR_PLAN_DEEP_RING) return SPEAR_ERR_INVALID_ARG;
+        if ((p.flags & ~(SPEAR_PLAN_DEEP_RING | SPEAR_PLAN_W4_TILES)) || !(p.flags & SPEAR_PLAN_W4_TILES))
+            return SPEAR_ERR_INVALID_ARG;
+        if (N % 128 != 0 || K % 128 != 0) return SPEAR_ERR_INVALID_ARG;
         if (p.tile_n != 128 || !(p.tile_m == 8 || p.tile_m == 16 || p.tile_m == 32 || p.tile_m == 64) || M > p.tile_m)
             return SPEAR_ERR_INVALID_ARG;
         if (!(p.split_k == 128 || p.split_k == 256) || K % p.split_k != 0) return SPEAR_ERR_INVALID_ARG;
@@ -243,7 +248,7 @@ spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K,
         a.N = N;
         a.K = K;
         a.rank = rank;
-        a.grid = stream_grid(N, K, p.split_k, device_sms(-1));
+        a.grid = stream_grid(N, K, p.split_k, device_sms(-1), (p.flags & SPEAR_PLAN_DEEP_RING) != 0);
         if (!stream_rk_configure(a, p.tile_m, p.split_k, (p.flags & SPEAR_PLAN_DEEP_RING) != 0)) return SPEAR_ERR_INVALID_ARG;
         return SPEAR_OK;
     }
@@ -258,7 +263,7 @@ spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K,
         a.N = N;
         a.K = K;
         a.rank = rank;
-        a.grid = stream_grid(N, K, p.split_k, device_sms(-1));
+        a.grid = stream_grid(N, K, p.split_k, device_sms(-1), (p.flags & SPEAR_PLAN_DEEP_RING) != 0);
         if (!stream_configure(a, p.tile_m, p.split_k, (p.flags & SPEAR_PLAN_DEEP_RING) != 0)) return SPEAR_ERR_INVALID_ARG;
         return SPEAR_OK;
     }
@@ -363,6 +368,44 @@ spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t rank, int 
     return SPEAR_OK;
 }
 
+spear_status spear_gemm_plan_tiled(int64_t M, int64_t N, int64_t K, int32_t rank, int device, spear_plan* out) {
+    if (!out) return SPEAR_ERR_INVALID_ARG;
+    spear_status st = check_shape(M, N, K, rank);
+    if (st != SPEAR_OK) return st;
+    if (M > 64 || N % 128 != 0 || K % 128 != 0 || rank > 128) return SPEAR_ERR_UNSUPPORTED_SHAPE;
+    const int sms = device_sms(device);
+    const int64_t m = M > 0 ? M : 1;
+    spear_plan p = {};
+    if (!lookup_measured(m, N, K, rank, sms, &p, true)) {
+        // Rules: the smallest token tile that holds M, 256-code stages where K allows, the deep
+        // ring for 64 tokens (the only ring with their registers), else the two-per-SM ring.
+        p.kernel_id = SPEAR_KERNEL_STREAM_RK;
+        p.tile_n = 128;
+        p.tile_m = m <= 8 ? 8 : (m <= 16 ? 16 : (m <= 32 ? 32 : 64));
+        p.split_k = (K % 256 == 0 && p.tile_m <= 16) ? 256 : 128;   // 32+ tokens: registers for 128
+        p.flags = SPEAR_PLAN_W4_TILES | (p.tile_m == 64 ? SPEAR_PLAN_DEEP_RING : 0);
+        p.reserved = 0;
+        if (validate_plan(p, m, N, K, rank) != SPEAR_OK) {
+            p.split_k = 128;
+            if (K % 128 != 0 || validate_plan(p, m, N, K, rank) != SPEAR_OK) return SPEAR_ERR_UNSUPPORTED_SHAPE;
+        }
+    }
+    p.workspace_bytes = workspace_bytes_for(p, M, N, K, rank, sms);
+    *out = p;
+    return SPEAR_OK;
+}
+
+spear_status spear_tile_w4(const void* packed, int64_t N, int64_t K, void* tiled, void* stream) {
+    if (!packed || !tiled) return SPEAR_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0) return SPEAR_ERR_INVALID_ARG;
+    if (N % 128 != 0 || K % 128 != 0) return SPEAR_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(packed) || !aligned16(tiled)) return SPEAR_ERR_MISALIGNED;
+    const uintptr_t a0 = (uintptr_t)packed, b0 = (uintptr_t)tiled, bytes = (uintptr_t)(N * K / 2);
+    if (a0 < b0 + bytes && b0 < a0 + bytes) return SPEAR_ERR_INVALID_ARG;   // overlapping buffers
+    cudaError_t e = launch_tile_w4(packed, N, K, tiled, (cudaStream_t)stream);
+    return e == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
+}
+
 spear_status spear_plan_update(spear_plan* plan, int64_t M, int64_t N, int64_t K, int32_t rank) {
     if (!plan) return SPEAR_ERR_INVALID_ARG;
     spear_status st = check_shape(M, N, K, rank);
@@ -465,8 +508,8 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         a.M = M;
         a.N = N;
         a.K = K;
-        a.grid = stream_grid(N, K, p.split_k, sms);
         const bool deep = (p.flags & SPEAR_PLAN_DEEP_RING) != 0;
+        a.grid = stream_grid(N, K, p.split_k, sms, deep);
         if (!(rk ? stream_rk_configure(a, p.tile_m, p.split_k, deep) : stream_configure(a, p.tile_m, p.split_k, deep)))
             return SPEAR_ERR_INVALID_ARG;
         a.tacc = (long long*)(ws + CTRL_BYTES);

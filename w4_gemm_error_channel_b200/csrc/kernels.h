@@ -158,7 +158,7 @@ struct StreamArgs {
     unsigned* ec_readers;   // CTAs that have read the accumulators (zeroed part)
     float* partial;         // [grid][BN][128] fp32 partial sums
 };
-int stream_grid(int64_t N, int64_t K, int kc, int sms);
+int stream_grid(int64_t N, int64_t K, int kc, int sms, bool deep);
 // The register-path variant (stream_rk.cu): same schedule and workspace, converted weights in
 // registers feeding mma.sync.  bn = 8, 16, 32 or 64 tokens; kc = 128 or 256; rank <= 128.
 bool stream_rk_configure(StreamArgs& a, int bn, int kc, bool deep);
@@ -196,6 +196,7 @@ cudaError_t launch_w4g_gemm(const GroupedArgs& a, cudaStream_t stream);
 
 cudaError_t launch_pack_w4(const void* W, bool w_is_bf16, int64_t N, int64_t K, void* packed, void* scale,
                            void* zero, cudaStream_t stream);
+cudaError_t launch_tile_w4(const void* packed, int64_t N, int64_t K, void* tiled, cudaStream_t stream);
 cudaError_t launch_unpack_w4(const void* packed, const void* zero, int64_t N, int64_t K, void* q_out,
                              void* qz_out, cudaStream_t stream);
 

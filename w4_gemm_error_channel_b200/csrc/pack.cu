@@ -151,6 +151,32 @@ __global__ void __launch_bounds__(256) unpack_w4_kernel(const uint8_t* __restric
     }
 }
 
+// Tile order of the register-path stream kernel: one thread per 32-bit word of the output.
+// Output word d = ((T * K/128 + B) * 128 + r) * 16 + i comes from row 128 T + r, word 16 B + i of
+// the row order; code j of the word moves from nibble j to nibble (j / 2) + 4 (j % 2).
+__global__ void __launch_bounds__(256) tile_w4_kernel(const uint32_t* __restrict__ packed, int64_t N, int64_t K,
+                                                      uint32_t* __restrict__ tiled) {
+    const int64_t d = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t words = N * (K / 8);
+    if (d >= words) return;
+    const int64_t nblk = K / 128;
+    const int64_t i = d & 15, r = (d >> 4) & 127, tb = d >> 11;
+    const int64_t T = tb / nblk, B = tb % nblk;
+    const uint32_t w = packed[(T * 128 + r) * (K / 8) + B * 16 + i];
+    uint32_t o = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o |= ((w >> (4 * j)) & 0xFu) << (4 * ((j >> 1) + 4 * (j & 1)));
+    tiled[d] = o;
+}
+
+cudaError_t launch_tile_w4(const void* packed, int64_t N, int64_t K, void* tiled, cudaStream_t stream) {
+    const int64_t words = N * (K / 8);
+    const dim3 grid((unsigned)((words + 255) / 256));
+    cudaGetLastError();   // report this launch only, not an earlier call's error
+    tile_w4_kernel<<<grid, 256, 0, stream>>>((const uint32_t*)packed, N, K, (uint32_t*)tiled);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_pack_w4(const void* W, bool w_is_bf16, int64_t N, int64_t K, void* packed, void* scale,
                            void* zero, cudaStream_t stream) {
     const int rows_per_block = 8;

@@ -489,9 +489,12 @@ w4_stream_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
 // ---------------------------------------------------------------------------------------------
 static int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
-int stream_grid(int64_t N, int64_t K, int kc, int sms) {
+int stream_grid(int64_t N, int64_t K, int kc, int sms, bool deep) {
+    // Two CTAs per SM with the shallow ring (each takes at most half of the SM's shared memory and
+    // TMEM), one with the deep ring.
     const int64_t units = (N / SK_ROWS) * (K / kc);
-    return (int)(units < sms ? units : sms);
+    const int64_t cap = (int64_t)sms * (deep ? 1 : 2);
+    return (int)(units < cap ? units : cap);
 }
 
 // Shared memory, TMEM and EC slicing for one launch; false if the configuration does not fit.
@@ -524,8 +527,8 @@ bool stream_configure(StreamArgs& a, int bn, int kc, bool deep) {
     a.ec_slices = 0;
     int a_bytes = 0, wg_bytes = 0, u_bytes = 0, g_bytes = 0;
     if (a.rank > 0) {
-        const int64_t per = (a.K + a.grid - 1) / a.grid;
-        a.ec_kr = (int)((per + 31) / 32 * 32);
+        a.ec_kr = sk_ec_rows(a.K, a.rank, a.grid);
+        if (a.ec_kr == 0) return false;
         a.ec_slices = (int)((a.K + a.ec_kr - 1) / a.ec_kr);
         if (a.ec_slices > a.grid || a.ec_slices > 255) return false;
         a_bytes = align_up(a.ec_kr * a.rank * 2, 1024);

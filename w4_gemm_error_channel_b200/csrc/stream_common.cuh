@@ -93,40 +93,78 @@ SPEAR_DEVI SkSeg sk_seg(const StreamArgs& a, int u0, int u1, int i) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// The compensator's accumulators: int64 words [M][r + 1] (t, then the gate pre-activation), each
+// word in a 32-byte sector of its own, so that the slices' additions to different words do not
+// queue behind one another in one sector.  64 tokens x 257 words x 32 bytes fit the workspace's
+// accumulator area.
+// ---------------------------------------------------------------------------------------------
+constexpr int SK_TACC_PAD = 4;
+static_assert(64 * 257 * SK_TACC_PAD * 8 <= TACC_BYTES, "accumulator area");
+constexpr int SK_EC_KR_MAX = 128;             // rows of A per compensator slice, at most
+SPEAR_DEVI unsigned long long* tacc_word(unsigned long long* tacc, const StreamArgs& a, int64_t m, int j) {
+    return tacc + ((int64_t)m * (a.rank + 1) + j) * SK_TACC_PAD;
+}
+SPEAR_DEVI const unsigned long long* tacc_word(const unsigned long long* tacc, const StreamArgs& a, int64_t m, int j) {
+    return tacc + ((int64_t)m * (a.rank + 1) + j) * SK_TACC_PAD;
+}
+// Rows of A per slice: about K / 64 (rounded up to 32), at most SK_EC_KR_MAX and 16 KiB of A, and
+// few enough slices for the 8-bit count and the grid.  0 if no such size exists.
+inline int sk_ec_rows(int64_t K, int rank, int grid) {
+    auto up32 = [](int64_t v) { return (v + 31) / 32 * 32; };
+    int64_t kr = up32((K + 63) / 64);
+    int64_t kr_max = (16384 / (2 * rank)) / 32 * 32;
+    if (kr_max > SK_EC_KR_MAX) kr_max = SK_EC_KR_MAX;
+    if (kr_max < 32) kr_max = 32;
+    if (kr > kr_max) kr = kr_max;
+    if (kr < 32) kr = 32;
+    const int64_t slices_max = grid < 255 ? grid : 255;
+    const int64_t need = up32((K + slices_max - 1) / slices_max);
+    if (kr < need) kr = need;
+    return kr <= SK_EC_KR_MAX ? (int)kr : 0;
+}
+
+// ---------------------------------------------------------------------------------------------
 // The compensator's slice (one warp): t and p over rows [k0, k0 + rows) of A, for every token.
 // Tokens are the M = 16 operand of mma.sync m16n8k16, columns of A the N = 8 operand; the 16
 // columns of a group form two n8 tiles (even and odd columns) so that one 32-bit shared-memory
 // word (two adjacent columns of a row) feeds both.  The gate is one more n8 tile with w_g in
-// column 0.
+// column 0.  The x fragments of a 16-token block are loaded once, all at the same time.
 // ---------------------------------------------------------------------------------------------
 SPEAR_DEVI void ec_slice(const StreamArgs& a, const uint16_t* As, const uint16_t* wgs, int64_t k0, int rows,
                          unsigned long long* tacc) {
+    constexpr int KS = SK_EC_KR_MAX / 16;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int r = a.rank, NG = r / 16;
     const float lim = SK_FIX_TOTAL / (float)a.ec_slices;
     const int ksteps = rows / 16;
     for (int m0 = 0; m0 < a.M; m0 += 16) {
         const int64_t ma = m0 + g, mb = m0 + g + 8;
+        uint32_t xa[KS][4];
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            const int64_t k = k0 + 16 * kk + 2 * t;
+            const bool in = kk < ksteps;
+            xa[kk][0] = in && ma < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + ma * a.K + k)) : 0u;
+            xa[kk][1] = in && mb < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb * a.K + k)) : 0u;
+            xa[kk][2] = in && ma < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + ma * a.K + k + 8)) : 0u;
+            xa[kk][3] = in && mb < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb * a.K + k + 8)) : 0u;
+        }
         for (int P = 0; P <= NG; ++P) {
             const bool gate = P == NG;
             float de[4] = {0.f, 0.f, 0.f, 0.f}, dod[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int kk = 0; kk < ksteps; ++kk) {
-                const int64_t k = k0 + 16 * kk + 2 * t;
-                uint32_t xa[4];
-                xa[0] = ma < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + ma * a.K + k)) : 0u;
-                xa[1] = mb < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb * a.K + k)) : 0u;
-                xa[2] = ma < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + ma * a.K + k + 8)) : 0u;
-                xa[3] = mb < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb * a.K + k + 8)) : 0u;
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                if (kk >= ksteps) break;
                 const int kr = 16 * kk + 2 * t;    // row of the slice
                 if (!gate) {
                     const uint16_t* p = As + (int64_t)kr * r + 16 * P + 2 * g;
                     const uint32_t w0 = lds_u32(p), w1 = lds_u32(p + r), w2 = lds_u32(p + 8 * r), w3 = lds_u32(p + 9 * r);
-                    mma_bf16_16816(de, xa, prmt(w0, w1, 0x5410u), prmt(w2, w3, 0x5410u));
-                    mma_bf16_16816(dod, xa, prmt(w0, w1, 0x7632u), prmt(w2, w3, 0x7632u));
+                    mma_bf16_16816(de, xa[kk], prmt(w0, w1, 0x5410u), prmt(w2, w3, 0x5410u));
+                    mma_bf16_16816(dod, xa[kk], prmt(w0, w1, 0x7632u), prmt(w2, w3, 0x7632u));
                 } else {
                     const uint32_t b0 = g == 0 ? lds_u32(wgs + kr) : 0u;
                     const uint32_t b1 = g == 0 ? lds_u32(wgs + kr + 8) : 0u;
-                    mma_bf16_16816(de, xa, b0, b1);
+                    mma_bf16_16816(de, xa[kk], b0, b1);
                 }
             }
             // Lane (g, t) holds columns 16P + 4t + {0, 1, 2, 3} (even tile: +0, +2; odd: +1, +3)
@@ -138,7 +176,7 @@ SPEAR_DEVI void ec_slice(const StreamArgs& a, const uint16_t* As, const uint16_t
                     v = 0.0f;
                 }
                 const unsigned long long fx = (unsigned long long)__float2ll_rn(v * SK_FIX_ONE);
-                red_add_u64(tacc + m * (r + 1) + col, (fx << SK_FIX_COUNT_BITS) | 1ull);
+                red_add_u64(tacc_word(tacc, a, m, col), (fx << SK_FIX_COUNT_BITS) | 1ull);
             };
             if (!gate) {
                 const int c = 16 * P + 4 * t;
@@ -168,7 +206,7 @@ SPEAR_DEVI void ec_compute_u(const StreamArgs& a, const unsigned long long* tacc
         float gv = 0.0f;
         if (m < a.M) {
             unsigned long long v;
-            if (!poll_until<unsigned long long>(ld_relaxed_u64, tacc + (int64_t)m * (r + 1) + r, complete, v))
+            if (!poll_until<unsigned long long>(ld_relaxed_u64, tacc_word(tacc, a, m, r), complete, v))
                 sk_fail(a.err, SK_ERR_FLAG, SITE_EC_TACC, m * (r + 1) + r);
             const float p = __ll2float_rn((long long)v >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE);
             gv = 1.0f / (1.0f + expf(-(p + a.b_g)));
@@ -181,7 +219,7 @@ SPEAR_DEVI void ec_compute_u(const StreamArgs& a, const unsigned long long* tacc
         float uv = 0.0f;
         if (m < a.M && j < r) {
             unsigned long long v;
-            if (!poll_until<unsigned long long>(ld_relaxed_u64, tacc + (int64_t)m * (r + 1) + j, complete, v))
+            if (!poll_until<unsigned long long>(ld_relaxed_u64, tacc_word(tacc, a, m, j), complete, v))
                 sk_fail(a.err, SK_ERR_FLAG, SITE_EC_TACC, m * (r + 1) + j);
             uv = __ll2float_rn((long long)v >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) * gs[m];
         }
@@ -201,7 +239,7 @@ SPEAR_DEVI void ec_retire(const StreamArgs& a, unsigned long long* tacc) {
     last = __shfl_sync(0xFFFFFFFFu, last, 0);
     if (last) {
         __threadfence();
-        for (int64_t w = lane; w < a.M * (int64_t)(a.rank + 1); w += 32) tacc[w] = 0ull;
+        for (int64_t w = lane; w < a.M * (int64_t)(a.rank + 1); w += 32) tacc[w * SK_TACC_PAD] = 0ull;
         __threadfence();
         __syncwarp();
         if (lane == 0) *a.ec_readers = 0u;

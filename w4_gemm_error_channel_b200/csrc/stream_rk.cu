@@ -9,28 +9,30 @@
 // Same work split as the tcgen05 stream kernel (stream.cu): 128-row weight tiles cut into K chunks
 // of KC codes, the chunks spread evenly over a persistent grid (stream-K), segments processed
 // last-first, partial tiles handed to the finalising CTA through the workspace in CTA order, and
-// the compensator's x A sliced over the CTAs into exact fixed-point accumulators.  What differs is
-// where the int4 -> bf16 conversion goes: into registers, straight into mma.sync m16n8k16.  At
-// decode sizes a tcgen05 MMA over 128 rows x 16 codes costs about the same whatever the token
-// count, so staging converted weights for it caps the stream; the register path has no staging and
-// leaves the issue slots to the conversion.  Per CTA, 10 warps:
-//   warp 0      TMA producer: per K chunk and 128-code window, the packed tile as two boxes, even
-//               weight rows and odd ones, 64 bytes per row.  The odd box starts one row pair early
-//               (65 rows; before the first tile it reads zeros), so that odd row 2p + 1 sits 64
-//               bytes past even row 2p in the 128-byte bank window and a quarter-warp's loads of
-//               rows 2p and 2p + 1 never collide, while every box stays 128-byte aligned as tensor
-//               copies require.  Then the bf16 x tile (64-code boxes, 128-byte swizzle).  The first
-//               stages' weights go before the wait on the previous kernel, x after it.  For each
-//               finalised tile with a compensator, B[:, tile] into a buffer of its own.
-//   warps 1-8   compute: warp w takes 16 * KC/128 weight rows and one 128-code window of each
-//               chunk (KC = 256: four row quarters x two K halves, exchanged once per segment in a
-//               fixed order).  Lane (g, t) holds 32 codes of rows g and g + 8 per row group; codes
-//               become exact bf16 (q - z) pairs (k, k + 4) and x is loaded with the same pairing.
-//               Then the segment's epilogue: partial sum out, or finalisation with the lower CTAs'
-//               partial sums, the compensator term E[n, m] = sum_j B[j, n] u[m, j] on mma.sync (B
-//               from shared memory by ldmatrix.trans, u split into bf16 hi + lo), y = s[n] D + E.
-//   warp 9      the compensator's slice of x A.  In a CTA that finalises a tile, the compute warps
-//               read the accumulators and form u (fp32) together at its first finalisation.
+// the compensator's x A sliced over the CTAs into exact fixed-point accumulators.  The int4 -> bf16
+// conversion goes into registers, straight into mma.sync m16n8k16: at decode sizes a tcgen05 MMA
+// over 128 rows x 16 codes costs about the same whatever the token count, so staging converted
+// weights for it caps the stream, while the register path leaves the issue slots to the
+// conversion.
+//
+// The weights come in the tile order written by spear_tile_w4 (pack.cu): 8 KiB blocks of 128
+// rows x 128 codes, a row's 64 bytes at row * 64, and inside each 32-bit word the nibbles ordered
+// so that the mask 0x000F000F after a shift by 4i picks two consecutive codes (2i, 2i + 1).  A unit
+// (KC codes of a tile) is then one contiguous bulk copy, every lane's weight load is a
+// conflict-free 16-byte read, and x pairs need no permutes.  Per CTA, 10 warps:
+//   warp 0      producer: per unit one bulk copy of the weights, then the bf16 x tile (64-code
+//               boxes, 128-byte swizzle), both on the stage's one barrier.  The first stages'
+//               weights go before the wait on the previous kernel, x after it.  For each finalised
+//               tile with a compensator, B[:, tile] into a buffer of its own.
+//   warps 1-8   compute: warp w takes 16 * KC/128 weight rows and one 128-code block of each unit
+//               (KC = 256: four row quarters x two blocks, exchanged once per segment in a fixed
+//               order).  Lane (g, t) holds 32 codes of rows g and g + 8 per row group.  Then the
+//               segment's epilogue: partial sum out, or finalisation with the lower CTAs' partial
+//               sums, the compensator term E[n, m] = sum_j B[j, n] u[m, j] on mma.sync (B from
+//               shared memory by ldmatrix.trans, u split into bf16 hi + lo), y = s[n] D + E.  In a
+//               CTA that finalises a tile they read the accumulators and form u (fp32) together at
+//               its first finalisation.
+//   warp 9      the compensator's slice of x A.
 // Every wait is bounded in time; on timeout a bit of the error word is set and the site recorded.
 #include "kernels.h"
 #include "stream_common.cuh"
@@ -39,22 +41,18 @@ namespace spear {
 
 constexpr int RK_THREADS = 320;
 constexpr int RK_COMPUTE_WARPS = 8;
-
-
-// Weight part of a stage with NWIN 128-code windows: even boxes (64 rows x 64 B) at window * 4096,
-// odd boxes (65 rows x 64 B, 128-byte padded) at NWIN * 4096 + window * 4224.
-constexpr int RK_EVEN_BOX = 64 * 64;
-constexpr int RK_ODD_BOX = 65 * 64;
-constexpr int RK_ODD_PITCH = 4224;                 // RK_ODD_BOX rounded up to 128 bytes
-constexpr int rk_w_bytes(int nwin) { return (nwin * RK_EVEN_BOX + (nwin - 1) * RK_ODD_PITCH + RK_ODD_BOX + 1023) / 1024 * 1024; }
-// Offset of the 64 bytes of weight row `row` (0..127) in window `win` of a stage.
-SPEAR_DEVI uint32_t rk_row_off(uint32_t row, uint32_t win, uint32_t nwin) {
-    return (row & 1u) ? nwin * RK_EVEN_BOX + win * RK_ODD_PITCH + ((row >> 1) + 1u) * 64u
-                      : win * RK_EVEN_BOX + (row >> 1) * 64u;
-}
+constexpr int RK_BLOCK_BYTES = 128 * 64;       // one 128 x 128-code block of the tile order
 
 SPEAR_DEVI void named_bar_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }   // warps 1-8
-SPEAR_DEVI uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+SPEAR_DEVI uint4 lds128(uint32_t saddr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr));
+    return v;
+}
+// Full-barrier wait with a cheap first test.
+SPEAR_DEVI bool rk_wait(uint64_t* bar, uint32_t parity) {
+    return mbar_try(bar, parity) || mbar_wait_ns(bar, parity, SK_WAIT_NS);
+}
 
 // All 256 compute threads: wait (bounded) until every accumulator word holds all slices, then
 // u[m][j] = sigmoid(p[m] + b_g) t[m][j] (fp32) for m < rows (zero past M) into ubuf [rows][ustride].
@@ -63,7 +61,7 @@ constexpr int RK_UB = 8;
 SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc, float* gs, float* ubuf, int ustride,
                              int rows) {
     const int tid = (int)threadIdx.x - 32;           // compute threads are 32 .. 287
-    const int r = a.rank, rs = r + 1;
+    const int r = a.rank;
     const unsigned long long want = (unsigned long long)a.ec_slices;
     // pass 0: the gate words (column r); pass 1: t.
     for (int pass = 0; pass < 2; ++pass) {
@@ -77,13 +75,13 @@ SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc
                 idx[q] = e < total ? e : -1;
             }
             const uint64_t t0 = globaltimer_ns();
-            for (uint32_t it = 0;; ++it) {
+            for (;;) {
                 bool done = true;
 #pragma unroll
                 for (int q = 0; q < RK_UB; ++q) {
                     const int e = idx[q];
                     const int m = pass == 0 ? e : e / r, j = pass == 0 ? r : e % r;
-                    v[q] = (e >= 0 && m < a.M) ? ld_relaxed_u64(tacc + (int64_t)m * rs + j) : want;
+                    v[q] = (e >= 0 && m < a.M) ? ld_relaxed_u64(tacc_word(tacc, a, m, j)) : want;
                 }
 #pragma unroll
                 for (int q = 0; q < RK_UB; ++q) done = done && ((v[q] & 0xFFull) == want);
@@ -110,22 +108,20 @@ SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc
 
 template <int NB, int KC>
 __global__ void __launch_bounds__(RK_THREADS, (NB <= 4 ? 2 : 1))
-w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_we, const __grid_constant__ CUtensorMap tmap_wo,
-                    const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_b,
+w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_b,
                     const StreamArgs a) {
     constexpr int BN = 8 * NB;                // token tile
-    constexpr int PITCH = KC / 2;             // bytes per weight row per chunk
-    constexpr int NWIN = KC / 128;            // 128-code windows per chunk
+    constexpr int NBLK = KC / 128;            // 128-code blocks per unit
     constexpr int RG = KC / 128;              // 16-row groups per compute warp
-    constexpr int WB = rk_w_bytes(NWIN);      // weight part of a stage; x follows
+    constexpr int WBYTES = NBLK * RK_BLOCK_BYTES;
     constexpr int XBOX = BN * 128;            // one 64-code x box
+    constexpr int XBYTES = (KC / 64) * XBOX;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int NST = a.nst;
-    uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + a.off_bar);    // weights landed
-    uint64_t* xfull = wfull + NST;                                        // x landed
-    uint64_t* sempty = xfull + NST;                                       // stage consumed (8 warps)
-    uint64_t* bfull = sempty + NST;                                       // B slice landed
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + a.off_bar);      // weights and x landed
+    uint64_t* empty = full + NST;                                         // stage consumed (8 warps)
+    uint64_t* bfull = empty + NST;                                        // B slice landed
     uint64_t* bempty = bfull + 1;                                         // B slice consumed (8 warps)
     uint64_t* ec_bar = bempty + 1;                                        // A and w_g slices landed
 
@@ -140,16 +136,17 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_we, const __grid_co
     const int ustride = a.rank + 4;
     uint16_t* As = reinterpret_cast<uint16_t*>(smem + a.off_a);
     uint16_t* wgs = reinterpret_cast<uint16_t*>(smem + a.off_wg);
-    float* red = reinterpret_cast<float*>(smem + a.off_red);  // K-half exchange [4][2][32][4 NB]
+    float* red = reinterpret_cast<float*>(smem + a.off_red);  // block exchange [4][2][32][4 NB]
     const bool has_slice = has_ec && c < a.ec_slices;
     const int64_t ec_k0 = (int64_t)c * a.ec_kr;
     const int ec_rows = has_slice ? (int)imin64(a.ec_kr, a.K - ec_k0) : 0;
 
     if (threadIdx.x == 0) {
+        prefetch_tmap(&tmap_x);
+        if (has_ec) prefetch_tmap(&tmap_b);
         for (int s = 0; s < NST; ++s) {
-            mbar_init(&wfull[s], 1);
-            mbar_init(&xfull[s], 1);
-            mbar_init(&sempty[s], RK_COMPUTE_WARPS);
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], RK_COMPUTE_WARPS);
         }
         mbar_init(bfull, 1);
         mbar_init(bempty, RK_COMPUTE_WARPS);
@@ -161,27 +158,25 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_we, const __grid_co
     pdl_launch_dependents();
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- producer ----------------
         if (lane == 0) {
             bool ok = true;
-            int issued_w = 0, issued_x = 0, bnext = 0;
+            int issued = 0, bnext = 0;
+            const int64_t nblk_row = a.K / 128;                   // blocks per tile
+            auto stage_of = [&](int sq) { return stages + (size_t)(sq % NST) * a.stage_bytes; };
+            // Weights of unit sq (its barrier expects the x bytes as well).
             auto issue_w = [&](int sq, int tile, int kci) {
                 const int s = sq % NST;
-                unsigned char* st = stages + (size_t)s * a.stage_bytes;
-                mbar_arrive_expect_tx(&wfull[s], (uint32_t)(NWIN * (RK_EVEN_BOX + RK_ODD_BOX)));
-                for (int w = 0; w < NWIN; ++w) {
-                    tma_load_3d(st + w * RK_EVEN_BOX, &tmap_we, kci * PITCH + 64 * w, 0, tile * 64, &wfull[s]);
-                    tma_load_3d(st + NWIN * RK_EVEN_BOX + w * RK_ODD_PITCH, &tmap_wo, kci * PITCH + 64 * w, 1,
-                                tile * 64 - 1, &wfull[s]);
-                }
-                issued_w = sq + 1;
+                mbar_arrive_expect_tx(&full[s], (uint32_t)(WBYTES + XBYTES));
+                bulk_load(stage_of(sq), a.packed + ((int64_t)tile * nblk_row + (int64_t)kci * NBLK) * RK_BLOCK_BYTES,
+                          (uint32_t)WBYTES, &full[s]);
+                issued = sq + 1;
             };
             auto issue_x = [&](int sq, int kci) {
                 const int s = sq % NST;
-                unsigned char* xs = stages + (size_t)s * a.stage_bytes + WB;
-                mbar_arrive_expect_tx(&xfull[s], (uint32_t)((KC / 64) * XBOX));
-                for (int b = 0; b < KC / 64; ++b) tma_load_2d(xs + b * XBOX, &tmap_x, kci * KC + 64 * b, 0, &xfull[s]);
-                issued_x = sq + 1;
+                unsigned char* xs = stage_of(sq) + WBYTES;
+#pragma unroll
+                for (int b = 0; b < KC / 64; ++b) tma_load_2d(xs + b * XBOX, &tmap_x, kci * KC + 64 * b, 0, &full[s]);
             };
             // B slice of the fe-th finalised tile (processing order).
             auto fin_tile = [&](int fe) {
@@ -223,7 +218,7 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_we, const __grid_co
                     const uint32_t ph = ((seq / NST) - 1) & 1;
                     const uint64_t t0 = globaltimer_ns();
                     for (uint32_t it = 0;; ++it) {
-                        if (mbar_try(&sempty[s], ph)) break;
+                        if (mbar_try(&empty[s], ph)) break;
                         if (bnext < nfin && mbar_try(bempty, (bnext - 1) & 1)) issue_b(bnext++);
                         if ((it & 63) == 63 && globaltimer_ns() - t0 > SK_WAIT_NS) {
                             sk_fail(a.err, SK_ERR_MBAR, SITE_PROD_SEMPTY, seq);
@@ -243,16 +238,13 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_we, const __grid_co
                 }
                 issue_b(bnext++);
             }
-            // Never leave with copies in flight: wait (bounded) for the last load of every stage.
-            for (int s = 0; s < NST; ++s) {
-                if (s < issued_w) {
-                    const int last = s + (issued_w - 1 - s) / NST * NST;
-                    if (!mbar_wait_ns(&wfull[s], (last / NST) & 1, SK_WAIT_NS)) sk_fail(a.err, SK_ERR_MBAR, SITE_EXIT, last);
-                }
-                if (s < issued_x) {
-                    const int last = s + (issued_x - 1 - s) / NST * NST;
-                    if (!mbar_wait_ns(&xfull[s], (last / NST) & 1, SK_WAIT_NS)) sk_fail(a.err, SK_ERR_MBAR, SITE_EXIT, last);
-                }
+            // Never leave with copies in flight: wait (bounded) for the last copies of every stage.
+            // Weights and x of a unit go out together once the first NST units' x are out, and
+            // a wait that gives up stops the loop before a unit's weights, so every issued stage
+            // also got its x.
+            for (int s = 0; s < NST && s < issued; ++s) {
+                const int last = s + (issued - 1 - s) / NST * NST;
+                if (!mbar_wait_ns(&full[s], (last / NST) & 1, SK_WAIT_NS)) sk_fail(a.err, SK_ERR_MBAR, SITE_EXIT, last);
             }
             if (bnext > 0 && !mbar_wait_ns(bfull, (bnext - 1) & 1, SK_WAIT_NS)) sk_fail(a.err, SK_ERR_MBAR, SITE_EXIT, -2);
         }
@@ -260,12 +252,33 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_we, const __grid_co
         // ---------------- compute warps ----------------
         const int cw = warp - 1;
         const int g = lane >> 2, t = lane & 3;
-        const int win = KC == 256 ? cw >> 2 : 0;              // 128-code window of each chunk
+        const int blk = KC == 256 ? cw >> 2 : 0;              // 128-code block of each unit
         const int rgb = KC == 256 ? 2 * (cw & 3) : cw;         // first 16-row group of this warp
+        // Lane-constant shared-memory offsets in a stage: weights of row 16 rgb + g (row group j:
+        // + 1024 j; rows + 8: + 512), and x chunk (box 2 blk + t/2, chunk 4 (t & 1) + w) of token
+        // g (token 8 b + g: + 1024 b), 128-byte swizzle on the token row.
+        const uint32_t wl = (uint32_t)(blk * RK_BLOCK_BYTES + (16 * rgb + g) * 64 + 16 * t);
+        uint32_t xl[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+            xl[w] = (uint32_t)(WBYTES + (2 * blk + (t >> 1)) * XBOX + g * 128 + (((4 * (t & 1) + w) ^ g) << 4));
+        const uint32_t sm_stages = smem_u32(stages);
+        const int rbase0 = 16 * rgb + g;                       // tile row of (j = 0, h = 0)
+        // Zero-points of the first segment, requested before the wait on the previous kernel.
+        unsigned short zn[RG][2];
+        if (nseg > 0) {
+            const int64_t tr = (int64_t)sk_seg(a, u0, u1, 0).tile * 128 + rbase0;
+#pragma unroll
+            for (int j = 0; j < RG; ++j)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) zn[j][h] = __half_as_ushort(a.zero[tr + 16 * j + 8 * h]);
+        }
         // Every wait below depends on x, which follows the previous kernel: wait for it first.
         pdl_wait_primary();
         bool ok = true;
-        int seq = 0, fe = 0;
+        int s = 0;
+        uint32_t ph = 0;
+        int fe = 0;
         bool u_seen = false;
         for (int i = 0; i < nseg; ++i) {
             const SkSeg sg = sk_seg(a, u0, u1, i);
@@ -273,46 +286,39 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_we, const __grid_co
 #pragma unroll
             for (int j = 0; j < RG; ++j)
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-                    zb[j][h] = zero_bias_bf16x2((uint32_t)__half2float(a.zero[(int64_t)sg.tile * 128 + 16 * (rgb + j) + g + 8 * h]));
+                for (int h = 0; h < 2; ++h) zb[j][h] = zero_bias_bf16x2((uint32_t)__half2float(__ushort_as_half(zn[j][h])));
+            // The next segment's zero-points, in flight during this one.
+            if (i + 1 < nseg) {
+                const int64_t tr = (int64_t)sk_seg(a, u0, u1, i + 1).tile * 128 + rbase0;
+#pragma unroll
+                for (int j = 0; j < RG; ++j)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) zn[j][h] = __half_as_ushort(a.zero[tr + 16 * j + 8 * h]);
+            }
             float acc[RG][NB][4];
 #pragma unroll
             for (int j = 0; j < RG; ++j)
 #pragma unroll
                 for (int b = 0; b < NB; ++b) acc[j][b][0] = acc[j][b][1] = acc[j][b][2] = acc[j][b][3] = 0.0f;
 
-            for (int kci = sg.kb; kci < sg.ke; ++kci, ++seq) {
-                const int s = seq % NST;
-                const uint32_t ph = (seq / NST) & 1;
-                if (ok && !(mbar_wait_ns(&wfull[s], ph, SK_WAIT_NS) && mbar_wait_ns(&xfull[s], ph, SK_WAIT_NS))) {
-                    sk_fail(a.err, SK_ERR_MBAR, SITE_CVT_WFULL, seq);
+            for (int kci = sg.kb; kci < sg.ke; ++kci) {
+                if (ok && !rk_wait(&full[s], ph)) {
+                    sk_fail(a.err, SK_ERR_MBAR, SITE_CVT_WFULL, kci);
                     ok = false;
                 }
-                const unsigned char* st = stages + (size_t)s * a.stage_bytes;
-                const unsigned char* xs = st + WB;
-                // 16 bytes (32 codes: window codes 32t .. 32t + 31) of rows g and g + 8 per row group.
+                const uint32_t st = sm_stages + (uint32_t)(s * a.stage_bytes);
                 uint4 wa[RG], wb[RG];
 #pragma unroll
                 for (int j = 0; j < RG; ++j) {
-                    const uint32_t r0 = (uint32_t)(16 * (rgb + j) + g);
-                    wa[j] = lds128(st + rk_row_off(r0, win, NWIN) + 16 * t);
-                    wb[j] = lds128(st + rk_row_off(r0 + 8, win, NWIN) + 16 * t);
+                    wa[j] = lds128(st + wl + 1024 * j);
+                    wb[j] = lds128(st + wl + 1024 * j + 512);
                 }
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
-                    // x codes 128 win + 32 t + 8 w .. + 7 of every token: box 2 win + t / 2, chunk
-                    // 4 (t % 2) + w, 128-byte swizzle on the token row.
-                    uint32_t xb[NB][4];
+                    // x codes 32 t + 8 w .. + 7 of the block, every token: natural bf16 pairs.
+                    uint4 xv[NB];
 #pragma unroll
-                    for (int b = 0; b < NB; ++b) {
-                        const uint32_t m = (uint32_t)(8 * b + g);
-                        const uint32_t chunk = (uint32_t)(4 * (t & 1) + w);
-                        const uint4 v = lds128(xs + (2 * win + (t >> 1)) * XBOX + m * 128 + ((chunk ^ (m & 7)) << 4));
-                        xb[b][0] = prmt(v.x, v.z, 0x5410u);   // (x0, x4)
-                        xb[b][1] = prmt(v.x, v.z, 0x7632u);   // (x1, x5)
-                        xb[b][2] = prmt(v.y, v.w, 0x5410u);   // (x2, x6)
-                        xb[b][3] = prmt(v.y, v.w, 0x7632u);   // (x3, x7)
-                    }
+                    for (int b = 0; b < NB; ++b) xv[b] = lds128(st + xl[w] + 1024 * b);
 #pragma unroll
                     for (int j = 0; j < RG; ++j) {
                         const uint32_t qa = w == 0 ? wa[j].x : w == 1 ? wa[j].y : w == 2 ? wa[j].z : wa[j].w;
@@ -320,39 +326,42 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_we, const __grid_co
                         uint32_t ra[4], rb[4];
                         cvt_w4_pairs_i_i4(qa, zb[j][0], ra);
                         cvt_w4_pairs_i_i4(qb, zb[j][1], rb);
+                        const uint32_t af0[4] = {ra[0], rb[0], ra[1], rb[1]};
+                        const uint32_t af1[4] = {ra[2], rb[2], ra[3], rb[3]};
 #pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const uint32_t af[4] = {ra[2 * hh], rb[2 * hh], ra[2 * hh + 1], rb[2 * hh + 1]};
-#pragma unroll
-                            for (int b = 0; b < NB; ++b) mma_bf16_16816(acc[j][b], af, xb[b][2 * hh], xb[b][2 * hh + 1]);
+                        for (int b = 0; b < NB; ++b) {
+                            mma_bf16_16816(acc[j][b], af0, xv[b].x, xv[b].y);
+                            mma_bf16_16816(acc[j][b], af1, xv[b].z, xv[b].w);
                         }
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sempty[s]);
+                if (lane == 0) mbar_arrive(&empty[s]);
+                if (++s == NST) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
 
-            // ---- this warp's final sums for one 16-row group (KC = 256: K halves exchanged) ----
+            // ---- this warp's final sums for one 16-row group (KC = 256: blocks exchanged) ----
             float fin[NB][4];
             int rgf = rgb;
             if constexpr (KC == 256) {
                 const int qd = cw & 3, h = cw >> 2;
                 float* give = red + ((qd * 2 + (1 - h)) * 32 + lane) * (4 * NB);   // the row group handed over
-                if (h == 0) {
 #pragma unroll
-                    for (int b = 0; b < NB; ++b)
-                        *reinterpret_cast<float4*>(give + 4 * b) = make_float4(acc[1][b][0], acc[1][b][1], acc[1][b][2], acc[1][b][3]);
-                } else {
-#pragma unroll
-                    for (int b = 0; b < NB; ++b)
-                        *reinterpret_cast<float4*>(give + 4 * b) = make_float4(acc[0][b][0], acc[0][b][1], acc[0][b][2], acc[0][b][3]);
+                for (int b = 0; b < NB; ++b) {
+                    // acc[1 - h][b], selected without indexing the array by a run-time value
+                    const float v0 = h ? acc[0][b][0] : acc[1][b][0], v1 = h ? acc[0][b][1] : acc[1][b][1];
+                    const float v2 = h ? acc[0][b][2] : acc[1][b][2], v3 = h ? acc[0][b][3] : acc[1][b][3];
+                    *reinterpret_cast<float4*>(give + 4 * b) = make_float4(v0, v1, v2, v3);
                 }
                 named_bar_compute();
                 const float* take = red + ((qd * 2 + h) * 32 + lane) * (4 * NB);
 #pragma unroll
                 for (int b = 0; b < NB; ++b) {
                     const float4 o = *reinterpret_cast<const float4*>(take + 4 * b);
-                    // Fixed order: window 0's sum, then window 1's.
+                    // Fixed order: block 0's sum, then block 1's.
                     if (h == 0) {
                         fin[b][0] = acc[0][b][0] + o.x; fin[b][1] = acc[0][b][1] + o.y;
                         fin[b][2] = acc[0][b][2] + o.z; fin[b][3] = acc[0][b][3] + o.w;
@@ -375,6 +384,7 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_we, const __grid_co
             float* own = a.partial + (size_t)c * BN * 128;
             if (!sg.fin) {
                 // Partial sum of a tile that a higher CTA finalises: [BN][128] fp32, then the flag.
+                // One thread publishes for the CTA after the barrier (its release is cumulative).
 #pragma unroll
                 for (int b = 0; b < NB; ++b) {
                     const int m = 8 * b + 2 * t;
@@ -383,11 +393,15 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_we, const __grid_co
                     __stcg(own + m * 128 + row0 + 8, fin[b][2]);
                     __stcg(own + (m + 1) * 128 + row0 + 8, fin[b][3]);
                 }
-                __threadfence();
                 named_bar_compute();
-                if (cw == 0 && lane == 0) st_release_gpu(a.flags + c, 1u);
+                if (cw == 0 && lane == 0) {
+                    __threadfence();
+                    st_release_gpu(a.flags + c, 1u);
+                }
                 continue;
             }
+            const int64_t n_lo = (int64_t)sg.tile * 128 + row0;
+            const float s_lo = __half2float(a.scale[n_lo]), s_hi = __half2float(a.scale[n_lo + 8]);
             const int c_lo = sg.kb > 0 ? sk_cta_of(a, sg.tile * a.nch) : c;
             if (c_lo < c) {
                 // Lower CTAs computed the tile's first chunks: add their partial sums in CTA order,
@@ -460,8 +474,6 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_we, const __grid_co
                 if (lane == 0) mbar_arrive(bempty);
                 ++fe;
             }
-            const int64_t n_lo = (int64_t)sg.tile * 128 + row0;
-            const float s_lo = __half2float(a.scale[n_lo]), s_hi = __half2float(a.scale[n_lo + 8]);
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
                 const int64_t m = 8 * b + 2 * t;
@@ -515,13 +527,13 @@ bool stream_rk_configure(StreamArgs& a, int bn, int kc, bool deep) {
     a.ntiles = (int)(a.N / 128);
     a.units = a.ntiles * a.nch;
     if (a.grid < 1 || a.grid > a.units || a.grid > (int)STREAM_GRID_MAX) return false;
-    a.stage_bytes = rk_align(rk_w_bytes(kc / 128) + (kc / 64) * bn * 128, 1024);
+    a.stage_bytes = rk_align((kc / 128) * RK_BLOCK_BYTES + (kc / 64) * bn * 128, 1024);
     a.jb = a.nbu = 0;
     a.ec_kr = a.ec_slices = 0;
     int b_bytes = 0, u_bytes = 0, a_bytes = 0, wg_bytes = 0, g_bytes = 0;
     if (a.rank > 0) {
-        const int64_t per = (a.K + a.grid - 1) / a.grid;
-        a.ec_kr = (int)((per + 31) / 32 * 32);
+        a.ec_kr = sk_ec_rows(a.K, a.rank, a.grid);
+        if (a.ec_kr == 0) return false;
         a.ec_slices = (int)((a.K + a.ec_kr - 1) / a.ec_kr);
         if (a.ec_slices > a.grid || a.ec_slices > 255) return false;
         b_bytes = 2 * a.rank * 128;
@@ -531,7 +543,7 @@ bool stream_rk_configure(StreamArgs& a, int bn, int kc, bool deep) {
         g_bytes = rk_align(bn * 4, 128);
     }
     const int red_bytes = kc == 256 ? 4 * 2 * 32 * 4 * (bn / 8) * 4 : 0;
-    const int bar_bytes = 8 * (3 * 16 + 4) + 16;
+    const int bar_bytes = 8 * (2 * 16 + 4) + 16;
     const int fixed = b_bytes + u_bytes + a_bytes + wg_bytes + g_bytes + red_bytes + bar_bytes + 1024;
     const int budget = deep ? (int)SMEM_OPTIN_MAX : 110 * 1024;
     int nst = (budget - fixed) / a.stage_bytes;
@@ -562,15 +574,7 @@ bool stream_rk_configure(StreamArgs& a, int bn, int kc, bool deep) {
 
 template <int NB, int KC>
 static cudaError_t launch_rk_t(const StreamArgs& a, cudaStream_t stream) {
-    CUtensorMap mwe, mwo, mx, mb;
-    // Packed weights [N][K/2] viewed as [N/2 row pairs][2][K/2]: boxes of 64 bytes of one row
-    // parity, 64 pairs (even rows) or 65 pairs (odd rows, starting one pair early).
-    const uint64_t wdims[3] = {(uint64_t)(a.K / 2), 2, (uint64_t)(a.N / 2)};
-    const uint64_t wstr[2] = {(uint64_t)(a.K / 2), (uint64_t)a.K};
-    const uint32_t ebox[3] = {64, 1, 64}, obox[3] = {64, 1, 65};
-    if (!make_map_3d(&mwe, a.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, wdims, wstr, ebox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map_3d(&mwo, a.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, wdims, wstr, obox, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
+    CUtensorMap mx, mb;
     if (!make_map_2d(&mx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.K, (uint64_t)a.M, 64, 8 * NB,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
@@ -595,10 +599,12 @@ static cudaError_t launch_rk_t(const StreamArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, w4_stream_rk_kernel<NB, KC>, mwe, mwo, mx, mb, a);
+    return cudaLaunchKernelEx(&cfg, w4_stream_rk_kernel<NB, KC>, mx, mb, a);
 }
 
 cudaError_t launch_stream_rk(const StreamArgs& a, int bn, cudaStream_t stream) {
+    // Bulk copies of the tile-ordered weights need a 16-byte aligned base.
+    if ((reinterpret_cast<uintptr_t>(a.packed) & 15u) != 0) return cudaErrorInvalidValue;
 #define SPEAR_RK(NB_)                                                                   \
     if (bn == 8 * NB_) return a.kc == 256 ? launch_rk_t<NB_, 256>(a, stream) : launch_rk_t<NB_, 128>(a, stream);
     SPEAR_RK(1) SPEAR_RK(2) SPEAR_RK(4) SPEAR_RK(8)

@@ -70,6 +70,10 @@ SPEAR_DEVI bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint64_t limit_ns) 
 // ---------------------------------------------------------------------------------------------
 // TMA and bulk copies (no multicast anywhere in this library)
 // ---------------------------------------------------------------------------------------------
+// Fetch a tensor map (a kernel parameter) into the descriptor cache ahead of its first copy.
+SPEAR_DEVI void prefetch_tmap(const CUtensorMap* m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
 SPEAR_DEVI void tma_load_2d(void* dst, const CUtensorMap* map, int32_t c0, int32_t c1, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
