@@ -82,7 +82,8 @@ size_t workspace_bytes_for(const spear_plan& p, int64_t M, int64_t N_for_ws, int
     if (p.kernel_id == SPEAR_KERNEL_STREAM || p.kernel_id == SPEAR_KERNEL_STREAM_RK) {
         // fp32 partial sums of the tiles that straddle two CTAs: [grid][tile_m][128].
         const int grid = p.split_k > 0 && K % p.split_k == 0 ? stream_grid(N_for_ws, K, p.split_k, sms, (p.flags & SPEAR_PLAN_DEEP_RING) != 0) : 0;
-        return b + (size_t)grid * p.tile_m * 128 * 4;
+        const size_t word = p.kernel_id == SPEAR_KERNEL_STREAM_RK ? 8 : 4;   // tagged 64-bit words there
+        return b + (size_t)grid * p.tile_m * 128 * word;
     }
     if (p.kernel_id == SPEAR_KERNEL_TC05 && rank > 0) b += tc05_u_bytes(M, rank);
     if (p.kernel_id == SPEAR_KERNEL_TC05 && (p.flags & SPEAR_PLAN_SEPARATE_EC) && rank > 0)

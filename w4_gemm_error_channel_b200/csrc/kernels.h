@@ -150,13 +150,16 @@ struct StreamArgs {
     int off_b, off_red, nfin;       // register path: B-slice buffer, K-half exchange buffer, finalised EC tiles
     uint32_t tmem_cols;
     int ec_kr, ec_slices;           // rows of A per compensator slice, slices (<= grid)
+    int ec_groups;                  // register path: 16-column groups of A (+ the gate) per slice;
+                                    // one (slice, group) item per CTA
     int finalizers;                 // CTAs that finalise at least one tile
     // workspace
     long long* tacc;        // [M][r + 1] int64 fixed-point accumulators (zeroed part)
     unsigned* err;          // error word
     unsigned* flags;        // [grid] partial-sum ready flags (zeroed part)
     unsigned* ec_readers;   // CTAs that have read the accumulators (zeroed part)
-    float* partial;         // [grid][BN][128] fp32 partial sums
+    float* partial;         // [grid][BN][128] fp32 partial sums (register path: 64-bit words,
+                            // ready tag in the high half; the reader zeroes them)
 };
 int stream_grid(int64_t N, int64_t K, int kc, int sms, bool deep);
 // The register-path variant (stream_rk.cu): same schedule and workspace, converted weights in

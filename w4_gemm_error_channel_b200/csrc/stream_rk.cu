@@ -42,7 +42,12 @@ namespace spear {
 constexpr int RK_THREADS = 320;
 constexpr int RK_COMPUTE_WARPS = 8;
 constexpr int RK_BLOCK_BYTES = 128 * 64;       // one 128 x 128-code block of the tile order
+constexpr int RK_EC_KR_MAX = 1024;             // rows of A per compensator item, at most
 
+SPEAR_DEVI void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+SPEAR_DEVI unsigned long long rk_tagged(float v) { return (1ull << 32) | (unsigned long long)__float_as_uint(v); }
 SPEAR_DEVI void named_bar_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }   // warps 1-8
 SPEAR_DEVI uint4 lds128(uint32_t saddr) {
     uint4 v;
@@ -54,55 +59,123 @@ SPEAR_DEVI bool rk_wait(uint64_t* bar, uint32_t parity) {
     return mbar_try(bar, parity) || mbar_wait_ns(bar, parity, SK_WAIT_NS);
 }
 
-// All 256 compute threads: wait (bounded) until every accumulator word holds all slices, then
-// u[m][j] = sigmoid(p[m] + b_g) t[m][j] (fp32) for m < rows (zero past M) into ubuf [rows][ustride].
-// Each thread reads its words in batches of RK_UB independent loads.
-constexpr int RK_UB = 8;
-SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc, float* gs, float* ubuf, int ustride,
-                             int rows) {
-    const int tid = (int)threadIdx.x - 32;           // compute threads are 32 .. 287
+// u for every token of the tile, by the 256 compute threads: warp w takes tokens w, w + 8, ...,
+// lane l the accumulator words l, l + 32, ... of a token (t, then the gate pre-activation in word
+// r).  A token's words are read together, TB tokens at a time, until every word holds all
+// slices (bounded); then u[m][j] = sigmoid(p[m] + b_g) t[m][j] (fp32, zero past M) goes to
+// ubuf [rows][ustride].  The caller synchronises the compute warps afterwards.
+SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc, float* ubuf, int ustride, int rows,
+                             int cw, int lane) {
+    constexpr int WMAX = 5;                              // words per lane and token: r + 1 <= 160
     const int r = a.rank;
+    const int nw = (r + 1 + 31) / 32;
+    const int gi = r / 32, gl = r % 32;                  // the gate word: chunk gi of lane gl
     const unsigned long long want = (unsigned long long)a.ec_slices;
-    // pass 0: the gate words (column r); pass 1: t.
-    for (int pass = 0; pass < 2; ++pass) {
-        const int total = pass == 0 ? rows : rows * r;
-        for (int base = 0; base < total; base += 256 * RK_UB) {
-            unsigned long long v[RK_UB];
-            int idx[RK_UB];
+    for (int m0 = cw; m0 < rows; m0 += 16) {
+        // Tokens m0 and m0 + 8, all their words in flight together.
+        const int m1 = m0 + 8;
+        unsigned long long v0[WMAX], v1[WMAX];
+        const uint64_t t0 = globaltimer_ns();
+        for (;;) {
+            bool done = true;
 #pragma unroll
-            for (int q = 0; q < RK_UB; ++q) {
-                const int e = base + tid + 256 * q;
-                idx[q] = e < total ? e : -1;
+            for (int i = 0; i < WMAX; ++i) {
+                const int j = lane + 32 * i;
+                const bool in = i < nw && j <= r;
+                v0[i] = in && m0 < a.M ? ld_relaxed_u64(tacc_word(tacc, a, m0, j)) : want;
+                v1[i] = in && m1 < a.M ? ld_relaxed_u64(tacc_word(tacc, a, m1, j)) : want;
+                done = done && ((v0[i] & 0xFFull) == want) && ((v1[i] & 0xFFull) == want);
             }
-            const uint64_t t0 = globaltimer_ns();
-            for (;;) {
-                bool done = true;
-#pragma unroll
-                for (int q = 0; q < RK_UB; ++q) {
-                    const int e = idx[q];
-                    const int m = pass == 0 ? e : e / r, j = pass == 0 ? r : e % r;
-                    v[q] = (e >= 0 && m < a.M) ? ld_relaxed_u64(tacc_word(tacc, a, m, j)) : want;
-                }
-#pragma unroll
-                for (int q = 0; q < RK_UB; ++q) done = done && ((v[q] & 0xFFull) == want);
-                if (done) break;
-                if (globaltimer_ns() - t0 > SK_WAIT_NS) {
-                    sk_fail(a.err, SK_ERR_FLAG, SITE_EC_TACC, base);
-                    break;
-                }
-                __nanosleep(64);
+            if (__all_sync(0xFFFFFFFFu, done)) break;
+            if (__any_sync(0xFFFFFFFFu, globaltimer_ns() - t0 > SK_WAIT_NS)) {
+                if (lane == 0) sk_fail(a.err, SK_ERR_FLAG, SITE_EC_TACC, m0);
+                break;
             }
+            __nanosleep(64);
+        }
+        unsigned long long g0 = 0, g1 = 0;
 #pragma unroll
-            for (int q = 0; q < RK_UB; ++q) {
-                const int e = idx[q];
-                if (e < 0) continue;
-                const int m = pass == 0 ? e : e / r, j = pass == 0 ? r : e % r;
-                const float val = m < a.M ? __ll2float_rn((long long)v[q] >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) : 0.0f;
-                if (pass == 0) gs[m] = m < a.M ? 1.0f / (1.0f + expf(-(val + a.b_g))) : 0.0f;
-                else ubuf[m * ustride + j] = val * gs[m];
+        for (int i = 0; i < WMAX; ++i)
+            if (i == gi) { g0 = v0[i]; g1 = v1[i]; }
+        g0 = __shfl_sync(0xFFFFFFFFu, g0, gl);
+        g1 = __shfl_sync(0xFFFFFFFFu, g1, gl);
+        const float gate0 = m0 < a.M ? 1.0f / (1.0f + expf(-(__ll2float_rn((long long)g0 >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) + a.b_g))) : 0.0f;
+        const float gate1 = m1 < a.M ? 1.0f / (1.0f + expf(-(__ll2float_rn((long long)g1 >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) + a.b_g))) : 0.0f;
+#pragma unroll
+        for (int i = 0; i < WMAX; ++i) {
+            const int j = lane + 32 * i;
+            if (i < nw && j < r) {
+                ubuf[m0 * ustride + j] = __ll2float_rn((long long)v0[i] >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) * gate0;
+                if (m1 < rows)
+                    ubuf[m1 * ustride + j] = __ll2float_rn((long long)v1[i] >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) * gate1;
             }
         }
-        named_bar_compute();
+    }
+}
+
+// The compensator's work item of one CTA (one warp): 16 columns of t = x A (column group grp < r/16)
+// or the gate pre-activation p = x w_g (grp == r/16) over rows [k0, k0 + rows) of A, every token.
+// Tokens are the M = 16 operand of mma.sync m16n8k16 and the 16 columns two n8 tiles (even and
+// odd columns) so that one 32-bit word of a row feeds both; the gate is one n8 tile with w_g in
+// column 0.  As: the group's columns, [rows][16] bf16; wgs: w_g rows.  Each accumulator word gets
+// one addition per K slice.
+SPEAR_DEVI void rk_ec_item(const StreamArgs& a, const uint16_t* As, const uint16_t* wgs, int64_t k0, int rows, int grp,
+                           unsigned long long* tacc) {
+    constexpr int KS = 8;                  // k16 steps whose x fragments are in flight together
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int r = a.rank;
+    const bool gate = grp == r / 16;
+    const float lim = SK_FIX_TOTAL / (float)a.ec_slices;
+    const int ksteps = rows / 16;
+    for (int m0 = 0; m0 < a.M; m0 += 16) {
+        const int64_t ma = m0 + g, mb = m0 + g + 8;
+        float de[4] = {0.f, 0.f, 0.f, 0.f}, dod[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int kb = 0; kb < ksteps; kb += KS) {
+            uint32_t xa[KS][4];
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                const int64_t k = k0 + 16 * (kb + kk) + 2 * t;
+                const bool in = kb + kk < ksteps;
+                xa[kk][0] = in && ma < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + ma * a.K + k)) : 0u;
+                xa[kk][1] = in && mb < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb * a.K + k)) : 0u;
+                xa[kk][2] = in && ma < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + ma * a.K + k + 8)) : 0u;
+                xa[kk][3] = in && mb < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb * a.K + k + 8)) : 0u;
+            }
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                if (kb + kk >= ksteps) break;
+                const int kr = 16 * (kb + kk) + 2 * t;    // row of the slice
+                if (!gate) {
+                    const uint16_t* p = As + kr * 16 + 2 * g;
+                    const uint32_t w0 = lds_u32(p), w1 = lds_u32(p + 16), w2 = lds_u32(p + 8 * 16), w3 = lds_u32(p + 9 * 16);
+                    mma_bf16_16816(de, xa[kk], prmt(w0, w1, 0x5410u), prmt(w2, w3, 0x5410u));
+                    mma_bf16_16816(dod, xa[kk], prmt(w0, w1, 0x7632u), prmt(w2, w3, 0x7632u));
+                } else {
+                    const uint32_t b0 = g == 0 ? lds_u32(wgs + kr) : 0u;
+                    const uint32_t b1 = g == 0 ? lds_u32(wgs + kr + 8) : 0u;
+                    mma_bf16_16816(de, xa[kk], b0, b1);
+                }
+            }
+        }
+        // Lane (g, t) holds columns 16 grp + 4t + {0, 1, 2, 3} (even tile: +0, +2; odd: +1, +3)
+        // of tokens ma (entries 0, 1) and mb (entries 2, 3); the gate tile's column 0 is in t == 0.
+        auto add = [&](int64_t m, int col, float v) {
+            if (m >= a.M) return;
+            if (!(fabsf(v) < lim)) {
+                atomicOr(a.err, SK_ERR_RANGE);
+                v = 0.0f;
+            }
+            const unsigned long long fx = (unsigned long long)__float2ll_rn(v * SK_FIX_ONE);
+            red_add_u64(tacc_word(tacc, a, m, col), (fx << SK_FIX_COUNT_BITS) | 1ull);
+        };
+        if (!gate) {
+            const int c0 = 16 * grp + 4 * t;
+            add(ma, c0, de[0]); add(ma, c0 + 1, dod[0]); add(ma, c0 + 2, de[1]); add(ma, c0 + 3, dod[1]);
+            add(mb, c0, de[2]); add(mb, c0 + 1, dod[2]); add(mb, c0 + 2, de[3]); add(mb, c0 + 3, dod[3]);
+        } else if (t == 0) {
+            add(ma, r, de[0]);
+            add(mb, r, de[2]);
+        }
     }
 }
 
@@ -137,8 +210,10 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     uint16_t* As = reinterpret_cast<uint16_t*>(smem + a.off_a);
     uint16_t* wgs = reinterpret_cast<uint16_t*>(smem + a.off_wg);
     float* red = reinterpret_cast<float*>(smem + a.off_red);  // block exchange [4][2][32][4 NB]
-    const bool has_slice = has_ec && c < a.ec_slices;
-    const int64_t ec_k0 = (int64_t)c * a.ec_kr;
+    // Compensator work item of this CTA: K slice c / ec_groups, column group c % ec_groups.
+    const bool has_slice = has_ec && c < a.ec_slices * a.ec_groups;
+    const int ec_grp = has_slice ? c % a.ec_groups : 0;
+    const int64_t ec_k0 = has_slice ? (int64_t)(c / a.ec_groups) * a.ec_kr : 0;
     const int ec_rows = has_slice ? (int)imin64(a.ec_kr, a.K - ec_k0) : 0;
 
     if (threadIdx.x == 0) {
@@ -295,6 +370,13 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
 #pragma unroll
                     for (int h = 0; h < 2; ++h) zn[j][h] = __half_as_ushort(a.zero[tr + 16 * j + 8 * h]);
             }
+            // Scales of the rows this warp finalises (KC = 256: row group rgb + blk), in flight
+            // during the main loop.
+            uint32_t s_pair = 0;                                 // fp16 scales of rows n_lo, n_lo + 8
+            if (sg.fin) {
+                const int64_t n = (int64_t)sg.tile * 128 + 16 * (KC == 256 ? rgb + blk : rgb) + g;
+                s_pair = (uint32_t)__half_as_ushort(a.scale[n]) | ((uint32_t)__half_as_ushort(a.scale[n + 8]) << 16);
+            }
             float acc[RG][NB][4];
 #pragma unroll
             for (int j = 0; j < RG; ++j)
@@ -345,7 +427,6 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
 
             // ---- this warp's final sums for one 16-row group (KC = 256: blocks exchanged) ----
             float fin[NB][4];
-            int rgf = rgb;
             if constexpr (KC == 256) {
                 const int qd = cw & 3, h = cw >> 2;
                 float* give = red + ((qd * 2 + (1 - h)) * 32 + lane) * (4 * NB);   // the row group handed over
@@ -370,7 +451,6 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                         fin[b][2] = o.z + acc[1][b][2]; fin[b][3] = o.w + acc[1][b][3];
                     }
                 }
-                rgf = rgb + h;
                 named_bar_compute();              // the exchange buffer is free again
             } else {
 #pragma unroll
@@ -380,67 +460,94 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
             }
 
             // ---- epilogue: rows 16 rgf + g (+ 8) of the tile; tokens 8 b + 2 t (+ 1) ----
+            const int rgf = KC == 256 ? rgb + blk : rgb;
             const int row0 = 16 * rgf + g;
-            float* own = a.partial + (size_t)c * BN * 128;
+            const int64_t n_lo = (int64_t)sg.tile * 128 + row0;
+            unsigned long long* parts = reinterpret_cast<unsigned long long*>(a.partial);
             if (!sg.fin) {
-                // Partial sum of a tile that a higher CTA finalises: [BN][128] fp32, then the flag.
-                // One thread publishes for the CTA after the barrier (its release is cumulative).
+                // Partial sum of a tile that a higher CTA finalises: [BN][128] 64-bit words, the fp32
+                // value in the low half and the ready tag 1 in the high half, each one store.  The
+                // reader polls the words themselves and zeroes them after use: no flag, no fence.
+                unsigned long long* own = parts + (size_t)c * BN * 128;
 #pragma unroll
                 for (int b = 0; b < NB; ++b) {
                     const int m = 8 * b + 2 * t;
-                    __stcg(own + m * 128 + row0, fin[b][0]);
-                    __stcg(own + (m + 1) * 128 + row0, fin[b][1]);
-                    __stcg(own + m * 128 + row0 + 8, fin[b][2]);
-                    __stcg(own + (m + 1) * 128 + row0 + 8, fin[b][3]);
-                }
-                named_bar_compute();
-                if (cw == 0 && lane == 0) {
-                    __threadfence();
-                    st_release_gpu(a.flags + c, 1u);
+                    st_relaxed_u64(own + m * 128 + row0, rk_tagged(fin[b][0]));
+                    st_relaxed_u64(own + (m + 1) * 128 + row0, rk_tagged(fin[b][1]));
+                    st_relaxed_u64(own + m * 128 + row0 + 8, rk_tagged(fin[b][2]));
+                    st_relaxed_u64(own + (m + 1) * 128 + row0 + 8, rk_tagged(fin[b][3]));
                 }
                 continue;
             }
-            const int64_t n_lo = (int64_t)sg.tile * 128 + row0;
-            const float s_lo = __half2float(a.scale[n_lo]), s_hi = __half2float(a.scale[n_lo + 8]);
+            const float s_lo = __half2float(__ushort_as_half((unsigned short)(s_pair & 0xFFFFu)));
+            const float s_hi = __half2float(__ushort_as_half((unsigned short)(s_pair >> 16)));
             const int c_lo = sg.kb > 0 ? sk_cta_of(a, sg.tile * a.nch) : c;
             if (c_lo < c) {
                 // Lower CTAs computed the tile's first chunks: add their partial sums in CTA order,
-                // then this CTA's own.
-                if (cw == 0 && lane == 0) {
-                    for (int cc = c_lo; cc < c; ++cc) {
-                        unsigned v;
-                        if (!poll_until<unsigned>(ld_acquire_gpu, a.flags + cc, [](unsigned w) { return w != 0u; }, v))
-                            sk_fail(a.err, SK_ERR_FLAG, SITE_EPI_FLAG, cc);
-                    }
-                }
-                named_bar_compute();
+                // then this CTA's own.  PB CTAs' words are polled at a time, all loads in flight
+                // together, until their tags say ready (bounded); each lane zeroes what it read.
+                constexpr int PB = NB <= 1 ? 4 : (NB <= 2 ? 2 : 1);
+                float p[NB][4];
+                for (int base = c_lo; base < c; base += PB) {
+                    unsigned long long q[PB][NB][4];
+                    const uint64_t t0 = globaltimer_ns();
+                    for (;;) {
+                        bool ready = true;
 #pragma unroll
-                for (int b = 0; b < NB; ++b) {
-                    const int m = 8 * b + 2 * t;
-                    float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-                    for (int cc = c_lo; cc < c; ++cc) {
-                        const float* pp = a.partial + (size_t)cc * BN * 128;
-                        const float q0 = __ldcg(pp + m * 128 + row0), q1 = __ldcg(pp + (m + 1) * 128 + row0);
-                        const float q2 = __ldcg(pp + m * 128 + row0 + 8), q3 = __ldcg(pp + (m + 1) * 128 + row0 + 8);
-                        if (cc == c_lo) { p0 = q0; p1 = q1; p2 = q2; p3 = q3; }
-                        else { p0 += q0; p1 += q1; p2 += q2; p3 += q3; }
+                        for (int k = 0; k < PB; ++k) {
+                            const int cc = base + k < c ? base + k : c - 1;
+                            const unsigned long long* pp = parts + (size_t)cc * BN * 128;
+#pragma unroll
+                            for (int b = 0; b < NB; ++b) {
+                                const int m = 8 * b + 2 * t;
+                                q[k][b][0] = ld_relaxed_u64(pp + m * 128 + row0);
+                                q[k][b][1] = ld_relaxed_u64(pp + (m + 1) * 128 + row0);
+                                q[k][b][2] = ld_relaxed_u64(pp + m * 128 + row0 + 8);
+                                q[k][b][3] = ld_relaxed_u64(pp + (m + 1) * 128 + row0 + 8);
+#pragma unroll
+                                for (int v = 0; v < 4; ++v) ready = ready && (q[k][b][v] >> 32) == 1ull;
+                            }
+                        }
+                        if (ready) break;
+                        if (globaltimer_ns() - t0 > SK_WAIT_NS) {
+                            sk_fail(a.err, SK_ERR_FLAG, SITE_EPI_FLAG, base);
+                            break;
+                        }
+                        __nanosleep(32);
                     }
-                    fin[b][0] = p0 + fin[b][0]; fin[b][1] = p1 + fin[b][1];
-                    fin[b][2] = p2 + fin[b][2]; fin[b][3] = p3 + fin[b][3];
+#pragma unroll
+                    for (int k = 0; k < PB; ++k) {
+                        if (base + k >= c) break;
+                        unsigned long long* pp = parts + (size_t)(base + k) * BN * 128;
+#pragma unroll
+                        for (int b = 0; b < NB; ++b) {
+                            const int m = 8 * b + 2 * t;
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                const float x = __uint_as_float((uint32_t)q[k][b][v]);
+                                p[b][v] = (base + k == c_lo) ? x : p[b][v] + x;
+                            }
+                            st_relaxed_u64(pp + m * 128 + row0, 0ull);
+                            st_relaxed_u64(pp + (m + 1) * 128 + row0, 0ull);
+                            st_relaxed_u64(pp + m * 128 + row0 + 8, 0ull);
+                            st_relaxed_u64(pp + (m + 1) * 128 + row0 + 8, 0ull);
+                        }
+                    }
                 }
-                named_bar_compute();
-                if (cw == 0 && lane == 0)
-                    for (int cc = c_lo; cc < c; ++cc) a.flags[cc] = 0u;   // re-armed for the next call
+#pragma unroll
+                for (int b = 0; b < NB; ++b)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) fin[b][v] = p[b][v] + fin[b][v];
             }
             float e[NB][4];
 #pragma unroll
             for (int b = 0; b < NB; ++b) e[b][0] = e[b][1] = e[b][2] = e[b][3] = 0.0f;
             if (has_ec) {
                 if (!u_seen) {
-                    // u for every token, read by all 256 compute threads in batches of independent
-                    // loads (one dependent round trip per batch, not per word).
-                    rk_compute_u(a, reinterpret_cast<const unsigned long long*>(a.tacc),
-                                 reinterpret_cast<float*>(smem + a.off_g), ubuf, ustride, BN);
+                    // u for every token, read by all 256 compute threads (one round trip of loads
+                    // per two tokens of a warp).
+                    rk_compute_u(a, reinterpret_cast<const unsigned long long*>(a.tacc), ubuf, ustride, BN, cw, lane);
+                    named_bar_compute();
                     if (cw == 0) ec_retire(a, reinterpret_cast<unsigned long long*>(a.tacc));
                     u_seen = true;
                 }
@@ -495,17 +602,25 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         }
     } else {
         // ---------------- compensator (warp 9) ----------------
-        if (has_slice && lane == 0) {
-            const uint32_t abytes = (uint32_t)(ec_rows * a.rank * 2), gbytes = (uint32_t)(ec_rows * 2);
-            mbar_arrive_expect_tx(ec_bar, abytes + gbytes);
-            bulk_load(As, a.A + ec_k0 * a.rank, abytes, ec_bar);
-            bulk_load(wgs, a.wg + ec_k0, gbytes, ec_bar);
+        // The item's rows of A (32 bytes each: its 16 columns) or of w_g, before the wait on the
+        // previous kernel (they do not depend on it).
+        const bool gate_item = ec_grp == a.rank / 16;
+        if (has_slice) {
+            if (lane == 0)
+                mbar_arrive_expect_tx(ec_bar, gate_item ? (uint32_t)(ec_rows * 2) : (uint32_t)(ec_rows * 32));
+            __syncwarp();
+            if (gate_item) {
+                if (lane == 0) bulk_load(wgs, a.wg + ec_k0, (uint32_t)(ec_rows * 2), ec_bar);
+            } else {
+                for (int i = lane; i < ec_rows; i += 32)
+                    bulk_load(As + i * 16, a.A + (ec_k0 + i) * a.rank + 16 * ec_grp, 32u, ec_bar);
+            }
         }
         pdl_wait_primary();
         unsigned long long* tacc = reinterpret_cast<unsigned long long*>(a.tacc);
         if (has_slice) {
             if (mbar_wait_ns(ec_bar, 0, SK_WAIT_NS))
-                ec_slice(a, As, wgs, ec_k0, ec_rows, tacc);
+                rk_ec_item(a, As, wgs, ec_k0, ec_rows, ec_grp, tacc);
             else if (lane == 0)
                 sk_fail(a.err, SK_ERR_MBAR, SITE_EC_BAR, 0);
         }
@@ -530,20 +645,28 @@ bool stream_rk_configure(StreamArgs& a, int bn, int kc, bool deep) {
     a.stage_bytes = rk_align((kc / 128) * RK_BLOCK_BYTES + (kc / 64) * bn * 128, 1024);
     a.jb = a.nbu = 0;
     a.ec_kr = a.ec_slices = 0;
+    a.ec_groups = 1;
     int b_bytes = 0, u_bytes = 0, a_bytes = 0, wg_bytes = 0, g_bytes = 0;
     if (a.rank > 0) {
-        a.ec_kr = sk_ec_rows(a.K, a.rank, a.grid);
-        if (a.ec_kr == 0) return false;
-        a.ec_slices = (int)((a.K + a.ec_kr - 1) / a.ec_kr);
-        if (a.ec_slices > a.grid || a.ec_slices > 255) return false;
+        // (K slice, column group) items, one per CTA: as many K slices as the grid allows
+        // (at most 255 for the 8-bit count), rows a multiple of 16, at most RK_EC_KR_MAX.
+        a.ec_groups = a.rank / 16 + 1;
+        int64_t slices = a.grid / a.ec_groups;
+        if (slices > 255) slices = 255;
+        if (slices < 1) return false;
+        int64_t kr = (a.K + slices - 1) / slices;
+        kr = (kr + 15) / 16 * 16;
+        if (kr > RK_EC_KR_MAX) return false;
+        a.ec_kr = (int)kr;
+        a.ec_slices = (int)((a.K + kr - 1) / kr);
+        if ((int64_t)a.ec_slices * a.ec_groups > a.grid) return false;
         b_bytes = 2 * a.rank * 128;
         u_bytes = rk_align(bn * (a.rank + 4) * 4, 128);
-        a_bytes = rk_align(a.ec_kr * a.rank * 2, 128);
+        a_bytes = rk_align(a.ec_kr * 32, 128);
         wg_bytes = rk_align(a.ec_kr * 2, 128);
-        g_bytes = rk_align(bn * 4, 128);
     }
     const int red_bytes = kc == 256 ? 4 * 2 * 32 * 4 * (bn / 8) * 4 : 0;
-    const int bar_bytes = 8 * (2 * 16 + 4) + 16;
+    const int bar_bytes = 8 * (2 * 16 + 5) + 16;
     const int fixed = b_bytes + u_bytes + a_bytes + wg_bytes + g_bytes + red_bytes + bar_bytes + 1024;
     const int budget = deep ? (int)SMEM_OPTIN_MAX : 110 * 1024;
     int nst = (budget - fixed) / a.stage_bytes;
