@@ -32,7 +32,8 @@
 //               shared memory by ldmatrix.trans, u split into bf16 hi + lo), y = s[n] D + E.  In a
 //               CTA that finalises a tile they read the accumulators and form u (fp32) together at
 //               its first finalisation.
-//   warp 9      the compensator's slice of x A.
+//   warp 9      the compensator's work item: one 16-column group of x A (or x w_g) over one K
+//               slice, A fragments loaded straight into registers.
 // Every wait is bounded in time; on timeout a bit of the error word is set and the site recorded.
 #include "kernels.h"
 #include "stream_common.cuh"
@@ -44,8 +45,18 @@ constexpr int RK_COMPUTE_WARPS = 8;
 constexpr int RK_BLOCK_BYTES = 128 * 64;       // one 128 x 128-code block of the tile order
 constexpr int RK_EC_KR_MAX = 1024;             // rows of A per compensator item, at most
 
-SPEAR_DEVI void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+// Tagged words (a value and its ready tag in one aligned 64-bit word) and the compensator's
+// accumulators are written and read as single 64-bit accesses at the L2 (.cg: never from a
+// stale L1 line), so a reader sees a word's tag and value from the same write.  These are plain
+// loads and stores: strong (.relaxed.gpu) ones were measured to issue one after another, which
+// made a finaliser's reads take one L2 round trip per word.
+SPEAR_DEVI void st_cg_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.global.cg.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+SPEAR_DEVI unsigned long long ld_cg_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.global.cg.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
 }
 SPEAR_DEVI unsigned long long rk_tagged(float v) { return (1ull << 32) | (unsigned long long)__float_as_uint(v); }
 SPEAR_DEVI void named_bar_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }   // warps 1-8
@@ -82,8 +93,8 @@ SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc
             for (int i = 0; i < WMAX; ++i) {
                 const int j = lane + 32 * i;
                 const bool in = i < nw && j <= r;
-                v0[i] = in && m0 < a.M ? ld_relaxed_u64(tacc_word(tacc, a, m0, j)) : want;
-                v1[i] = in && m1 < a.M ? ld_relaxed_u64(tacc_word(tacc, a, m1, j)) : want;
+                v0[i] = in && m0 < a.M ? ld_cg_u64(tacc_word(tacc, a, m0, j)) : want;
+                v1[i] = in && m1 < a.M ? ld_cg_u64(tacc_word(tacc, a, m1, j)) : want;
                 done = done && ((v0[i] & 0xFFull) == want) && ((v1[i] & 0xFFull) == want);
             }
             if (__all_sync(0xFFFFFFFFu, done)) break;
@@ -117,64 +128,96 @@ SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc
 // or the gate pre-activation p = x w_g (grp == r/16) over rows [k0, k0 + rows) of A, every token.
 // Tokens are the M = 16 operand of mma.sync m16n8k16 and the 16 columns two n8 tiles (even and
 // odd columns) so that one 32-bit word of a row feeds both; the gate is one n8 tile with w_g in
-// column 0.  As: the group's columns, [rows][16] bf16; wgs: w_g rows.  Each accumulator word gets
-// one addition per K slice.
-SPEAR_DEVI void rk_ec_item(const StreamArgs& a, const uint16_t* As, const uint16_t* wgs, int64_t k0, int rows, int grp,
-                           unsigned long long* tacc) {
-    constexpr int KS = 8;                  // k16 steps whose x fragments are in flight together
+// column 0.  The fragments of A come straight from global memory in chunks of KS k-steps, the
+// first chunk before the wait on the previous kernel (A does not depend on it), x after it.
+// Each accumulator word gets one addition per K slice.
+SPEAR_DEVI void rk_ec_item(const StreamArgs& a, int64_t k0, int rows, int grp, unsigned long long* tacc) {
+    constexpr int KS = 4;                   // k16 steps per chunk
+    constexpr int MB = 4;                   // 16-token blocks (M <= 64)
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int r = a.rank;
     const bool gate = grp == r / 16;
     const float lim = SK_FIX_TOTAL / (float)a.ec_slices;
     const int ksteps = rows / 16;
-    for (int m0 = 0; m0 < a.M; m0 += 16) {
-        const int64_t ma = m0 + g, mb = m0 + g + 8;
-        float de[4] = {0.f, 0.f, 0.f, 0.f}, dod[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int kb = 0; kb < ksteps; kb += KS) {
+    const int mblocks = (int)((a.M + 15) / 16);
+    float de[MB][4], dod[MB][4];
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) de[mb][v] = dod[mb][v] = 0.0f;
+    uint32_t w[KS][4];
+    auto load_a = [&](int kb) {
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            const int kr = 16 * (kb + kk) + 2 * t;
+            const bool in = kb + kk < ksteps;
+            if (!gate) {
+                const uint16_t* p = a.A + (k0 + kr) * r + 16 * grp + 2 * g;
+                w[kk][0] = in ? ldg_u32_nc(p) : 0u;
+                w[kk][1] = in ? ldg_u32_nc(p + r) : 0u;
+                w[kk][2] = in ? ldg_u32_nc(p + 8 * r) : 0u;
+                w[kk][3] = in ? ldg_u32_nc(p + 9 * r) : 0u;
+            } else {
+                const uint16_t* p = a.wg + k0 + kr;
+                w[kk][0] = in && g == 0 ? ldg_u32_nc(p) : 0u;
+                w[kk][1] = in && g == 0 ? ldg_u32_nc(p + 8) : 0u;
+                w[kk][2] = w[kk][3] = 0u;
+            }
+        }
+    };
+    load_a(0);
+    pdl_wait_primary();
+    for (int kb = 0; kb < ksteps; kb += KS) {
+        if (kb > 0) load_a(kb);
+#pragma unroll
+        for (int mb = 0; mb < MB; ++mb) {
+            if (mb >= mblocks) break;
+            const int64_t ma = 16 * mb + g, mb8 = ma + 8;
             uint32_t xa[KS][4];
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
                 const int64_t k = k0 + 16 * (kb + kk) + 2 * t;
                 const bool in = kb + kk < ksteps;
                 xa[kk][0] = in && ma < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + ma * a.K + k)) : 0u;
-                xa[kk][1] = in && mb < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb * a.K + k)) : 0u;
+                xa[kk][1] = in && mb8 < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb8 * a.K + k)) : 0u;
                 xa[kk][2] = in && ma < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + ma * a.K + k + 8)) : 0u;
-                xa[kk][3] = in && mb < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb * a.K + k + 8)) : 0u;
+                xa[kk][3] = in && mb8 < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb8 * a.K + k + 8)) : 0u;
             }
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
                 if (kb + kk >= ksteps) break;
-                const int kr = 16 * (kb + kk) + 2 * t;    // row of the slice
                 if (!gate) {
-                    const uint16_t* p = As + kr * 16 + 2 * g;
-                    const uint32_t w0 = lds_u32(p), w1 = lds_u32(p + 16), w2 = lds_u32(p + 8 * 16), w3 = lds_u32(p + 9 * 16);
-                    mma_bf16_16816(de, xa[kk], prmt(w0, w1, 0x5410u), prmt(w2, w3, 0x5410u));
-                    mma_bf16_16816(dod, xa[kk], prmt(w0, w1, 0x7632u), prmt(w2, w3, 0x7632u));
+                    mma_bf16_16816(de[mb], xa[kk], prmt(w[kk][0], w[kk][1], 0x5410u), prmt(w[kk][2], w[kk][3], 0x5410u));
+                    mma_bf16_16816(dod[mb], xa[kk], prmt(w[kk][0], w[kk][1], 0x7632u), prmt(w[kk][2], w[kk][3], 0x7632u));
                 } else {
-                    const uint32_t b0 = g == 0 ? lds_u32(wgs + kr) : 0u;
-                    const uint32_t b1 = g == 0 ? lds_u32(wgs + kr + 8) : 0u;
-                    mma_bf16_16816(de, xa[kk], b0, b1);
+                    mma_bf16_16816(de[mb], xa[kk], w[kk][0], w[kk][1]);
                 }
             }
         }
-        // Lane (g, t) holds columns 16 grp + 4t + {0, 1, 2, 3} (even tile: +0, +2; odd: +1, +3)
-        // of tokens ma (entries 0, 1) and mb (entries 2, 3); the gate tile's column 0 is in t == 0.
-        auto add = [&](int64_t m, int col, float v) {
-            if (m >= a.M) return;
-            if (!(fabsf(v) < lim)) {
-                atomicOr(a.err, SK_ERR_RANGE);
-                v = 0.0f;
-            }
-            const unsigned long long fx = (unsigned long long)__float2ll_rn(v * SK_FIX_ONE);
-            red_add_u64(tacc_word(tacc, a, m, col), (fx << SK_FIX_COUNT_BITS) | 1ull);
-        };
+    }
+    // Lane (g, t) holds columns 16 grp + 4t + {0, 1, 2, 3} (even tile: +0, +2; odd: +1, +3) of
+    // tokens 16 mb + g (entries 0, 1) and 16 mb + g + 8 (entries 2, 3); the gate tile's column 0
+    // is in t == 0.
+    auto add = [&](int64_t m, int col, float v) {
+        if (m >= a.M) return;
+        if (!(fabsf(v) < lim)) {
+            atomicOr(a.err, SK_ERR_RANGE);
+            v = 0.0f;
+        }
+        const unsigned long long fx = (unsigned long long)__float2ll_rn(v * SK_FIX_ONE);
+        red_add_u64(tacc_word(tacc, a, m, col), (fx << SK_FIX_COUNT_BITS) | 1ull);
+    };
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb) {
+        if (mb >= mblocks) break;
+        const int64_t ma = 16 * mb + g, mb8 = ma + 8;
         if (!gate) {
             const int c0 = 16 * grp + 4 * t;
-            add(ma, c0, de[0]); add(ma, c0 + 1, dod[0]); add(ma, c0 + 2, de[1]); add(ma, c0 + 3, dod[1]);
-            add(mb, c0, de[2]); add(mb, c0 + 1, dod[2]); add(mb, c0 + 2, de[3]); add(mb, c0 + 3, dod[3]);
+            add(ma, c0, de[mb][0]); add(ma, c0 + 1, dod[mb][0]); add(ma, c0 + 2, de[mb][1]); add(ma, c0 + 3, dod[mb][1]);
+            add(mb8, c0, de[mb][2]); add(mb8, c0 + 1, dod[mb][2]); add(mb8, c0 + 2, de[mb][3]); add(mb8, c0 + 3, dod[mb][3]);
         } else if (t == 0) {
-            add(ma, r, de[0]);
-            add(mb, r, de[2]);
+            add(ma, r, de[mb][0]);
+            add(mb8, r, de[mb][2]);
         }
     }
 }
@@ -196,7 +239,6 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     uint64_t* empty = full + NST;                                         // stage consumed (8 warps)
     uint64_t* bfull = empty + NST;                                        // B slice landed
     uint64_t* bempty = bfull + 1;                                         // B slice consumed (8 warps)
-    uint64_t* ec_bar = bempty + 1;                                        // A and w_g slices landed
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x;
@@ -207,8 +249,6 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     unsigned char* bbuf = smem + a.off_b;                 // B[:, tile]: two [r][64] boxes, 128-byte swizzle
     float* ubuf = reinterpret_cast<float*>(smem + a.off_u);   // u fp32 [BN][r + 4]
     const int ustride = a.rank + 4;
-    uint16_t* As = reinterpret_cast<uint16_t*>(smem + a.off_a);
-    uint16_t* wgs = reinterpret_cast<uint16_t*>(smem + a.off_wg);
     float* red = reinterpret_cast<float*>(smem + a.off_red);  // block exchange [4][2][32][4 NB]
     // Compensator work item of this CTA: K slice c / ec_groups, column group c % ec_groups.
     const bool has_slice = has_ec && c < a.ec_slices * a.ec_groups;
@@ -225,7 +265,6 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         }
         mbar_init(bfull, 1);
         mbar_init(bempty, RK_COMPUTE_WARPS);
-        mbar_init(ec_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -472,10 +511,10 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
 #pragma unroll
                 for (int b = 0; b < NB; ++b) {
                     const int m = 8 * b + 2 * t;
-                    st_relaxed_u64(own + m * 128 + row0, rk_tagged(fin[b][0]));
-                    st_relaxed_u64(own + (m + 1) * 128 + row0, rk_tagged(fin[b][1]));
-                    st_relaxed_u64(own + m * 128 + row0 + 8, rk_tagged(fin[b][2]));
-                    st_relaxed_u64(own + (m + 1) * 128 + row0 + 8, rk_tagged(fin[b][3]));
+                    st_cg_u64(own + m * 128 + row0, rk_tagged(fin[b][0]));
+                    st_cg_u64(own + (m + 1) * 128 + row0, rk_tagged(fin[b][1]));
+                    st_cg_u64(own + m * 128 + row0 + 8, rk_tagged(fin[b][2]));
+                    st_cg_u64(own + (m + 1) * 128 + row0 + 8, rk_tagged(fin[b][3]));
                 }
                 continue;
             }
@@ -495,15 +534,16 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                         bool ready = true;
 #pragma unroll
                         for (int k = 0; k < PB; ++k) {
-                            const int cc = base + k < c ? base + k : c - 1;
-                            const unsigned long long* pp = parts + (size_t)cc * BN * 128;
+                            const bool in = base + k < c;
+                            const unsigned long long* pp = parts + (size_t)(in ? base + k : base) * BN * 128;
+                            constexpr unsigned long long kReady = 1ull << 32;
 #pragma unroll
                             for (int b = 0; b < NB; ++b) {
                                 const int m = 8 * b + 2 * t;
-                                q[k][b][0] = ld_relaxed_u64(pp + m * 128 + row0);
-                                q[k][b][1] = ld_relaxed_u64(pp + (m + 1) * 128 + row0);
-                                q[k][b][2] = ld_relaxed_u64(pp + m * 128 + row0 + 8);
-                                q[k][b][3] = ld_relaxed_u64(pp + (m + 1) * 128 + row0 + 8);
+                                q[k][b][0] = in ? ld_cg_u64(pp + m * 128 + row0) : kReady;
+                                q[k][b][1] = in ? ld_cg_u64(pp + (m + 1) * 128 + row0) : kReady;
+                                q[k][b][2] = in ? ld_cg_u64(pp + m * 128 + row0 + 8) : kReady;
+                                q[k][b][3] = in ? ld_cg_u64(pp + (m + 1) * 128 + row0 + 8) : kReady;
 #pragma unroll
                                 for (int v = 0; v < 4; ++v) ready = ready && (q[k][b][v] >> 32) == 1ull;
                             }
@@ -527,10 +567,10 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                                 const float x = __uint_as_float((uint32_t)q[k][b][v]);
                                 p[b][v] = (base + k == c_lo) ? x : p[b][v] + x;
                             }
-                            st_relaxed_u64(pp + m * 128 + row0, 0ull);
-                            st_relaxed_u64(pp + (m + 1) * 128 + row0, 0ull);
-                            st_relaxed_u64(pp + m * 128 + row0 + 8, 0ull);
-                            st_relaxed_u64(pp + (m + 1) * 128 + row0 + 8, 0ull);
+                            st_cg_u64(pp + m * 128 + row0, 0ull);
+                            st_cg_u64(pp + (m + 1) * 128 + row0, 0ull);
+                            st_cg_u64(pp + m * 128 + row0 + 8, 0ull);
+                            st_cg_u64(pp + (m + 1) * 128 + row0 + 8, 0ull);
                         }
                     }
                 }
@@ -602,28 +642,8 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         }
     } else {
         // ---------------- compensator (warp 9) ----------------
-        // The item's rows of A (32 bytes each: its 16 columns) or of w_g, before the wait on the
-        // previous kernel (they do not depend on it).
-        const bool gate_item = ec_grp == a.rank / 16;
-        if (has_slice) {
-            if (lane == 0)
-                mbar_arrive_expect_tx(ec_bar, gate_item ? (uint32_t)(ec_rows * 2) : (uint32_t)(ec_rows * 32));
-            __syncwarp();
-            if (gate_item) {
-                if (lane == 0) bulk_load(wgs, a.wg + ec_k0, (uint32_t)(ec_rows * 2), ec_bar);
-            } else {
-                for (int i = lane; i < ec_rows; i += 32)
-                    bulk_load(As + i * 16, a.A + (ec_k0 + i) * a.rank + 16 * ec_grp, 32u, ec_bar);
-            }
-        }
-        pdl_wait_primary();
-        unsigned long long* tacc = reinterpret_cast<unsigned long long*>(a.tacc);
-        if (has_slice) {
-            if (mbar_wait_ns(ec_bar, 0, SK_WAIT_NS))
-                rk_ec_item(a, As, wgs, ec_k0, ec_rows, ec_grp, tacc);
-            else if (lane == 0)
-                sk_fail(a.err, SK_ERR_MBAR, SITE_EC_BAR, 0);
-        }
+        if (has_slice) rk_ec_item(a, ec_k0, ec_rows, ec_grp, reinterpret_cast<unsigned long long*>(a.tacc));
+        else pdl_wait_primary();
     }
     __syncthreads();
 }
@@ -662,8 +682,7 @@ bool stream_rk_configure(StreamArgs& a, int bn, int kc, bool deep) {
         if ((int64_t)a.ec_slices * a.ec_groups > a.grid) return false;
         b_bytes = 2 * a.rank * 128;
         u_bytes = rk_align(bn * (a.rank + 4) * 4, 128);
-        a_bytes = rk_align(a.ec_kr * 32, 128);
-        wg_bytes = rk_align(a.ec_kr * 2, 128);
+        a_bytes = wg_bytes = 0;               // the compensator's warp reads A and w_g into registers
     }
     const int red_bytes = kc == 256 ? 4 * 2 * 32 * 4 * (bn / 8) * 4 : 0;
     const int bar_bytes = 8 * (2 * 16 + 5) + 16;
