@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--workload", default="decode-qo", choices=sorted(WORKLOADS) + sorted(SWEEP_ONLY))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the secondary prefill measurement")
+    ap.add_argument("--no-detail", action="store_true",
+                    help="skip the secondary decode-mlp and 16-layer model figures of the default run")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--sweep", action="store_true",
                     help="time every valid decode tiling for the workload's batches and print a table")
@@ -62,6 +64,8 @@ def parse():
     ap.add_argument("--once", type=int, default=0, metavar="M",
                     help="run 5 layer calls of the workload with M tokens and exit (for profilers)")
     ap.add_argument("--no-ec", action="store_true", help="with --once: the plain W4 layer")
+    ap.add_argument("--linear", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="with --once --workload sweep-1b: which linear of the model's layer 0")
     ap.add_argument("--plan", default="", metavar="KERNEL,TILE_N,TILE_M,SPLIT_K,FLAGS",
                     help="with --once: this plan (checked by spear_plan_update) instead of the planner's")
     ap.add_argument("--model-sweep", action="store_true",
@@ -258,16 +262,27 @@ def run_ours(args, rank, world, torch, dist):
     dev = torch.device("cuda")
     xs = {M: torch.from_numpy(L.x(M).view(np.int16)).to(dev).view(torch.bfloat16) for M in batches}
     ys = {M: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for M in batches}
-    plans = {M: spear.spear_gemm_plan(M, N, K, r) for M in batches}
-    ws = spear.alloc_workspace(max(p.workspace_bytes for p in plans.values()))
+    # Both code orders at hand (the tile order is made once, like the packing): each batch size is
+    # planned on the order measured faster for it.
+    tileable = kind == "decode" and N % 128 == 0 and K % 128 == 0
+    tiled = [spear.spear_tile_w4(p) for (p, *_) in sets] if tileable else None
+    fmts = spear.SPEAR_W4_ROWS | (spear.SPEAR_W4_TILES if tileable else 0)
+    plans = {M: spear.spear_gemm_plan_formats(M, N, K, r, fmts) for M in batches}
+    plans_no_ec = {M: spear.spear_gemm_plan_formats(M, N, K, 0, fmts) for M in batches}
+    ws = spear.alloc_workspace(max(p.workspace_bytes for p in list(plans.values()) + list(plans_no_ec.values())))
     stream = torch.cuda.Stream()
     calls_per_step = len(batches)
 
+    def codes(i, plan):
+        return tiled[i] if plan.flags & spear.SPEAR_PLAN_W4_TILES else sets[i][0]
+
     def step_calls(step_idx, use_ec=True):
         for j, M in enumerate(batches):
-            p, s, z, A, B, wg = sets[(step_idx * calls_per_step + j) % copies]
+            i = (step_idx * calls_per_step + j) % copies
+            p, s, z, A, B, wg = sets[i]
             ec = spear.EC(A, B, wg, L.b_g) if use_ec else None
-            spear.spear_w4ec_gemm(xs[M], p, s, z, ec, y=ys[M], workspace=ws, plan=plans[M], stream=stream)
+            spear.spear_w4ec_gemm(xs[M], codes(i, plans[M]), s, z, ec, y=ys[M], workspace=ws, plan=plans[M],
+                                  stream=stream)
 
     def graph_of(n_steps, use_ec=True, only_M=None):
         g = torch.cuda.CUDAGraph()
@@ -282,8 +297,9 @@ def run_ours(args, rank, world, torch, dist):
                     else:
                         p, s, z, A, B, wg = sets[i % copies]
                         ec = spear.EC(A, B, wg, L.b_g) if use_ec else None
-                        spear.spear_w4ec_gemm(xs[only_M], p, s, z, ec, y=ys[only_M], workspace=ws,
-                                              plan=plans[only_M], stream=stream)
+                        pl = plans[only_M] if use_ec else plans_no_ec[only_M]
+                        spear.spear_w4ec_gemm(xs[only_M], codes(i % copies, pl), s, z, ec, y=ys[only_M],
+                                              workspace=ws, plan=pl, stream=stream)
         return g
 
     def time_graph(g, reps=1):
@@ -347,8 +363,10 @@ def run_ours(args, rank, world, torch, dist):
         per_m[M] = {"us": t_on * 1e6, "us_no_ec": t_off * 1e6, "GBps": b_on / t_on / 1e9,
                     "GBps_no_ec": b_off / t_off / 1e9, "TFLOPs": layer_flops(M, N, K, r) / t_on / 1e12,
                     "ec_overhead": t_on / t_off - 1.0, "ec_byte_floor": b_on / b_off - 1.0,
-                    "plan": {"kernel": plans[M].kernel_id, "tile_n": plans[M].tile_n,
-                             "split_k": plans[M].split_k, "tile_m": plans[M].tile_m}}
+                    "plan": {"kernel": kernel_name(spear, plans[M]), "tile_n": plans[M].tile_n,
+                             "split_k": plans[M].split_k, "tile_m": plans[M].tile_m, "flags": plans[M].flags},
+                    "plan_no_ec": {"kernel": kernel_name(spear, plans_no_ec[M]), "split_k": plans_no_ec[M].split_k,
+                                   "tile_m": plans_no_ec[M].tile_m, "flags": plans_no_ec[M].flags}}
         del g_on, g_off
 
     # e2e through the public API with pinned host buffers: a step's activations travel in one
@@ -368,7 +386,8 @@ def run_ours(args, rank, world, torch, dist):
     e2e_steps = max(3, min(args.steps, 20))
 
     # The public API a serving loop uses: each weight set bound once as a W4ECLayer.
-    e2e_layers = [spear.W4ECLayer(p, s, z, spear.EC(A, B, wg, L.b_g)) for (p, s, z, A, B, wg) in sets]
+    e2e_layers = [spear.W4ECLayer(p, s, z, spear.EC(A, B, wg, L.b_g), tiled=tiled[i] if tiled else None)
+                  for i, (p, s, z, A, B, wg) in enumerate(sets)]
     for lay in e2e_layers:
         for M in batches:
             lay.plan(M)
@@ -415,7 +434,7 @@ def run_ours(args, rank, world, torch, dist):
                                                         args.workload == "decode-qo" and Mr == 16) else None
         rl = {"bound": "hbm", "achieved": per_m[Mr]["GBps"], "peak": hbm_peak, "unit": "GB/s",
               "frac": per_m[Mr]["GBps"] / hbm_peak, "traffic": tr["bytes_per_launch"] if tr else None,
-              "kernel": f"spear_w4ec_gemm M={Mr} (w4ec_decode_kernel: EC fused into the weight-streaming kernel)",
+              "kernel": f"spear_w4ec_gemm M={Mr} ({kernel_name(spear, plans[Mr])}, EC fused into the weight stream)",
               "peak_source": f"{peak_src} hbm_gbs (copy)", "algorithmic_bytes": layer_bytes(Mr, N, K, r)}
     else:
         metric_val = replica_throughput(step_flops * args.steps, world, t_main) / 1e12
@@ -439,7 +458,7 @@ def run_ours(args, rank, world, torch, dist):
         "e2e": {"value": e2e_val, "unit": unit,
                 "h2d_bytes_per_step": sum(2 * M * K for M in batches),
                 "d2h_bytes_per_step": sum(2 * M * N for M in batches)},
-        "gpu_launches": args.steps * sum(2 if r else 1 for _ in batches),
+        "gpu_launches": args.steps * sum(launches_per_call(spear, plans[M], M, r > 0) for M in batches),
         "roofline": rl,
         "clocks": clocks,
         "detail": {str(M): v for M, v in per_m.items()},
@@ -545,12 +564,12 @@ def _sweep_shape(torch, spear, L, batches):
                                            for split in (1, 2, 4, 8) for fl in (0, 1)]
         for fl in ((0, 1) if M >= 128 else (0,)):
             candidates += [(2, 128, 1, fl, 128)] + ([(2, 128, 1, fl, 256)] if M >= 256 else [])
-        # The stream-K kernel (kernel 3) up to 64 tokens: token tile, K codes per stage, and the ring
-        # mode (flags 2: one CTA per SM with a deep ring).
+        # The register-path stream kernel (kernel 4) up to 64 tokens: token tile (8-token tiles from
+        # M <= 8, 64 only with the deep ring), K codes per stage, and the ring mode (flags 2: one CTA
+        # per SM with a deep ring).  The tcgen05 stream kernel (kernel 3) is slower on every measured
+        # shape and is left out of the sweep.
         if M <= 64:
             bn = 16 if M <= 16 else (32 if M <= 32 else 64)
-            candidates += [(3, 128, kc, fl, bn) for kc in (128, 256) for fl in (0, 2) if K % kc == 0]
-            # The register-path stream kernel (kernel 4): 8-token tiles from M <= 8, 64 only deep.
             bn_rk = 8 if M <= 8 else bn
             # (codes in the tile order of spear_tile_w4: flag 4)
             candidates += [(4, 128, kc, fl | 4, bn_rk) for kc in (128, 256) for fl in (0, 2)
@@ -621,9 +640,15 @@ def run_once(args):
     import w4_gemm_error_channel_b200 as spear
     from synthetic import config_layers
     torch.cuda.set_device(0)
-    cfg, batches, kind = WORKLOADS[args.workload]
-    M = args.once
-    L = config_layers(cfg, M=M)[0]
+    if args.workload in SWEEP_ONLY:
+        # One linear of the 16-layer model (--linear: 0 qkv, 1 o, 2 up+gate, 3 down) of layer 0.
+        cfg = SWEEP_ONLY[args.workload][0]
+        M = args.once
+        L = config_layers(cfg, M=M, layers=(0,))[args.linear]
+    else:
+        cfg, batches, kind = WORKLOADS[args.workload]
+        M = args.once
+        L = config_layers(cfg, M=M)[0]
     packed, scale, zero = spear.spear_pack_w4(torch.from_numpy(L.W).cuda())
     bf = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
     ec = None if args.no_ec else spear.EC(bf(L.A_bits), bf(L.B_bits), bf(L.wg_bits), L.b_g)
@@ -714,7 +739,9 @@ def _sweep_model(torch, spear, Mmax):
             packed, scale, zero = spear.spear_pack_w4(W)
             del W
             ec = spear.EC(bf(L.A_bits), bf(L.B_bits), bf(L.wg_bits), L.b_g) if rank else None
-            linears.append((N, K, rank, spear.W4ECLayer(packed, scale, zero, ec)))
+            # Both code orders at hand: the layer plans each batch size on the faster one.
+            tiled = spear.spear_tile_w4(packed) if N % 128 == 0 and K % 128 == 0 else None
+            linears.append((N, K, rank, spear.W4ECLayer(packed, scale, zero, ec, tiled=tiled)))
     xs = {K: bf(make_layer(f"x{K}", 1004 + K, Mmax, 128, K, 0, outlier_frac=0.01, outlier_scale=20.0).x_bits)
           for K in sorted({K for (_, K, _, _) in linears})}
     ys = {N: torch.empty((Mmax, N), dtype=torch.bfloat16, device=dev) for N in sorted({N for (N, _, _, _) in linears})}
@@ -788,15 +815,33 @@ def slo_check(args):
                                     "in_model_table": lut, "picks": rows}}))
 
 
-def model_sweep(args):
+def kernel_name(spear, p):
+    if p.kernel_id == spear.SPEAR_KERNEL_TC05:
+        return "tcgen05"
+    if p.kernel_id == spear.SPEAR_KERNEL_STREAM_RK:
+        return "stream-K register path (tile order)"
+    if p.kernel_id == spear.SPEAR_KERNEL_STREAM:
+        return "stream-K tcgen05"
+    return "split-K decode"
+
+
+def launches_per_call(spear, p, M, has_ec):
+    """This library's kernel launches for one spear_w4ec_gemm call with plan p."""
+    sep = has_ec and p.flags & spear.SPEAR_PLAN_SEPARATE_EC
+    if p.kernel_id == spear.SPEAR_KERNEL_TC05:
+        return 3 if sep else 1                        # semi-fused: EC tiles, main tiles, u B add
+    if p.kernel_id == spear.SPEAR_KERNEL_SPLITK:
+        chunks = (M + 255) // 256                     # launches of at most 256 tokens
+        return chunks * (2 if sep else 1)
+    return 1                                          # the stream-K kernels
+
+
+def model_pass_rows(torch, spear, batches=(1, 16, 256, 4096)):
     """Config 4: one pass over the 64 linears of the 16-layer model (qkv, o, up+gate, down per
-    layer; compensators of rank 32 on layers 0, 1, 7, 15) for M in {1, 16, 256, 4096}, each call
-    planned by spear_gemm_plan.  Weights are distinct per linear (512 MiB of W4 in all, > 2x L2);
-    each linear reads a synthetic x of its K.  Timed as a CUDA graph of the whole pass."""
-    import torch
-    import w4_gemm_error_channel_b200 as spear
-    torch.cuda.set_device(0)
-    batches = [1, 16, 256, 4096]
+    layer; compensators of rank 32 on layers 0, 1, 7, 15) per M, each call planned by the layer
+    (spear_gemm_plan_formats over both code orders).  Weights are distinct per linear (512 MiB of
+    W4 in each order, > 2x L2); each linear reads a synthetic x of its K.  Timed as a CUDA graph of
+    the whole pass."""
     Mmax = max(batches)
     linears, xs, ys = _sweep_model(torch, spear, Mmax)
     peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
@@ -808,8 +853,7 @@ def model_sweep(args):
     for M in batches:
         kinds = {}
         for (N, K, rank, lay) in linears:
-            p = lay.plan(M)
-            key = "tcgen05" if p.kernel_id == spear.SPEAR_KERNEL_TC05 else "split-K decode"
+            key = kernel_name(spear, lay.plan(M))
             kinds[key] = kinds.get(key, 0) + 1
 
         def one_pass():
@@ -842,10 +886,57 @@ def model_sweep(args):
         rows.append({"M": M, "us_per_pass": t * 1e6, "GBps": byts / t / 1e9, "TFLOPs": flops / t / 1e12,
                      "roofline_frac": bound / t, "bound": "hbm" if byts / (hbm * 1e9) >= flops / (tc * 1e12) else "tensor",
                      "kernels": kinds, "device_status": status})
-    print(json.dumps({"model_sweep": {"workload": "16 layers x (qkv 6144x2048, o 2048x2048, up 16384x2048, "
-                                                  "down 2048x8192), EC r=32 on layers 0, 1, 7, 15, synthetic",
-                                      "peaks": {"hbm_gbs": hbm, "bf16_tflops": tc, "note": "sustained bf16 peak"},
-                                      "passes": rows}}))
+    del linears, xs, ys
+    torch.cuda.empty_cache()
+    return {"workload": "16 layers x (qkv 6144x2048, o 2048x2048, up 16384x2048, down 2048x8192), EC r=32 on "
+                        "layers 0, 1, 7, 15, synthetic",
+            "peaks": {"hbm_gbs": hbm, "bf16_tflops": tc, "note": "sustained bf16 peak"}, "passes": rows}
+
+
+def model_sweep(args):
+    """The 16-layer model pass for M in {1, 16, 256, 4096} (model_pass_rows), printed alone."""
+    import torch
+    import w4_gemm_error_channel_b200 as spear
+    torch.cuda.set_device(0)
+    print(json.dumps({"model_sweep": model_pass_rows(torch, spear)}))
+
+
+def layer_detail(torch, spear, workload, batches):
+    """Per batch size M of one workload layer: device time per call with and without the
+    compensator (64 chained calls in a CUDA graph, weights rotating over copies larger than 2x
+    L2), GB/s of algorithmic bytes, and the plan the layer chose over both code orders."""
+    from synthetic import config_layers
+    cfg = WORKLOADS[workload][0]
+    L = config_layers(cfg, M=max(batches))[0]
+    N, K, r = L.N, L.K, L.rank
+    copies = max(2, int(np.ceil(2 * L2_BYTES / layer_bytes(max(batches), N, K, r))) + 1)
+    sets = make_device_layer(torch, spear, L, copies)
+    tiled = [spear.spear_tile_w4(p) for (p, *_) in sets]
+    dev = torch.device("cuda")
+    stream = torch.cuda.Stream()
+    out = {}
+    for M in batches:
+        x = torch.from_numpy(L.x(M).view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        row = {}
+        for use_ec in (True, False):
+            lays = [spear.W4ECLayer(p, sc, z, spear.EC(A, B, wg, L.b_g) if use_ec else None, tiled=t)
+                    for (p, sc, z, A, B, wg), t in zip(sets, tiled)]
+            plan = lays[0].plan(M)
+            calls = [(lambda lay=lays[i % copies]: lay(x, y=y, stream=stream)) for i in range(64)]
+            t = _time_calls(torch, stream, calls, 3) / 64
+            rr = r if use_ec else 0
+            key = "" if use_ec else "_no_ec"
+            row["us" + key] = t * 1e6
+            row["GBps" + key] = layer_bytes(M, N, K, rr) / t / 1e9
+            row["plan" + key] = {"kernel": kernel_name(spear, plan), "tile_n": plan.tile_n, "tile_m": plan.tile_m,
+                                 "split_k": plan.split_k, "flags": plan.flags}
+            row["device_status" + key] = spear.spear_get_device_status(lays[0].workspace)
+        row["ec_overhead"] = row["us"] / row["us_no_ec"] - 1.0
+        out[str(M)] = row
+    del sets, tiled
+    torch.cuda.empty_cache()
+    return {"workload": f"{workload}: N={N}, K={K}, EC rank {r}", "per_M": out}
 
 
 def grouped_compare(args):
@@ -1038,6 +1129,18 @@ def main():
     else:
         torch.cuda.set_device(0)
     out = run_ours(args, rank, world, torch, dist)
+    if world == 1 and args.workload == "decode-qo" and not args.no_detail:
+        # Secondary per-shape figures (one GPU only): the decode-mlp layer at M in {1, 8, 32, 64}
+        # and one pass of the 16-layer model at M in {1, 16, 256, 4096}.
+        import w4_gemm_error_channel_b200 as spear
+        try:
+            out["detail_decode_mlp"] = layer_detail(torch, spear, "decode-mlp", [1, 8, 32, 64])
+        except Exception as e:
+            out["detail_decode_mlp"] = {"error": str(e)}
+        try:
+            out["detail_model_pass"] = model_pass_rows(torch, spear)
+        except Exception as e:
+            out["detail_model_pass"] = {"error": str(e)}
     if rank == 0 and not args.no_prefill and args.workload != "prefill":
         import w4_gemm_error_channel_b200 as spear
         try:

@@ -209,6 +209,19 @@ SPEAR_API spear_status spear_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t 
 SPEAR_API spear_status spear_gemm_plan_tiled(int64_t M, int64_t N, int64_t K, int32_t rank, int device,
                                    spear_plan* out);
 
+/* Code orders a caller holds, for spear_gemm_plan_formats. */
+enum { SPEAR_W4_ROWS = 1, SPEAR_W4_TILES = 2 };
+
+/*
+ * spear_gemm_plan_formats -- as spear_gemm_plan, choosing among the code orders the caller holds
+ * (SPEAR_W4_ROWS: spear_pack_w4's; SPEAR_W4_TILES: spear_tile_w4's; either or both).  With both,
+ * the plan reads the tile order (flags include SPEAR_PLAN_W4_TILES) when the measured latency
+ * table has that order faster for this shape, and the row order otherwise.  The caller passes
+ * the matching codes to spear_w4ec_gemm.  SPEAR_ERR_INVALID_ARG for an empty or unknown set.
+ */
+SPEAR_API spear_status spear_gemm_plan_formats(int64_t M, int64_t N, int64_t K, int32_t rank, int device,
+                                     int32_t formats, spear_plan* out);
+
 /*
  * spear_plan_update -- check a plan whose fields the caller has changed (kernel, tiling, flags)
  * for this shape and recompute plan->workspace_bytes in place.  The semi-fused prefill path

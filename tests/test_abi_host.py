@@ -293,3 +293,21 @@ def test_tiled_plan_and_tile_order_argument_checks():
     assert tile(ctypes.c_void_p(4096), 128, 192, ctypes.c_void_p(1 << 20), None) == SHAPE
     assert tile(ctypes.c_void_p(4104), 128, 128, ctypes.c_void_p(1 << 20), None) == MISALIGNED
     assert tile(ctypes.c_void_p(4096), 128, 128, ctypes.c_void_p(4096 + 16), None) == INVALID   # overlap
+
+
+def test_plan_formats_picks_among_code_orders():
+    p = spear.spear_plan()
+    f = spear._lib.spear_gemm_plan_formats
+    assert f(4, 4096, 4096, 64, -1, 0, ctypes.byref(p)) == INVALID
+    assert f(4, 4096, 4096, 64, -1, 8, ctypes.byref(p)) == INVALID
+    st, rows = _plan(4, 4096, 4096, 64)
+    assert f(4, 4096, 4096, 64, -1, spear.SPEAR_W4_ROWS, ctypes.byref(p)) == OK
+    assert (p.kernel_id, p.tile_n, p.split_k, p.tile_m, p.flags) == (rows.kernel_id, rows.tile_n, rows.split_k,
+                                                                     rows.tile_m, rows.flags)
+    assert f(4, 4096, 4096, 64, -1, spear.SPEAR_W4_TILES, ctypes.byref(p)) == OK
+    assert p.kernel_id == spear.SPEAR_KERNEL_STREAM_RK and p.flags & spear.SPEAR_PLAN_W4_TILES
+    for M, N, K in ((1, 22016, 4096), (16, 4096, 4096), (64, 22016, 4096), (2048, 4096, 14336)):
+        assert f(M, N, K, 64, -1, spear.SPEAR_W4_ROWS | spear.SPEAR_W4_TILES, ctypes.byref(p)) == OK
+        # The plan's flag names the order it reads; only the register path reads tiles.
+        assert bool(p.flags & spear.SPEAR_PLAN_W4_TILES) == (p.kernel_id == spear.SPEAR_KERNEL_STREAM_RK)
+        assert spear._lib.spear_plan_update(ctypes.byref(p), M, N, K, 64) == OK

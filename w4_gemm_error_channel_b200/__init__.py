@@ -23,10 +23,12 @@ SPEAR_OK = 0
 SPEAR_BF16, SPEAR_FP32 = 0, 1
 SPEAR_KERNEL_AUTO, SPEAR_KERNEL_SPLITK, SPEAR_KERNEL_TC05, SPEAR_KERNEL_STREAM, SPEAR_KERNEL_STREAM_RK = 0, 1, 2, 3, 4
 SPEAR_PLAN_SEPARATE_EC, SPEAR_PLAN_DEEP_RING, SPEAR_PLAN_W4_TILES = 1, 2, 4
+SPEAR_W4_ROWS, SPEAR_W4_TILES = 1, 2
 STATUS_NAMES = {0: "SPEAR_OK", 1: "SPEAR_ERR_INVALID_ARG", 2: "SPEAR_ERR_UNSUPPORTED_SHAPE",
                 3: "SPEAR_ERR_MISALIGNED", 4: "SPEAR_ERR_WORKSPACE_TOO_SMALL", 5: "SPEAR_ERR_CUDA",
                 6: "SPEAR_ERR_TIMEOUT"}
 EXPORTED = ["spear_pack_w4", "spear_debug_unpack_w4", "spear_tile_w4", "spear_gemm_plan", "spear_gemm_plan_tiled",
+            "spear_gemm_plan_formats",
             "spear_plan_update", "spear_w4ec_gemm",
             "spear_w4ec_gemm_noalloc", "spear_noalloc_get_device_status", "spear_get_device_status", "spear_status_string", "spear_version",
             "spear_latency_table", "spear_predict_step_us", "spear_pick_prefill_chunk",
@@ -76,6 +78,8 @@ def _load():
     lib.spear_tile_w4.argtypes = [P, I64, I64, P, P]
     lib.spear_gemm_plan.argtypes = [I64, I64, I64, ctypes.c_int32, ctypes.c_int, ctypes.POINTER(spear_plan)]
     lib.spear_gemm_plan_tiled.argtypes = [I64, I64, I64, ctypes.c_int32, ctypes.c_int, ctypes.POINTER(spear_plan)]
+    lib.spear_gemm_plan_formats.argtypes = [I64, I64, I64, ctypes.c_int32, ctypes.c_int, ctypes.c_int32,
+                                            ctypes.POINTER(spear_plan)]
     lib.spear_plan_update.argtypes = [ctypes.POINTER(spear_plan), I64, I64, I64, ctypes.c_int32]
     lib.spear_w4ec_gemm.argtypes = [ctypes.POINTER(spear_plan), P, I64, I64, I64, P, P, P,
                                     ctypes.POINTER(spear_ec), P, ctypes.c_int, P, ctypes.c_size_t, P]
@@ -222,6 +226,15 @@ def spear_gemm_plan_tiled(M: int, N: int, K: int, rank: int = 0, device: int = -
     """Plan for codes in spear_tile_w4's tile order (the register-path stream kernel, M <= 64)."""
     plan = spear_plan()
     _check("spear_gemm_plan_tiled", _lib.spear_gemm_plan_tiled(M, N, K, rank, device, ctypes.byref(plan)))
+    return plan
+
+
+def spear_gemm_plan_formats(M: int, N: int, K: int, rank: int = 0, formats: int = SPEAR_W4_ROWS | SPEAR_W4_TILES,
+                            device: int = -1) -> spear_plan:
+    """Plan among the code orders held (SPEAR_W4_ROWS, SPEAR_W4_TILES): the tile order where it was
+    measured faster for this shape."""
+    plan = spear_plan()
+    _check("spear_gemm_plan_formats", _lib.spear_gemm_plan_formats(M, N, K, rank, device, formats, ctypes.byref(plan)))
     return plan
 
 
@@ -402,26 +415,36 @@ class W4ECLayer:
     """
 
     def __init__(self, packed: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor, ec: Optional[EC] = None,
-                 y_dtype=torch.bfloat16):
+                 y_dtype=torch.bfloat16, tiled: Optional[torch.Tensor] = None):
         for name, t in (("packed", packed), ("scale", scale), ("zero", zero)):
             _dev(t, name)
+        if tiled is not None:
+            _dev(tiled, "tiled")
+            if tiled.numel() != packed.numel():
+                raise ValueError("tiled must hold the same codes as packed (spear_tile_w4(packed))")
         self.N, self.K = int(packed.shape[0]), int(packed.shape[1]) * 2
         self.device = packed.device
         self._index = packed.get_device()
         self.y_dtype = y_dtype
         self._yd = SPEAR_FP32 if y_dtype == torch.float32 else SPEAR_BF16
         self.rank = ec.rank if ec is not None else 0
-        self._keep = (packed, scale, zero, ec)
+        self._keep = (packed, scale, zero, ec, tiled)
         self._ec_c = ec.as_c() if ec is not None else None
         self._ec_ref = ctypes.byref(self._ec_c) if ec is not None else None
         self._w = (packed.data_ptr(), scale.data_ptr(), zero.data_ptr())
+        # The tile order serves the scalar gate only.
+        self._tiled = tiled.data_ptr() if tiled is not None and (ec is None or ec.gate_w1 is None) else None
         self._plans = {}
         self._ws = None
 
     def plan(self, M: int) -> spear_plan:
         p = self._plans.get(M)
         if p is None:
-            p = spear_gemm_plan(M, self.N, self.K, self.rank, self.device.index)
+            if self._tiled is not None:
+                p = spear_gemm_plan_formats(M, self.N, self.K, self.rank, SPEAR_W4_ROWS | SPEAR_W4_TILES,
+                                            self.device.index)
+            else:
+                p = spear_gemm_plan(M, self.N, self.K, self.rank, self.device.index)
             if self._ws is None or self._ws.numel() < p.workspace_bytes:
                 self._ws = alloc_workspace(p.workspace_bytes, self.device)
             self._plans[M] = (p, ctypes.byref(p))
@@ -448,7 +471,8 @@ class W4ECLayer:
             raise ValueError("y must be a contiguous [M, N] tensor of the layer's output dtype on its device")
         sh = stream.cuda_stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
         ws = self._ws
-        st = _lib.spear_w4ec_gemm(entry[1], x.data_ptr(), M, self.N, self.K, self._w[0], self._w[1], self._w[2],
+        codes = self._tiled if entry[0].flags & SPEAR_PLAN_W4_TILES else self._w[0]
+        st = _lib.spear_w4ec_gemm(entry[1], x.data_ptr(), M, self.N, self.K, codes, self._w[1], self._w[2],
                                   self._ec_ref, y.data_ptr(), self._yd, ws.data_ptr(), ws.numel(), sh)
         if st != SPEAR_OK:
             raise SpearError("spear_w4ec_gemm", st)

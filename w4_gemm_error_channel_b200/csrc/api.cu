@@ -113,7 +113,8 @@ spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K,
 
 // tiles: only the register-path stream kernel's entries (codes in tile order); otherwise every
 // other kernel's.
-bool lookup_measured(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spear_plan* p, bool tiles = false) {
+bool lookup_measured(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spear_plan* p, bool tiles = false,
+                     double* us = nullptr) {
     const int has_ec = rank > 0 ? 1 : 0;
     const int nb = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
     const MeasuredPlan* best = nullptr;
@@ -126,6 +127,7 @@ bool lookup_measured(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spe
         if (!best || std::llabs(e.M - M) < std::llabs(best->M - M)) best = &e;
     }
     if (!best) return false;
+    if (us) *us = best->us;
     if (best->kernel_id == SPEAR_KERNEL_STREAM || best->kernel_id == SPEAR_KERNEL_STREAM_RK) {
         // The measured stage width and ring mode; the token tile must hold M.
         const int bn = (best->kernel_id == SPEAR_KERNEL_STREAM_RK && M <= 8) ? 8 : M <= 16 ? 16 : (M <= 32 ? 32 : 64);
@@ -394,6 +396,24 @@ spear_status spear_gemm_plan_tiled(int64_t M, int64_t N, int64_t K, int32_t rank
     p.workspace_bytes = workspace_bytes_for(p, M, N, K, rank, sms);
     *out = p;
     return SPEAR_OK;
+}
+
+spear_status spear_gemm_plan_formats(int64_t M, int64_t N, int64_t K, int32_t rank, int device, int32_t formats,
+                                    spear_plan* out) {
+    if (!out || formats <= 0 || (formats & ~(SPEAR_W4_ROWS | SPEAR_W4_TILES))) return SPEAR_ERR_INVALID_ARG;
+    if (!(formats & SPEAR_W4_TILES)) return spear_gemm_plan(M, N, K, rank, device, out);
+    if (!(formats & SPEAR_W4_ROWS)) return spear_gemm_plan_tiled(M, N, K, rank, device, out);
+    spear_status st = check_shape(M, N, K, rank);
+    if (st != SPEAR_OK) return st;
+    // Both orders at hand: the tile order where this shape was measured faster with it.
+    const int sms = device_sms(device);
+    const int64_t m = M > 0 ? M : 1;
+    spear_plan rows = {}, tiles = {};
+    double us_rows = 0.0, us_tiles = 0.0;
+    const bool have_rows = lookup_measured(m, N, K, rank, sms, &rows, false, &us_rows);
+    const bool have_tiles = M <= 64 && lookup_measured(m, N, K, rank, sms, &tiles, true, &us_tiles);
+    if (have_tiles && (!have_rows || us_tiles < us_rows)) return spear_gemm_plan_tiled(M, N, K, rank, device, out);
+    return spear_gemm_plan(M, N, K, rank, device, out);
 }
 
 spear_status spear_tile_w4(const void* packed, int64_t N, int64_t K, void* tiled, void* stream) {
