@@ -20,6 +20,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libspear.so")
 
 SPEAR_OK = 0
+(SPEAR_ERR_INVALID_ARG, SPEAR_ERR_UNSUPPORTED_SHAPE, SPEAR_ERR_MISALIGNED, SPEAR_ERR_WORKSPACE_TOO_SMALL,
+ SPEAR_ERR_CUDA, SPEAR_ERR_TIMEOUT) = 1, 2, 3, 4, 5, 6
 SPEAR_BF16, SPEAR_FP32 = 0, 1
 SPEAR_KERNEL_AUTO, SPEAR_KERNEL_SPLITK, SPEAR_KERNEL_TC05, SPEAR_KERNEL_STREAM, SPEAR_KERNEL_STREAM_RK = 0, 1, 2, 3, 4
 SPEAR_PLAN_SEPARATE_EC, SPEAR_PLAN_DEEP_RING, SPEAR_PLAN_W4_TILES = 1, 2, 4

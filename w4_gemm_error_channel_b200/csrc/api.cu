@@ -295,6 +295,58 @@ spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K,
     return SPEAR_OK;
 }
 
+// The split-K decode kernel over launches of at most LAUNCH_TOKENS_MAX tokens.  group > 0: scale
+// and zero [N][K / group] with K slices of k_slice codes (a multiple of 128); else per-channel.
+spear_status run_decode(const spear_plan& p, const void* x, int64_t M, int64_t N, int64_t K, const void* packed,
+                        const void* scale, const void* zero, const spear_ec* ec, void* y, spear_dtype y_dtype,
+                        unsigned char* ws, int64_t group, int64_t k_slice, cudaStream_t s) {
+    const int32_t rank = ec ? ec->rank : 0;
+    unsigned* ctrl = (unsigned*)ws;
+    const int nb = nb_for_tile_m(p.tile_m);
+    const int g = p.tile_n / 16;
+
+    DecodeArgs a;
+    a.packed = (const uint8_t*)packed;
+    a.scale = (const __half*)scale;
+    a.zero = (const __half*)zero;
+    a.A = ec ? (const uint16_t*)ec->A : nullptr;
+    a.B = ec ? (const uint16_t*)ec->B : nullptr;
+    a.wg = ec ? (const uint16_t*)ec->w_g : nullptr;
+    a.b_g = ec ? ec->b_g : 0.0f;
+    a.mlp = gate_mlp_of(ec);
+    a.rank = rank;
+    a.y_fp32 = (y_dtype == SPEAR_FP32);
+    a.N = N;
+    a.K = K;
+    a.k_slice = group > 0 ? k_slice : k_slice_for(K, p.split_k);
+    a.group = group;
+    a.split = p.split_k;
+    a.ec_jr = ec_jr_for(rank, p.split_k);
+    a.ec_splits = decode_ec_ctas_per_chunk(K, rank);
+    a.row_tiles = (int)(N / p.tile_n);
+    a.tacc = (long long*)(ws + CTRL_BYTES);
+    a.err = ctrl;
+    a.arrivals = ctrl + CTRL_HEADER_WORDS;
+    a.consumed = a.arrivals + CHUNKS_MAX;
+    a.consumed1 = a.consumed + CHUNKS_MAX;
+    const bool separate = rank > 0 && (p.flags & SPEAR_PLAN_SEPARATE_EC);
+    a.ymain = separate ? (float*)(ws + ZEROED_BYTES) : nullptr;
+    const size_t ysz = y_dtype == SPEAR_FP32 ? 4 : 2;
+    // Launches of at most LAUNCH_TOKENS_MAX tokens, in token order on one stream.
+    for (int64_t m0 = 0; m0 < M; m0 += LAUNCH_TOKENS_MAX) {
+        const int64_t ml = (M - m0) < LAUNCH_TOKENS_MAX ? (M - m0) : LAUNCH_TOKENS_MAX;
+        a.x = (const uint16_t*)x + m0 * K;
+        a.y = (unsigned char*)y + (size_t)m0 * N * ysz;
+        a.M = ml;
+        a.mchunks = (int)((ml + p.tile_m - 1) / p.tile_m);
+        const int e = a.ec_splits * a.mchunks;
+        a.ec_ctas = (e + p.split_k - 1) / p.split_k * p.split_k;
+        if (launch_decode(a, nb, g, wpw_for(a.k_slice), s) != cudaSuccess) return SPEAR_ERR_CUDA;
+        if (separate && launch_apply(a, s) != cudaSuccess) return SPEAR_ERR_CUDA;
+    }
+    return SPEAR_OK;
+}
+
 }  // namespace
 
 namespace spear {
@@ -541,48 +593,7 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         const cudaError_t e = rk ? launch_stream_rk(a, p.tile_m, s) : launch_stream(a, p.tile_m, s);
         return e == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
     }
-    const int nb = nb_for_tile_m(p.tile_m);
-    const int g = p.tile_n / 16;
-
-    DecodeArgs a;
-    a.packed = (const uint8_t*)packed;
-    a.scale = (const __half*)scale;
-    a.zero = (const __half*)zero;
-    a.A = ec ? (const uint16_t*)ec->A : nullptr;
-    a.B = ec ? (const uint16_t*)ec->B : nullptr;
-    a.wg = ec ? (const uint16_t*)ec->w_g : nullptr;
-    a.b_g = ec ? ec->b_g : 0.0f;
-    a.mlp = gate_mlp_of(ec);
-    a.rank = rank;
-    a.y_fp32 = (y_dtype == SPEAR_FP32);
-    a.N = N;
-    a.K = K;
-    a.k_slice = k_slice_for(K, p.split_k);
-    a.split = p.split_k;
-    a.ec_jr = ec_jr_for(rank, p.split_k);
-    a.ec_splits = decode_ec_ctas_per_chunk(K, rank);
-    a.row_tiles = (int)(N / p.tile_n);
-    a.tacc = (long long*)(ws + CTRL_BYTES);
-    a.err = ctrl;
-    a.arrivals = ctrl + CTRL_HEADER_WORDS;
-    a.consumed = a.arrivals + CHUNKS_MAX;
-    a.consumed1 = a.consumed + CHUNKS_MAX;
-    const bool separate = rank > 0 && (p.flags & SPEAR_PLAN_SEPARATE_EC);
-    a.ymain = separate ? (float*)(ws + ZEROED_BYTES) : nullptr;
-    const size_t ysz = y_dtype == SPEAR_FP32 ? 4 : 2;
-    // Launches of at most LAUNCH_TOKENS_MAX tokens, in token order on one stream.
-    for (int64_t m0 = 0; m0 < M; m0 += LAUNCH_TOKENS_MAX) {
-        const int64_t ml = (M - m0) < LAUNCH_TOKENS_MAX ? (M - m0) : LAUNCH_TOKENS_MAX;
-        a.x = (const uint16_t*)x + m0 * K;
-        a.y = (unsigned char*)y + (size_t)m0 * N * ysz;
-        a.M = ml;
-        a.mchunks = (int)((ml + p.tile_m - 1) / p.tile_m);
-        const int e = a.ec_splits * a.mchunks;
-        a.ec_ctas = (e + p.split_k - 1) / p.split_k * p.split_k;
-        if (launch_decode(a, nb, g, wpw_for(a.k_slice), s) != cudaSuccess) return SPEAR_ERR_CUDA;
-        if (separate && launch_apply(a, s) != cudaSuccess) return SPEAR_ERR_CUDA;
-    }
-    return SPEAR_OK;
+    return run_decode(p, x, M, N, K, packed, scale, zero, ec, y, y_dtype, ws, 0, 0, s);
 }
 
 spear_status spear_pack_w4_grouped(const void* W, spear_dtype w_dtype, int64_t N, int64_t K, int64_t group,
@@ -648,6 +659,24 @@ spear_status spear_w4ec_gemm_grouped(const void* x, int64_t M, int64_t N, int64_
     ga.y = y;
     ga.y_fp32 = (y_dtype == SPEAR_FP32);
     ga.ymain = nullptr;
+    // Decode batches: the fused decode kernel with the group scale applied per 128-code window,
+    // its K slices rounded to whole windows; otherwise the grouped kernel (below).
+    if (M <= LAUNCH_TOKENS_MAX) {
+        spear_plan p;
+        const int sms = device_sms(-1);
+        if (!lookup_measured(M, N, K, rank > 0 ? 1 : 0, sms, &p) || p.kernel_id != SPEAR_KERNEL_SPLITK)
+            st = plan_decode(M, N, K, rank, sms, &p);
+        if (st == SPEAR_OK && p.kernel_id == SPEAR_KERNEL_SPLITK) {
+            p.flags = 0;
+            for (; p.split_k >= 1; p.split_k /= 2) {
+                const int64_t ksl = (K + p.split_k - 1) / p.split_k;
+                const int64_t k_slice = (ksl + 127) / 128 * 128;
+                if ((p.split_k - 1) * k_slice >= K) continue;
+                if (!decode_config_supported(nb_for_tile_m(p.tile_m), p.tile_n / 16, wpw_for(k_slice))) continue;
+                return run_decode(p, x, M, N, K, packed, scale, zero, ec, y, y_dtype, ws, group, k_slice, s);
+            }
+        }
+    }
     if (rank == 0) return launch_w4g_gemm(ga, s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
 
     // The compensator beside the grouped GEMM, as on the semi-fused prefill path.

@@ -235,7 +235,11 @@ SPEAR_DEVI void st_dsmem_f4(float4* local, unsigned rank, float4 v) {
 // ---------------------------------------------------------------------------------------------
 // GEMM role.
 // ---------------------------------------------------------------------------------------------
-template <int NB, int G, int WPW>
+// GROUPED: scale and zero-point per (row, group of a.group codes), a.group a multiple of 128 and
+// every K slice a multiple of 128, so that each 128-code window lies inside one group: the window's
+// products are scaled by s[n, group] as they are added to the accumulators, and the epilogue's
+// per-row scale is 1.
+template <int NB, int G, int WPW, bool GROUPED>
 SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsigned char* dyn) {
     constexpr int RT = 16 * G;        // weight rows per CTA
     constexpr int TM = 8 * NB;        // tokens per CTA
@@ -276,13 +280,16 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    for (int i = threadIdx.x; i < RT; i += DK_THREADS) s_scale[i] = __half2float(a.scale[n0 + i]);
+    for (int i = threadIdx.x; i < RT; i += DK_THREADS) s_scale[i] = GROUPED ? 1.0f : __half2float(a.scale[n0 + i]);
     uint32_t zb[G][2];
+    if (!GROUPED) {
 #pragma unroll
-    for (int i = 0; i < G; ++i)
+        for (int i = 0; i < G; ++i)
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-            zb[i][h] = zero_bias_bf16x2((uint32_t)__half2float(a.zero[n0 + 16 * i + g + 8 * h]));
+            for (int h = 0; h < 2; ++h)
+                zb[i][h] = zero_bias_bf16x2((uint32_t)__half2float(a.zero[n0 + 16 * i + g + 8 * h]));
+    }
+    const int64_t ngroups = GROUPED ? a.K / a.group : 1;
     // Unconditional loads (a lane past the slice end re-reads the slice start) keep every request
     // in flight before the wait below; such lanes feed zero activations instead.
     uint4 wq[WPW][G][2];
@@ -311,6 +318,20 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
     for (int w8 = 0; w8 < WPW; ++w8) {
         const int64_t kt = kbeg + (int64_t)(warp + DK_WARPS * w8) * DK_WIN + 32 * t;
         const bool active = kt < kend;
+        float sc[G][2];
+        if (GROUPED) {
+            // The window's group (clamped for lanes past the slice end, whose x is zero).
+            const int64_t kw = kbeg + (int64_t)(warp + DK_WARPS * w8) * DK_WIN;
+            const int64_t grp = imin64(kw / a.group, ngroups - 1);
+#pragma unroll
+            for (int i = 0; i < G; ++i)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int64_t o = (n0 + 16 * i + g + 8 * h) * ngroups + grp;
+                    zb[i][h] = zero_bias_bf16x2((uint32_t)__half2float(a.zero[o]));
+                    sc[i][h] = __half2float(a.scale[o]);
+                }
+        }
         // Activations: for word w (codes k..k+7) the B operand pairs are (x_i, x_{i+4}).
         uint32_t xb[NB][4][4];
 #pragma unroll
@@ -331,6 +352,11 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
         for (int i = 0; i < G; ++i) {
             const uint32_t wa[4] = {wq[w8][i][0].x, wq[w8][i][0].y, wq[w8][i][0].z, wq[w8][i][0].w};
             const uint32_t wb[4] = {wq[w8][i][1].x, wq[w8][i][1].y, wq[w8][i][1].z, wq[w8][i][1].w};
+            float part[NB][4];                 // GROUPED: this window's products, scaled below
+            if (GROUPED) {
+#pragma unroll
+                for (int b = 0; b < NB; ++b) part[b][0] = part[b][1] = part[b][2] = part[b][3] = 0.0f;
+            }
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
                 uint32_t ra[4], rb[4];
@@ -341,7 +367,17 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
                     const uint32_t af[4] = {ra[2 * hh], rb[2 * hh], ra[2 * hh + 1], rb[2 * hh + 1]};
 #pragma unroll
                     for (int b = 0; b < NB; ++b)
-                        mma_bf16_16816(acc[i][b], af, xb[b][w][2 * hh], xb[b][w][2 * hh + 1]);
+                        mma_bf16_16816(GROUPED ? part[b] : acc[i][b], af, xb[b][w][2 * hh], xb[b][w][2 * hh + 1]);
+                }
+            }
+            if (GROUPED) {
+                // [0], [1]: row g (tokens 2t, 2t + 1); [2], [3]: row g + 8.
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    acc[i][b][0] = fmaf(sc[i][0], part[b][0], acc[i][b][0]);
+                    acc[i][b][1] = fmaf(sc[i][0], part[b][1], acc[i][b][1]);
+                    acc[i][b][2] = fmaf(sc[i][1], part[b][2], acc[i][b][2]);
+                    acc[i][b][3] = fmaf(sc[i][1], part[b][3], acc[i][b][3]);
                 }
             }
         }
@@ -659,7 +695,7 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
     retire_accumulators();
 }
 
-template <int NB, int G, int WPW>
+template <int NB, int G, int WPW, bool GROUPED>
 __global__ void __launch_bounds__(DK_THREADS, 4) w4ec_decode_kernel(DecodeArgs a) {
     extern __shared__ __align__(16) unsigned char dyn_smem[];
     int bid = blockIdx.x;
@@ -671,7 +707,7 @@ __global__ void __launch_bounds__(DK_THREADS, 4) w4ec_decode_kernel(DecodeArgs a
     bid -= a.ec_ctas;
     const int ks = bid % a.split;          // = the rank within the cluster
     const int rest = bid / a.split;
-    gemm_role<NB, G, WPW>(a, rest % a.row_tiles, ks, rest / a.row_tiles, dyn_smem);
+    gemm_role<NB, G, WPW, GROUPED>(a, rest % a.row_tiles, ks, rest / a.row_tiles, dyn_smem);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -831,7 +867,7 @@ bool decode_config_supported(int nb, int g, int wpw) {
     return false;
 }
 
-template <int NB, int G, int WPW>
+template <int NB, int G, int WPW, bool GROUPED>
 static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     static_assert(WPW * G <= 8, "weight registers");
     const unsigned grid = (unsigned)(a.ec_ctas + a.row_tiles * a.split * a.mchunks);
@@ -839,7 +875,7 @@ static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     // Static plus dynamic shared memory above 48 KB needs the opt-in attribute (once per device).
     static std::mutex mu;
     static size_t opted[kMaxDevices] = {0};
-    cudaError_t oe = opt_in_smem_at_least((const void*)w4ec_decode_kernel<NB, G, WPW>, dyn, mu, opted);
+    cudaError_t oe = opt_in_smem_at_least((const void*)w4ec_decode_kernel<NB, G, WPW, GROUPED>, dyn, mu, opted);
     if (oe != cudaSuccess) return oe;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -855,12 +891,13 @@ static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.split > 1 ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, w4ec_decode_kernel<NB, G, WPW>, a);
+    return cudaLaunchKernelEx(&cfg, w4ec_decode_kernel<NB, G, WPW, GROUPED>, a);
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, int nb, int g, int wpw, cudaStream_t stream) {
 #define SPEAR_DK_CASE(NB_, G_, W_) \
-    if (nb == NB_ && g == G_ && wpw == W_) return launch_t<NB_, G_, W_>(a, stream);
+    if (nb == NB_ && g == G_ && wpw == W_)                                                          \
+        return a.group > 0 ? launch_t<NB_, G_, W_, true>(a, stream) : launch_t<NB_, G_, W_, false>(a, stream);
 #define SPEAR_DK_NB(NB_)                                                                              \
     SPEAR_DK_CASE(NB_, 1, 1) SPEAR_DK_CASE(NB_, 1, 2) SPEAR_DK_CASE(NB_, 1, 4) SPEAR_DK_CASE(NB_, 1, 8) \
     SPEAR_DK_CASE(NB_, 2, 1) SPEAR_DK_CASE(NB_, 2, 2) SPEAR_DK_CASE(NB_, 2, 4)                          \

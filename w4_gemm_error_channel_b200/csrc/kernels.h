@@ -99,6 +99,8 @@ struct DecodeArgs {
     unsigned* consumed1;    // [mchunks][GROUPS_MAX] level-1 consumer counters
     float* ymain;           // separate EC pass: fp32 main term [M][N] (workspace); null when fused
     GateMlp mlp;            // bottleneck-MLP gate (w1 == null: the scalar gate)
+    int64_t group;          // 0: per-channel scale/zero [N]; else group-wise [N][K / group], group a
+                            // multiple of 128 and k_slice a multiple of 128
 };
 
 // Prefill (tcgen05) kernel arguments.

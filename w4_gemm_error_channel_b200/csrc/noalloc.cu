@@ -130,6 +130,7 @@ extern "C" spear_status spear_w4ec_gemm_noalloc(const spear_plan* plan, const vo
     a.consumed1 = a.consumed + CHUNKS_MAX;
     a.ymain = nullptr;                                    // the compensator stays fused here
     a.mlp = GateMlp{};                                    // the scalar gate
+    a.group = 0;                                          // per-channel scales
     return launch_decode(a, nb, p.tile_n / 16, wpw_of(ksl), s) == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
 }
 

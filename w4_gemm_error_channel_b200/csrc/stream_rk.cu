@@ -29,11 +29,10 @@
 //               order).  Lane (g, t) holds 32 codes of rows g and g + 8 per row group.  Then the
 //               segment's epilogue: partial sum out, or finalisation with the lower CTAs' partial
 //               sums, the compensator term E[n, m] = sum_j B[j, n] u[m, j] on mma.sync (B from
-//               shared memory by ldmatrix.trans, u split into bf16 hi + lo), y = s[n] D + E.  In a
-//               CTA that finalises a tile they read the accumulators and form u (fp32) together at
-//               its first finalisation.
+//               shared memory by ldmatrix.trans, u split into bf16 hi + lo), y = s[n] D + E.
 //   warp 9      the compensator's work item: one 16-column group of x A (or x w_g) over one K
-//               slice, A fragments loaded straight into registers.
+//               slice, A fragments loaded straight into registers; then, in a CTA that finalises
+//               a tile, u for every token (off the compute warps' path).
 // Every wait is bounded in time; on timeout a bit of the error word is set and the site recorded.
 #include "kernels.h"
 #include "stream_common.cuh"
@@ -70,21 +69,20 @@ SPEAR_DEVI bool rk_wait(uint64_t* bar, uint32_t parity) {
     return mbar_try(bar, parity) || mbar_wait_ns(bar, parity, SK_WAIT_NS);
 }
 
-// u for every token of the tile, by the 256 compute threads: warp w takes tokens w, w + 8, ...,
-// lane l the accumulator words l, l + 32, ... of a token (t, then the gate pre-activation in word
-// r).  A token's words are read together, TB tokens at a time, until every word holds all
-// slices (bounded); then u[m][j] = sigmoid(p[m] + b_g) t[m][j] (fp32, zero past M) goes to
-// ubuf [rows][ustride].  The caller synchronises the compute warps afterwards.
+// u for every token of the tile, by one warp: token pairs (2p, 2p + 1) for p = first, first + step,
+// ...; lane l reads the accumulator words l, l + 32, ... of both tokens (t, then the gate
+// pre-activation in word r), all at once, until every word holds all slices (bounded); then
+// u[m][j] = sigmoid(p[m] + b_g) t[m][j] (fp32, zero past M) goes to ubuf [rows][ustride].
 SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc, float* ubuf, int ustride, int rows,
-                             int cw, int lane) {
+                             int first, int step, int lane) {
     constexpr int WMAX = 5;                              // words per lane and token: r + 1 <= 160
     const int r = a.rank;
     const int nw = (r + 1 + 31) / 32;
     const int gi = r / 32, gl = r % 32;                  // the gate word: chunk gi of lane gl
     const unsigned long long want = (unsigned long long)a.ec_slices;
-    for (int m0 = cw; m0 < rows; m0 += 16) {
-        // Tokens m0 and m0 + 8, all their words in flight together.
-        const int m1 = m0 + 8;
+    for (int m0 = 2 * first; m0 < rows; m0 += 2 * step) {
+        // Tokens m0 and m0 + 1, all their words in flight together.
+        const int m1 = m0 + 1;
         unsigned long long v0[WMAX], v1[WMAX];
         const uint64_t t0 = globaltimer_ns();
         for (;;) {
@@ -239,6 +237,7 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     uint64_t* empty = full + NST;                                         // stage consumed (8 warps)
     uint64_t* bfull = empty + NST;                                        // B slice landed
     uint64_t* bempty = bfull + 1;                                         // B slice consumed (8 warps)
+    uint64_t* u_ready = bempty + 1;                                       // u in shared memory
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x;
@@ -265,6 +264,7 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         }
         mbar_init(bfull, 1);
         mbar_init(bempty, RK_COMPUTE_WARPS);
+        mbar_init(u_ready, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -584,11 +584,11 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
             for (int b = 0; b < NB; ++b) e[b][0] = e[b][1] = e[b][2] = e[b][3] = 0.0f;
             if (has_ec) {
                 if (!u_seen) {
-                    // u for every token, read by all 256 compute threads (one round trip of loads
-                    // per two tokens of a warp).
-                    rk_compute_u(a, reinterpret_cast<const unsigned long long*>(a.tacc), ubuf, ustride, BN, cw, lane);
-                    named_bar_compute();
-                    if (cw == 0) ec_retire(a, reinterpret_cast<unsigned long long*>(a.tacc));
+                    // u for every token, formed by the compensator's warp once its item is done.
+                    if (!mbar_wait_ns(u_ready, 0, SK_WAIT_NS)) {
+                        if (lane == 0) sk_fail(a.err, SK_ERR_MBAR, SITE_MMA_UREADY, fe);
+                        ok = false;
+                    }
                     u_seen = true;
                 }
                 // E[n, m] = sum_j B[j, n] u[m, j]: B^T fragments by ldmatrix.trans from the B buffer
@@ -642,8 +642,19 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         }
     } else {
         // ---------------- compensator (warp 9) ----------------
-        if (has_slice) rk_ec_item(a, ec_k0, ec_rows, ec_grp, reinterpret_cast<unsigned long long*>(a.tacc));
+        unsigned long long* tacc = reinterpret_cast<unsigned long long*>(a.tacc);
+        if (has_slice) rk_ec_item(a, ec_k0, ec_rows, ec_grp, tacc);
         else pdl_wait_primary();
+        // In a CTA that finalises a tile: u for every token while the compute warps still stream
+        // weights, off their path; then this CTA's read of the accumulators is retired.
+        bool fin_any = false;
+        for (int i = 0; i < nseg; ++i) fin_any = fin_any || sk_seg(a, u0, u1, i).fin;
+        if (has_ec && fin_any) {
+            rk_compute_u(a, tacc, ubuf, ustride, BN, 0, 1, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(u_ready);
+            ec_retire(a, tacc);
+        }
     }
     __syncthreads();
 }
@@ -685,7 +696,7 @@ bool stream_rk_configure(StreamArgs& a, int bn, int kc, bool deep) {
         a_bytes = wg_bytes = 0;               // the compensator's warp reads A and w_g into registers
     }
     const int red_bytes = kc == 256 ? 4 * 2 * 32 * 4 * (bn / 8) * 4 : 0;
-    const int bar_bytes = 8 * (2 * 16 + 5) + 16;
+    const int bar_bytes = 8 * (2 * 16 + 6) + 16;
     const int fixed = b_bytes + u_bytes + a_bytes + wg_bytes + g_bytes + red_bytes + bar_bytes + 1024;
     const int budget = deep ? (int)SMEM_OPTIN_MAX : 110 * 1024;
     int nst = (budget - fixed) / a.stage_bytes;
