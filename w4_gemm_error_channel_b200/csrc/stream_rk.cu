@@ -416,11 +416,16 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                 const int64_t n = (int64_t)sg.tile * 128 + 16 * (KC == 256 ? rgb + blk : rgb) + g;
                 s_pair = (uint32_t)__half_as_ushort(a.scale[n]) | ((uint32_t)__half_as_ushort(a.scale[n + 8]) << 16);
             }
-            float acc[RG][NB][4];
+            // One 8-token tile: each word pair's second MMA goes to a second set of accumulators, so
+            // consecutive MMAs do not wait on one another (added together at the segment end).
+            constexpr bool SPLIT = NB == 1;
+            float acc[RG][NB][4], acc2[RG][NB][4];
 #pragma unroll
             for (int j = 0; j < RG; ++j)
 #pragma unroll
-                for (int b = 0; b < NB; ++b) acc[j][b][0] = acc[j][b][1] = acc[j][b][2] = acc[j][b][3] = 0.0f;
+                for (int b = 0; b < NB; ++b)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[j][b][q] = acc2[j][b][q] = 0.0f;
 
             for (int kci = sg.kb; kci < sg.ke; ++kci) {
                 if (ok && !rk_wait(&full[s], ph)) {
@@ -452,7 +457,7 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
 #pragma unroll
                         for (int b = 0; b < NB; ++b) {
                             mma_bf16_16816(acc[j][b], af0, xv[b].x, xv[b].y);
-                            mma_bf16_16816(acc[j][b], af1, xv[b].z, xv[b].w);
+                            mma_bf16_16816(SPLIT ? acc2[j][b] : acc[j][b], af1, xv[b].z, xv[b].w);
                         }
                     }
                 }
@@ -464,6 +469,14 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                 }
             }
 
+            if constexpr (SPLIT) {
+#pragma unroll
+                for (int j = 0; j < RG; ++j)
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) acc[j][b][q] += acc2[j][b][q];
+            }
             // ---- this warp's final sums for one 16-row group (KC = 256: blocks exchanged) ----
             float fin[NB][4];
             if constexpr (KC == 256) {
