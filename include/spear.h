@@ -182,8 +182,9 @@ SPEAR_API spear_status spear_debug_unpack_w4(const void* packed, const void* zer
  *
  * Tile order: blocks of 128 rows x 128 codes (8192 bytes); block (T, B) holds rows 128T ..
  * 128T + 127 and codes 128B .. 128B + 127 and starts at byte (T * K/128 + B) * 8192.  Inside a
- * block, row r's 64 bytes start at r * 64 as 16 little-endian 32-bit words; word i holds codes
- * 8i .. 8i + 7 of the block row, code 8i + j in bits 4p .. 4p + 3 with p = (j / 2) + 4 (j % 2)
+ * block, row r's 64 bytes start at r * 64 as 16 little-endian 32-bit words; word i = 4c + w
+ * (c, w = 0..3) holds codes 8s .. 8s + 7 of the block row with s = 2c + w for w < 2 and
+ * s = 8 + 2c + (w - 2) for w >= 2, code 8s + j in bits 4p .. 4p + 3 with p = (j / 2) + 4 (j % 2)
  * (codes 2i' and 2i' + 1 sit in nibbles i' and i' + 4).  The scales and zero-points are unchanged.
  * Requires N % 128 == 0 and K % 128 == 0.  A pure permutation of the 4-bit codes: bit-exact.
  */

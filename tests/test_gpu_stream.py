@@ -309,8 +309,11 @@ def test_rejects_bad_stream_plans():
 
 def _tile_order_numpy(packed, N, K):
     """The tile order restated on the host: 128 x 128-code blocks, row r's 64 bytes at r * 64,
-    code 8i + j of a block row in nibble (j // 2) + 4 (j % 2) of word i."""
+    word 4c + w of a block row holding codes 8s .. 8s + 7 (s = 2c + w, or 8 + 2c + w - 2 for
+    w >= 2), code 8s + j in nibble (j // 2) + 4 (j % 2)."""
     words = np.ascontiguousarray(packed).view(np.uint32).reshape(N, K // 8)
+    src = [2 * (i // 4) + i % 4 if i % 4 < 2 else 8 + 2 * (i // 4) + i % 4 - 2 for i in range(16)]
+    words = words.reshape(N, K // 128, 16)[:, :, src].reshape(N, K // 8)
     codes = np.stack([(words >> (4 * j)) & 0xF for j in range(8)], axis=-1)        # [N, K/8, 8]
     out_words = np.zeros_like(words)
     for j in range(8):

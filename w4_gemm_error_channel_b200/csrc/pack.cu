@@ -152,8 +152,9 @@ __global__ void __launch_bounds__(256) unpack_w4_kernel(const uint8_t* __restric
 }
 
 // Tile order of the register-path stream kernel: one thread per 32-bit word of the output.
-// Output word d = ((T * K/128 + B) * 128 + r) * 16 + i comes from row 128 T + r, word 16 B + i of
-// the row order; code j of the word moves from nibble j to nibble (j / 2) + 4 (j % 2).
+// Output word d = ((T * K/128 + B) * 128 + r) * 16 + i, i = 4c + w, comes from row 128 T + r, word
+// 16 B + s of the row order with s = 2c + w (w < 2) or 8 + 2c + w - 2 (w >= 2); code j of the word
+// moves from nibble j to nibble (j / 2) + 4 (j % 2).
 __global__ void __launch_bounds__(256) tile_w4_kernel(const uint32_t* __restrict__ packed, int64_t N, int64_t K,
                                                       uint32_t* __restrict__ tiled) {
     const int64_t d = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -162,7 +163,9 @@ __global__ void __launch_bounds__(256) tile_w4_kernel(const uint32_t* __restrict
     const int64_t nblk = K / 128;
     const int64_t i = d & 15, r = (d >> 4) & 127, tb = d >> 11;
     const int64_t T = tb / nblk, B = tb % nblk;
-    const uint32_t w = packed[(T * 128 + r) * (K / 8) + B * 16 + i];
+    const int64_t c = i >> 2, wi = i & 3;
+    const int64_t src = wi < 2 ? 2 * c + wi : 8 + 2 * c + (wi - 2);
+    const uint32_t w = packed[(T * 128 + r) * (K / 8) + B * 16 + src];
     uint32_t o = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) o |= ((w >> (4 * j)) & 0xFu) << (4 * ((j >> 1) + 4 * (j & 1)));

@@ -369,13 +369,15 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         const int blk = KC == 256 ? cw >> 2 : 0;              // 128-code block of each unit
         const int rgb = KC == 256 ? 2 * (cw & 3) : cw;         // first 16-row group of this warp
         // Lane-constant shared-memory offsets in a stage: weights of row 16 rgb + g (row group j:
-        // + 1024 j; rows + 8: + 512), and x chunk (box 2 blk + t/2, chunk 4 (t & 1) + w) of token
-        // g (token 8 b + g: + 1024 b), 128-byte swizzle on the token row.
+        // + 1024 j; rows + 8: + 512), and for word w of the lane's 16 bytes (codes 16 t + 8 w, or
+        // 64 + 16 t + 8 (w - 2) for w >= 2, in the tile order) the x chunk (box 2 blk + w/2, chunk
+        // 2 t + w % 2) of token g (token 8 b + g: + 1024 b), 128-byte swizzle on the token row.  The
+        // four lanes t of a quarter-warp read four different chunks of one box: no bank conflict.
         const uint32_t wl = (uint32_t)(blk * RK_BLOCK_BYTES + (16 * rgb + g) * 64 + 16 * t);
         uint32_t xl[4];
 #pragma unroll
         for (int w = 0; w < 4; ++w)
-            xl[w] = (uint32_t)(WBYTES + (2 * blk + (t >> 1)) * XBOX + g * 128 + (((4 * (t & 1) + w) ^ g) << 4));
+            xl[w] = (uint32_t)(WBYTES + (2 * blk + (w >> 1)) * XBOX + g * 128 + (((2 * t + (w & 1)) ^ g) << 4));
         const uint32_t sm_stages = smem_u32(stages);
         const int rbase0 = 16 * rgb + g;                       // tile row of (j = 0, h = 0)
         // Zero-points of the first segment, requested before the wait on the previous kernel.
@@ -441,7 +443,7 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                 }
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
-                    // x codes 32 t + 8 w .. + 7 of the block, every token: natural bf16 pairs.
+                    // x codes of word w, every token: natural bf16 pairs.
                     uint4 xv[NB];
 #pragma unroll
                     for (int b = 0; b < NB; ++b) xv[b] = lds128(st + xl[w] + 1024 * b);
