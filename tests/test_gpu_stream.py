@@ -344,3 +344,20 @@ def test_tiled_planner_runs(M):
     ws = spear.alloc_workspace(plan.workspace_bytes)
     check_close(host_f64(d.run(M, plan, ws)), d.ref(M), True, f"tiled planner M={M}")
     ok_status(ws)
+
+
+def test_w4eclayer_with_both_code_orders():
+    # A layer holding both code orders plans each batch size on the order measured faster (the
+    # tile order on decode-mlp at M = 1), passes the matching codes, and matches the oracle.
+    d = dev(2)
+    L = d.L
+    lay = spear.W4ECLayer(d.packed, d.scale, d.zero, d.ec, tiled=d.tiled)
+    for M in (1, 8):
+        p = lay.plan(M)
+        assert bool(p.flags & spear.SPEAR_PLAN_W4_TILES) == (p.kernel_id == spear.SPEAR_KERNEL_STREAM_RK)
+        y = lay(d.x(M))
+        torch.cuda.synchronize()
+        rows = np.arange(M)
+        check_close(host_f64(y)[rows], d.ref(M, rows=rows), True, f"W4ECLayer both orders M={M}")
+        assert spear.spear_get_device_status(lay.workspace) == 0
+    assert lay.plan(1).kernel_id == spear.SPEAR_KERNEL_STREAM_RK

@@ -69,10 +69,12 @@ SPEAR_DEVI bool rk_wait(uint64_t* bar, uint32_t parity) {
     return mbar_try(bar, parity) || mbar_wait_ns(bar, parity, SK_WAIT_NS);
 }
 
-// u for every token of the tile, by one warp: token pairs (2p, 2p + 1) for p = first, first + step,
-// ...; lane l reads the accumulator words l, l + 32, ... of both tokens (t, then the gate
-// pre-activation in word r), all at once, until every word holds all slices (bounded); then
-// u[m][j] = sigmoid(p[m] + b_g) t[m][j] (fp32, zero past M) goes to ubuf [rows][ustride].
+// u for every token of the tile, by one warp: groups of RK_UT tokens (RK_UT g .. RK_UT g + RK_UT - 1
+// for g = first, first + step, ...); lane l reads the accumulator words l, l + 32, ... of every token
+// of the group (t, then the gate pre-activation in word r), all at once, until each holds all
+// slices (bounded); then u[m][j] = sigmoid(p[m] + b_g) t[m][j] (fp32, zero past M) goes to ubuf
+// [rows][ustride].  One round of loads per RK_UT tokens.
+constexpr int RK_UT = 4;
 SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc, float* ubuf, int ustride, int rows,
                              int first, int step, int lane) {
     constexpr int WMAX = 5;                              // words per lane and token: r + 1 <= 160
@@ -80,21 +82,20 @@ SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc
     const int nw = (r + 1 + 31) / 32;
     const int gi = r / 32, gl = r % 32;                  // the gate word: chunk gi of lane gl
     const unsigned long long want = (unsigned long long)a.ec_slices;
-    for (int m0 = 2 * first; m0 < rows; m0 += 2 * step) {
-        // Tokens m0 and m0 + 1, all their words in flight together.
-        const int m1 = m0 + 1;
-        unsigned long long v0[WMAX], v1[WMAX];
+    for (int m0 = RK_UT * first; m0 < rows; m0 += RK_UT * step) {
+        unsigned long long v[RK_UT][WMAX];
         const uint64_t t0 = globaltimer_ns();
         for (;;) {
             bool done = true;
 #pragma unroll
-            for (int i = 0; i < WMAX; ++i) {
-                const int j = lane + 32 * i;
-                const bool in = i < nw && j <= r;
-                v0[i] = in && m0 < a.M ? ld_cg_u64(tacc_word(tacc, a, m0, j)) : want;
-                v1[i] = in && m1 < a.M ? ld_cg_u64(tacc_word(tacc, a, m1, j)) : want;
-                done = done && ((v0[i] & 0xFFull) == want) && ((v1[i] & 0xFFull) == want);
-            }
+            for (int q = 0; q < RK_UT; ++q)
+#pragma unroll
+                for (int i = 0; i < WMAX; ++i) {
+                    const int j = lane + 32 * i;
+                    const bool in = i < nw && j <= r && m0 + q < a.M;
+                    v[q][i] = in ? ld_cg_u64(tacc_word(tacc, a, m0 + q, j)) : want;
+                    done = done && ((v[q][i] & 0xFFull) == want);
+                }
             if (__all_sync(0xFFFFFFFFu, done)) break;
             if (__any_sync(0xFFFFFFFFu, globaltimer_ns() - t0 > SK_WAIT_NS)) {
                 if (lane == 0) sk_fail(a.err, SK_ERR_FLAG, SITE_EC_TACC, m0);
@@ -102,21 +103,19 @@ SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc
             }
             __nanosleep(64);
         }
-        unsigned long long g0 = 0, g1 = 0;
 #pragma unroll
-        for (int i = 0; i < WMAX; ++i)
-            if (i == gi) { g0 = v0[i]; g1 = v1[i]; }
-        g0 = __shfl_sync(0xFFFFFFFFu, g0, gl);
-        g1 = __shfl_sync(0xFFFFFFFFu, g1, gl);
-        const float gate0 = m0 < a.M ? 1.0f / (1.0f + expf(-(__ll2float_rn((long long)g0 >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) + a.b_g))) : 0.0f;
-        const float gate1 = m1 < a.M ? 1.0f / (1.0f + expf(-(__ll2float_rn((long long)g1 >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) + a.b_g))) : 0.0f;
+        for (int q = 0; q < RK_UT; ++q) {
+            unsigned long long gw = 0;
 #pragma unroll
-        for (int i = 0; i < WMAX; ++i) {
-            const int j = lane + 32 * i;
-            if (i < nw && j < r) {
-                ubuf[m0 * ustride + j] = __ll2float_rn((long long)v0[i] >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) * gate0;
-                if (m1 < rows)
-                    ubuf[m1 * ustride + j] = __ll2float_rn((long long)v1[i] >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) * gate1;
+            for (int i = 0; i < WMAX; ++i) gw = i == gi ? v[q][i] : gw;
+            gw = __shfl_sync(0xFFFFFFFFu, gw, gl);
+            const int m = m0 + q;
+            const float gate = m < a.M ? 1.0f / (1.0f + expf(-(__ll2float_rn((long long)gw >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) + a.b_g))) : 0.0f;
+#pragma unroll
+            for (int i = 0; i < WMAX; ++i) {
+                const int j = lane + 32 * i;
+                if (i < nw && j < r && m < rows)
+                    ubuf[m * ustride + j] = __ll2float_rn((long long)v[q][i] >> SK_FIX_COUNT_BITS) * (1.0f / SK_FIX_ONE) * gate;
             }
         }
     }
