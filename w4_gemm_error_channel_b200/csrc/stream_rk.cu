@@ -74,7 +74,7 @@ SPEAR_DEVI bool rk_wait(uint64_t* bar, uint32_t parity) {
 // of the group (t, then the gate pre-activation in word r), all at once, until each holds all
 // slices (bounded); then u[m][j] = sigmoid(p[m] + b_g) t[m][j] (fp32, zero past M) goes to ubuf
 // [rows][ustride].  One round of loads per RK_UT tokens.
-template <int RK_UT>
+constexpr int RK_UT = 4;
 SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc, float* ubuf, int ustride, int rows,
                              int first, int step, int lane) {
     constexpr int WMAX = 5;                              // words per lane and token: r + 1 <= 160
@@ -128,10 +128,9 @@ SPEAR_DEVI void rk_compute_u(const StreamArgs& a, const unsigned long long* tacc
 // column 0.  The fragments of A come straight from global memory in chunks of KS k-steps, the
 // first chunk before the wait on the previous kernel (A does not depend on it), x after it.
 // Each accumulator word gets one addition per K slice.
-template <int MB>
 SPEAR_DEVI void rk_ec_item(const StreamArgs& a, int64_t k0, int rows, int grp, unsigned long long* tacc) {
     constexpr int KS = 4;                   // k16 steps per chunk
-    // MB: 16-token blocks whose x fragments of a chunk are loaded in one round (the token tile's).
+    constexpr int MB = 4;                   // 16-token blocks (M <= 64)
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int r = a.rank;
     const bool gate = grp == r / 16;
@@ -167,31 +166,28 @@ SPEAR_DEVI void rk_ec_item(const StreamArgs& a, int64_t k0, int rows, int grp, u
     pdl_wait_primary();
     for (int kb = 0; kb < ksteps; kb += KS) {
         if (kb > 0) load_a(kb);
-        uint32_t xa[MB][KS][4];
-#pragma unroll
-        for (int mb = 0; mb < MB; ++mb) {
-            const int64_t ma = 16 * mb + g, mb8 = ma + 8;
-#pragma unroll
-            for (int kk = 0; kk < KS; ++kk) {
-                const int64_t k = k0 + 16 * (kb + kk) + 2 * t;
-                const bool in = kb + kk < ksteps && mb < mblocks;
-                xa[mb][kk][0] = in && ma < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + ma * a.K + k)) : 0u;
-                xa[mb][kk][1] = in && mb8 < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb8 * a.K + k)) : 0u;
-                xa[mb][kk][2] = in && ma < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + ma * a.K + k + 8)) : 0u;
-                xa[mb][kk][3] = in && mb8 < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb8 * a.K + k + 8)) : 0u;
-            }
-        }
 #pragma unroll
         for (int mb = 0; mb < MB; ++mb) {
             if (mb >= mblocks) break;
+            const int64_t ma = 16 * mb + g, mb8 = ma + 8;
+            uint32_t xa[KS][4];
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                const int64_t k = k0 + 16 * (kb + kk) + 2 * t;
+                const bool in = kb + kk < ksteps;
+                xa[kk][0] = in && ma < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + ma * a.K + k)) : 0u;
+                xa[kk][1] = in && mb8 < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb8 * a.K + k)) : 0u;
+                xa[kk][2] = in && ma < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + ma * a.K + k + 8)) : 0u;
+                xa[kk][3] = in && mb8 < a.M ? __ldcg(reinterpret_cast<const unsigned*>(a.x + mb8 * a.K + k + 8)) : 0u;
+            }
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
                 if (kb + kk >= ksteps) break;
                 if (!gate) {
-                    mma_bf16_16816(de[mb], xa[mb][kk], prmt(w[kk][0], w[kk][1], 0x5410u), prmt(w[kk][2], w[kk][3], 0x5410u));
-                    mma_bf16_16816(dod[mb], xa[mb][kk], prmt(w[kk][0], w[kk][1], 0x7632u), prmt(w[kk][2], w[kk][3], 0x7632u));
+                    mma_bf16_16816(de[mb], xa[kk], prmt(w[kk][0], w[kk][1], 0x5410u), prmt(w[kk][2], w[kk][3], 0x5410u));
+                    mma_bf16_16816(dod[mb], xa[kk], prmt(w[kk][0], w[kk][1], 0x7632u), prmt(w[kk][2], w[kk][3], 0x7632u));
                 } else {
-                    mma_bf16_16816(de[mb], xa[mb][kk], w[kk][0], w[kk][1]);
+                    mma_bf16_16816(de[mb], xa[kk], w[kk][0], w[kk][1]);
                 }
             }
         }
@@ -661,14 +657,14 @@ w4_stream_rk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     } else {
         // ---------------- compensator (warp 9) ----------------
         unsigned long long* tacc = reinterpret_cast<unsigned long long*>(a.tacc);
-        if (has_slice) rk_ec_item<(BN + 15) / 16>(a, ec_k0, ec_rows, ec_grp, tacc);
+        if (has_slice) rk_ec_item(a, ec_k0, ec_rows, ec_grp, tacc);
         else pdl_wait_primary();
         // In a CTA that finalises a tile: u for every token while the compute warps still stream
         // weights, off their path; then this CTA's read of the accumulators is retired.
         bool fin_any = false;
         for (int i = 0; i < nseg; ++i) fin_any = fin_any || sk_seg(a, u0, u1, i).fin;
         if (has_ec && fin_any) {
-            rk_compute_u<NB == 8 ? 8 : 4>(a, tacc, ubuf, ustride, BN, 0, 1, lane);
+            rk_compute_u(a, tacc, ubuf, ustride, BN, 0, 1, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(u_ready);
             ec_retire(a, tacc);
