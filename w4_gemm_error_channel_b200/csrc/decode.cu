@@ -428,6 +428,13 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
         for (int q = 0; q < UPT; ++q) v[q] = main_part(threadIdx.x + q * DK_THREADS);
     }
 
+    // This CTA's reader counter (level 1 of the two-level consumer counters; see
+    // retire_accumulators) and thread 0's ticket from it.
+    unsigned reader_ticket = 0u;
+    auto reader_counter = [&]() {
+        const int grp = (tile * S + ks) / CONSUMER_GROUP;
+        return a.consumed1 + (int64_t)chunk * GROUPS_MAX + grp;
+    };
     if (has_ec) {
         // u = sigmoid(p + b_g) t for this CTA's EC columns.  Element c = mm * nj + jj; thread i
         // takes c = i, i + 128, ... (stepping without dividing) and reads the words of t[mm, j0 + jj]
@@ -568,6 +575,9 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
             asm volatile("cp.async.wait_all;" ::: "memory");
         }
         __syncthreads();
+        // Every thread has read its accumulator words: count this CTA as a reader now, so that the
+        // atomic's round trip overlaps the epilogue instead of delaying the CTA's exit.
+        if (threadIdx.x == 0) reader_ticket = atomicAdd(reader_counter(), 1u);
 
         // This slice's EC columns: sum_j u[m, j] B[j, n] added to each unit.
         if (spread) {
@@ -644,9 +654,9 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
         }
     }
 
-    // Every GEMM CTA of the chunk has read the accumulators (before the barrier above): the last
-    // one clears them and the arrival counter for the next call.  Two counter levels (groups of
-    // CONSUMER_GROUP CTAs, then groups) keep same-address atomics few; this is off the path to y.
+    // Every GEMM CTA of the chunk has read the accumulators and counted itself (its ticket, taken
+    // right after its reads): the last one clears them and the arrival counter for the next call.
+    // Two counter levels (groups of CONSUMER_GROUP CTAs, then groups) keep same-address atomics few.
     auto retire_accumulators = [&]() {
         if (!has_ec) return;
         if (threadIdx.x == 0) {
@@ -657,7 +667,7 @@ SPEAR_DEVI void gemm_role(const DecodeArgs& a, int tile, int ks, int chunk, unsi
             const int groups = (per_chunk + CONSUMER_GROUP - 1) / CONSUMER_GROUP;
             unsigned* c1 = a.consumed1 + (int64_t)chunk * GROUPS_MAX + grp;
             unsigned last = 0u;
-            if (atomicAdd(c1, 1u) == (unsigned)in_grp - 1) {
+            if (reader_ticket == (unsigned)in_grp - 1) {
                 *c1 = 0u;                                  // group complete: re-arm
                 last = (atomicAdd(&a.consumed[chunk], 1u) == (unsigned)groups - 1) ? 1u : 0u;
             }
