@@ -564,6 +564,12 @@ def _sweep_shape(torch, spear, L, batches):
                                            for split in (1, 2, 4, 8) for fl in (0, 1)]
         for fl in ((0, 1) if M >= 128 else (0,)):
             candidates += [(2, 128, 1, fl, 128)] + ([(2, 128, 1, fl, 256)] if M >= 256 else [])
+        # The tcgen05 kernel with its K range split over a cluster of 2, 4 or 8 CTAs, where its
+        # grid (weight tiles x token blocks) leaves SMs idle.
+        if M >= 32:
+            for bn in ((128, 256) if M >= 256 else (128,)):
+                grid = (N // 128) * -(-M // bn)
+                candidates += [(2, 128, sk, 0, bn) for sk in (2, 4, 8) if grid * sk <= 4 * 148]
         # The register-path stream kernel (kernel 4) up to 64 tokens: token tile (8-token tiles from
         # M <= 8, 64 only with the deep ring), K codes per stage, and the ring mode (flags 2: one CTA
         # per SM with a deep ring).  The tcgen05 stream kernel (kernel 3) is slower on every measured

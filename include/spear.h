@@ -63,7 +63,13 @@ typedef enum {
     SPEAR_KERNEL_AUTO = 0,      /* let spear_gemm_plan decide */
     SPEAR_KERNEL_SPLITK = 1,    /* decode: split-K weight-streaming kernel (mma.sync on registers); EC
                                    CTAs of the same launch reduce x A through int64 accumulators */
-    SPEAR_KERNEL_TC05 = 2,      /* prefill: TMA + tcgen05/TMEM kernel, EC applied in its epilogue */
+    SPEAR_KERNEL_TC05 = 2,      /* prefill: TMA + tcgen05/TMEM kernel, EC applied in its epilogue.
+                                   tile_n = 128 weight rows (or 256 with tile_m = 128), tile_m = 128,
+                                   160, 192 or 256 tokens.  split_k = 1, or 2, 4 or 8 with 128 weight
+                                   rows, tile_m 128 or 256 and (K / 64) divisible by it: the tile's K
+                                   range is split over a thread-block cluster of split_k CTAs whose
+                                   partial tiles are summed in shared memory in rank order (for small
+                                   grids with long K); not with SPEAR_PLAN_SEPARATE_EC. */
     SPEAR_KERNEL_STREAM = 3,    /* decode and small batches (M <= 64): persistent stream-K TMA + tcgen05
                                    kernel; every SM streams an equal share of the weight tiles' K chunks,
                                    partial tiles meet through the workspace in a fixed order, and the
@@ -372,7 +378,8 @@ typedef struct {
 /*
  * spear_latency_table -- copy the library's built-in latency table: for each shape measured on
  * a B200, the device time per call of its fastest plan in a chained CUDA graph (the dispatcher's
- * table).  out may be NULL to query *len_out only; otherwise capacity must be >= *len_out.
+ * table; one row per (M, N, K, compensator or not), the faster code order where the table holds
+ * both).  out may be NULL to query *len_out only; otherwise capacity must be >= *len_out.
  */
 SPEAR_API spear_status spear_latency_table(spear_latency_entry* out, int32_t capacity, int32_t* len_out);
 

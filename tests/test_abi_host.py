@@ -201,6 +201,34 @@ def test_plan_update_and_semifused_workspace():
         spear.spear_plan_update(q2, M, N, K, r)
 
 
+def test_tc05_k_split_plan_checks():
+    # The tcgen05 kernel's K split: 2, 4 or 8 CTAs per tile (a cluster), 128 weight rows, token
+    # tiles of 128 or 256, (K / 64) divisible by the split, fused compensator only.
+    M, N, K, r = 256, 2048, 8192, 32
+    st, p = _plan(M, N, K, r)
+    assert st == OK
+
+    def upd(split, tile_m=128, tile_n=128, flags=0, k=K, rank=r):
+        q = spear.spear_plan.from_buffer_copy(p)
+        q.kernel_id, q.tile_n, q.split_k, q.tile_m, q.flags = 2, tile_n, split, tile_m, flags
+        return spear._lib.spear_plan_update(ctypes.byref(q), M, N, k, rank), q
+    for split in (1, 2, 4, 8):
+        for tile_m in (128, 256):
+            st, q = upd(split, tile_m)
+            assert st == OK, (split, tile_m)
+            assert q.workspace_bytes == upd(1, tile_m)[1].workspace_bytes   # no workspace of its own
+    for kw in ({"split": 3}, {"split": 16}, {"split": 0}, {"split": 2, "tile_n": 256},
+               {"split": 4, "tile_m": 160}, {"split": 8, "tile_m": 192},
+               {"split": 8, "k": 64 * 12}, {"split": 2, "flags": spear.SPEAR_PLAN_SEPARATE_EC}):
+        assert upd(**kw)[0] == INVALID, kw
+    # Each owner's share of the token tile is a multiple of 16: 160 tokens split 2 ways (80 each),
+    # 192 split 2 or 4 ways (96, 48).
+    assert upd(2, tile_m=160)[0] == OK
+    assert upd(4, tile_m=192)[0] == OK
+    # The split does not combine with the separate-EC flag, with or without a compensator.
+    assert upd(2, flags=spear.SPEAR_PLAN_SEPARATE_EC, rank=0)[0] == INVALID
+
+
 def test_grouped_host_checks():
     # Group-wise scales: groups of a multiple of 128 dividing K for the layer (any even divisor for
     # the packer), compensator rank <= 128.  Fake, never-dereferenced addresses throughout.

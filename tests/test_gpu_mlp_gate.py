@@ -71,6 +71,19 @@ def test_mlp_gate_tc05(M, r, H, tile_m):
     check_close(y, ref, True, f"MLP gate tcgen05 M={M} r={r} H={H}")
 
 
+@pytest.mark.parametrize("M,split,tile_m", [(128, 2, 128), (300, 4, 128), (300, 8, 256)])
+def test_mlp_gate_tc05_k_split(M, split, tile_m):
+    # With the MLP gate the EC tiles keep the whole K range (one CTA per 128 tokens, padded to whole
+    # clusters) while the main tiles split theirs.
+    L = make_layer("mlpk", 90 + M + split, M, 256, 1024, 64, outlier_frac=0.01, outlier_scale=20.0, ec_std=0.05)
+
+    def fix(p):
+        p.kernel_id, p.tile_n, p.split_k, p.tile_m, p.flags = spear.SPEAR_KERNEL_TC05, 128, split, tile_m, 0
+    y, ref, plan, ws = _run(L, M, 16, 1.2, plan_fix=fix)
+    check_close(y, ref, True, f"MLP gate tcgen05 K split {split} M={M}")
+    assert int(ws[: (128 + 1024) * 1024].count_nonzero().item()) == 0, "EC flags not re-armed"
+
+
 def test_mlp_gate_fp32_and_limits():
     # fp32 output meets the literal bound; gamma = 0 (b2 = -inf, W2 = 0) gives the plain layer.
     L = make_layer("mlpf", 81, 8, 256, 512, 32, ec_std=0.05)

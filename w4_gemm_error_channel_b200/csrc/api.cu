@@ -144,6 +144,7 @@ bool lookup_measured(int64_t M, int64_t N, int64_t K, int32_t rank, int sms, spe
     if (best->kernel_id == SPEAR_KERNEL_TC05) {
         if (plan_tc05(M, N, sms, p) != SPEAR_OK) return false;
         if (best->tile_m == 128 || best->tile_m == 256) p->tile_m = best->tile_m;   // the measured width
+        if (tc05_split_supported(p->tile_m, p->tile_n, best->split_k, K)) p->split_k = best->split_k;
         return true;
     }
     p->kernel_id = SPEAR_KERNEL_SPLITK;
@@ -273,10 +274,12 @@ spear_status validate_plan(const spear_plan& p, int64_t M, int64_t N, int64_t K,
     if (p.kernel_id == SPEAR_KERNEL_TC05) {
         if (rank > TC05_MAX_RANK || (p.flags & ~SPEAR_PLAN_SEPARATE_EC)) return SPEAR_ERR_INVALID_ARG;
         if ((M + p.tile_m - 1) / p.tile_m > (int64_t)TC_BLOCKS_MAX) return SPEAR_ERR_INVALID_ARG;
-        if (p.split_k != 1 || !(p.tile_m == 128 || p.tile_m == 160 || p.tile_m == 192 || p.tile_m == 256))
-            return SPEAR_ERR_INVALID_ARG;
+        if (!(p.tile_m == 128 || p.tile_m == 160 || p.tile_m == 192 || p.tile_m == 256)) return SPEAR_ERR_INVALID_ARG;
         // 128 weight rows per tile, or 256 (two sub-tiles sharing x) with 128 tokens.
         if (!(p.tile_n == 128 || (p.tile_n == 256 && p.tile_m == 128 && N % 256 == 0))) return SPEAR_ERR_INVALID_ARG;
+        // K split over a cluster of split_k CTAs (fused compensator only).
+        if (!tc05_split_supported(p.tile_m, p.tile_n, p.split_k, K)) return SPEAR_ERR_INVALID_ARG;
+        if (p.split_k > 1 && (p.flags & SPEAR_PLAN_SEPARATE_EC)) return SPEAR_ERR_INVALID_ARG;
         return SPEAR_OK;
     }
     if (p.kernel_id != SPEAR_KERNEL_SPLITK) return SPEAR_ERR_INVALID_ARG;
@@ -561,7 +564,7 @@ spear_status spear_w4ec_gemm(const spear_plan* plan, const void* x, int64_t M, i
         if (rank > 0 && (p.flags & SPEAR_PLAN_SEPARATE_EC))
             e = launch_semifused(t, p.tile_m, p.tile_n, (float*)(ws + ZEROED_BYTES + tc05_u_bytes(M, rank)), s);
         else
-            e = launch_tc05(t, p.tile_m, p.tile_n, s);
+            e = launch_tc05(t, p.tile_m, p.tile_n, s, true, 0, p.split_k);
         return e == cudaSuccess ? SPEAR_OK : SPEAR_ERR_CUDA;
     }
     if (p.kernel_id == SPEAR_KERNEL_STREAM || p.kernel_id == SPEAR_KERNEL_STREAM_RK) {

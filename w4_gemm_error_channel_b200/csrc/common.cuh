@@ -109,4 +109,27 @@ SPEAR_DEVI int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
 
 SPEAR_DEVI float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
 
+// ---------------------------------------------------------------------------------------------
+// Cluster helpers (distributed shared memory).
+// ---------------------------------------------------------------------------------------------
+// Split form of the cluster barrier: the arrive at kernel start and the wait before the first
+// remote store make sure every CTA of the cluster is running before its shared memory is written.
+SPEAR_DEVI void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
+SPEAR_DEVI void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+SPEAR_DEVI void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Store to the same shared-memory offset in cluster rank `rank`.
+SPEAR_DEVI void st_dsmem_f32(float* local, unsigned rank, float v) {
+    uint32_t la = (uint32_t)__cvta_generic_to_shared(local), ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(la), "r"(rank));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+}
+SPEAR_DEVI void st_dsmem_f4(float4* local, unsigned rank, float4 v) {
+    uint32_t la = (uint32_t)__cvta_generic_to_shared(local), ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(la), "r"(rank));
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(ra), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
 }  // namespace spear

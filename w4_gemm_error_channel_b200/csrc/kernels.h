@@ -123,6 +123,7 @@ struct TcArgs {
     unsigned* ec_consumed;  // [token blocks] main tiles that have seen the flag
     GateMlp mlp;            // bottleneck-MLP gate (w1 == null: the scalar gate)
     int ec_only;            // 1: launch the EC tiles alone (u only, no ready flags); 0: the whole layer
+    int split;              // K splits per weight tile, one cluster of `split` CTAs (set by launch_tc05)
 };
 
 // Small-batch stream-K kernel (stream.cu).  The host fills the problem fields and `grid`, then
@@ -175,7 +176,10 @@ cudaError_t launch_stream(const StreamArgs& a, int bn, cudaStream_t stream);
 
 // bn = tokens per tile; rows = weight rows per tile (128, or 256 with bn = 128).  pdl: launch as a
 // programmatic dependent of the previous kernel in the stream; priority: 0 or a launch priority.
-cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream, bool pdl = true, int priority = 0);
+cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream, bool pdl = true, int priority = 0,
+                        int split = 1);
+// Whether launch_tc05 takes this K split for a tile of bn tokens and `rows` weight rows.
+bool tc05_split_supported(int bn, int rows, int split, int64_t K);
 
 // The compensator beside a main-term launch: the tcgen05 kernel's EC tiles alone (u = g t) on a
 // side stream of the library, `main` (which writes the fp32 main term to ymain [M][N]) on the

@@ -25,6 +25,10 @@
 // its ready flag.  A main tile, after its K loop, waits (bounded) for the flags of its tokens, loads
 // the u tile and the B slice (MN-major, from [r, N]) by TMA and accumulates E[n, m] = sum_j
 // B[j, n] u[m, j] into TMEM; the epilogue writes y = s[n] D + E.
+// K split (small grids with long K): a tile's K range is split over a cluster of 2, 4 or 8 CTAs;
+// after their K loops the partial tiles meet in the owners' idle stage buffers through distributed
+// shared memory and are summed in rank order.  EC tiles split the same way and sum t and the gate
+// pre-activation before forming u.
 // Every mbarrier and flag wait is bounded: on timeout the kernel records an error bit and stops.
 #include <mutex>
 
@@ -70,9 +74,11 @@ struct TcSmem {
 };
 constexpr int TC_EB = 128;               // tokens per EC tile
 
-// Tiles: the first `ec_tiles` blocks are EC tiles (one per 128 tokens; compute u), the rest are
-// main tiles (128 SUB weight rows, token block mb of BN tokens), token-block major.  With SUB = 2
-// the two 128-row sub-tiles share every x stage, which halves the x traffic from L2.
+// Tiles: the first blocks are EC tiles (one per 128 tokens; compute u), the rest are main tiles
+// (128 SUB weight rows, token block mb of BN tokens), token-block major.  With SUB = 2 the two
+// 128-row sub-tiles share every x stage, which halves the x traffic from L2.  With a K split of
+// S > 1 every tile is a cluster of S consecutive CTAs, one per K range (EC tiles too, unless the
+// MLP gate is on), and the EC CTAs are padded to whole clusters.
 template <int BN, int STAGES, int SUB>
 __global__ void __launch_bounds__(TC_THREADS, (TcSmem<BN, STAGES, SUB>::MIN_BLOCKS))
 w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
@@ -93,17 +99,28 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool has_ec = a.rank > 0;
+    const int S = a.split;                                                 // K splits per weight tile
     const int eblocks = (int)((a.M + TC_EB - 1) / TC_EB);
-    const int ec_tiles = has_ec ? eblocks : 0;
-    const bool is_ec = (int)blockIdx.x < ec_tiles;
-    const int t = is_ec ? (int)blockIdx.x : (int)blockIdx.x - ec_tiles;
+    // EC tiles split their K range the same way (one cluster per 128-token block), except with the
+    // bottleneck-MLP gate, whose epilogue needs the whole of t in one CTA.
+    const int SE = a.mlp.w1 != nullptr ? 1 : S;
+    const int ec_ctas = has_ec ? eblocks * SE : 0;
+    const int ec_pad = (ec_ctas + S - 1) / S * S;                          // EC CTAs, padded to whole clusters
+    if ((int)blockIdx.x >= ec_ctas && (int)blockIdx.x < ec_pad) return;    // idle CTA of the last EC cluster
+    const bool is_ec = (int)blockIdx.x < ec_ctas;
+    const int KS = is_ec ? SE : S;                                         // K splits of this CTA's tile
+    const int bi = is_ec ? (int)blockIdx.x : (int)blockIdx.x - ec_pad;
+    const int ks = bi % KS;                                                // this CTA's K split = cluster rank
+    const int t = bi / KS;
     const int ntiles = (int)(a.N / (TC_BM * SUB));
     const int mb = is_ec ? t : t / ntiles;                                 // EC: 128-token block; main: BN block
     const int64_t n0 = is_ec ? 0 : (int64_t)(t % ntiles) * TC_BM * SUB;
     const int64_t m0 = (int64_t)mb * (is_ec ? TC_EB : BN);
-    const int ksteps = (int)(a.K / TC_BK);
-    // EC MMA steps: 64 columns of u per chunk, one step per (chunk, sub-tile).
-    const int ec_chunks = (!is_ec && has_ec) ? ((a.rank + 63) / 64) * SUB : 0;
+    const int ksteps = (int)(a.K / TC_BK) / KS;                            // K stages of this CTA
+    const int kbase = ks * ksteps;                                         // its first K stage
+    // EC MMA steps: 64 columns of u per chunk, one step per (chunk, sub-tile); with a K split the
+    // first split of the tile adds the EC term.
+    const int ec_chunks = (!is_ec && has_ec && ks == 0) ? ((a.rank + 63) / 64) * SUB : 0;
     const int rboxes = (a.rank + 63) / 64;                                 // 64-wide boxes of A per stage
     const int e_lo = (int)(m0 / TC_EB);                                    // EC blocks this main tile needs
     const int e_hi = min(eblocks, (int)((m0 + BN + TC_EB - 1) / TC_EB));
@@ -129,6 +146,8 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     const uint32_t tmem_d = *tmem_slot;
     const uint32_t tmem_a = tmem_d + SUB * BN;   // converted weight stages (main K loop)
     const uint32_t tmem_e = tmem_d + SUB * BN;   // EC accumulators (after the main K loop)
+    bool epi_ok = true;                          // converter warps: the accumulators completed
+    float pg_part = 0.0f;                        // EC converter warps: gate pre-activation over this K split
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -139,12 +158,12 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                     unsigned char* as = smem + L::A_OFF + s * L::A_BYTES;
                     mbar_arrive_expect_tx(&full[s], TC_EB * TC_BK * 2 + rboxes * (TC_BK * 64 * 2) + TC_BK * 2);
                     for (int bx = 0; bx < rboxes; ++bx)
-                        tma_load_2d(as + bx * (TC_BK * 64 * 2), &tmap_a, bx * 64, kt * TC_BK, &full[s]);
-                    tma_load_2d(smem + L::WG_OFF + s * TC_BK * 2, &tmap_g, kt * TC_BK, 0, &full[s]);
+                        tma_load_2d(as + bx * (TC_BK * 64 * 2), &tmap_a, bx * 64, (kbase + kt) * TC_BK, &full[s]);
+                    tma_load_2d(smem + L::WG_OFF + s * TC_BK * 2, &tmap_g, (kbase + kt) * TC_BK, 0, &full[s]);
                 } else {
                     mbar_arrive_expect_tx(&full[s], L::X_BYTES + L::P_BYTES);
                     for (int sb = 0; sb < SUB; ++sb)
-                        tma_load_2d(smem + L::P_OFF + s * L::P_BYTES + sb * L::P_SUB, &tmap_w, kt * (TC_BK / 2),
+                        tma_load_2d(smem + L::P_OFF + s * L::P_BYTES + sb * L::P_SUB, &tmap_w, (kbase + kt) * (TC_BK / 2),
                                     (int32_t)(n0 + sb * TC_BM), &full[s]);
                 }
             };
@@ -159,13 +178,14 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                     load_weights(kt, s);
                 }
                 unsigned char* xs = smem + L::X_OFF + s * L::X_BYTES;
-                tma_load_2d(xs, is_ec ? &tmap_x128 : &tmap_x, kt * TC_BK, (int32_t)m0, &full[s]);
+                tma_load_2d(xs, is_ec ? &tmap_x128 : &tmap_x, (kbase + kt) * TC_BK, (int32_t)m0, &full[s]);
             }
             if (ok && ec_chunks > 0) {
-                // u of these tokens is written by their EC tiles: wait (bounded) for the flags.
+                // u of these tokens is written by their EC tiles: wait (bounded) until each flag
+                // counts all SE EC CTAs of its block.
                 for (int e = e_lo; e < e_hi && ok; ++e) {
                     unsigned it = 0;
-                    while (ld_acquire_gpu(&a.ec_ready[e]) == 0u) {
+                    while (ld_acquire_gpu(&a.ec_ready[e]) < (unsigned)SE) {
                         if (++it > WAIT_LIMIT) { atomicOr(a.err, 8u); ok = false; break; }
                         if (it > 64) __nanosleep(128);
                     }
@@ -302,8 +322,12 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 
         const bool acc_ok = ok && mbar_wait(acc_full, 0);
         if (!acc_ok) atomicOr(a.err, 4u);
+        epi_ok = acc_ok;
+        pg_part = pg;
         tc_fence_after();
-        if (is_ec) {
+        if (is_ec && SE > 1) {
+            // K-split EC tile: the partial t and gate pre-activations meet after the block barrier.
+        } else if (is_ec) {
             if (a.mlp.w1 != nullptr) {
                 // Bottleneck-MLP gate: t is staged as [token][j] in the idle stages, then thread row
                 // takes token m0 + row: h = relu(W1 t + b1), u[m, j] = alpha sigmoid(W2 h + b2)_j t_j.
@@ -362,7 +386,7 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             // EC tiles launched alone (the semi-fused path) have no main tiles to signal.
             if (row == 0 && acc_ok && !a.ec_only)
                 asm volatile("st.release.gpu.global.u32 [%0], 1;" ::"l"(&a.ec_ready[mb]) : "memory");
-        } else {
+        } else if (S == 1) {
             // y[m, n] = s[n] D[n, m] (+ E[n, m]), sub-tile by sub-tile.  bf16 output: the tile is
             // staged in the (now idle) x stages as y[m][n] rows and leaves in one TMA store,
             // which also drops the rows past M; fp32 debug output is stored directly.
@@ -401,6 +425,94 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 
     tc_fence_before();
     __syncthreads();
+    if (KS > 1) {
+        // K split: the KS CTAs of this cluster hold partial sums of one tile.  Each has seen its
+        // accumulators complete (before the block barrier above), so its stage area is idle; after
+        // one cluster barrier it receives the partial tiles of the columns it owns: rank ks owns
+        // columns [ks C / KS, (ks + 1) C / KS) of the tile's C token columns and sums the KS
+        // partials in rank order (fixed order, so the result does not depend on timing).
+        //   main tile: a partial is s[n] D + E (E on rank 0 only), summed into y;
+        //   EC tile:   a partial is t[j, m] plus the gate pre-activation of token m, summed into
+        //              u = sigmoid(p + b_g) t, after which the rank adds 1 to the block's ready flag.
+        const int cols = is_ec ? TC_EB : BN;
+        const int bno = cols / KS, rstride = bno + 4;    // padded rows: conflict-free float4 access
+        float* recv = reinterpret_cast<float*>(smem + L::X_OFF);   // [KS][128 rows][bno + 4]
+        float* recv_p = recv + KS * TC_BM * rstride;               // EC: [KS][128 tokens]
+        __syncwarp();
+        cluster_sync_all();
+        tc_fence_after();
+        if (warp >= 2) {
+            const int row = (warp & 3) * 32 + lane;
+            const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+            const float sc = is_ec ? 1.0f : __half2float(a.scale[n0 + row]);
+            const bool with_e = ec_chunks > 0;
+            for (int c0 = 0; c0 < cols; c0 += 16) {
+                float v[16], e[16];
+                tmem_ld16(tmem_d + lane_base + (uint32_t)c0, v);
+                if (with_e) tmem_ld16(tmem_e + lane_base + (uint32_t)c0, e);
+                const int owner = c0 / bno;                // bno is a multiple of 16
+                float* dst = recv + (ks * TC_BM + row) * rstride + (c0 - owner * bno);
+#pragma unroll
+                for (int i = 0; i < 16; i += 4) {
+                    const float4 w = with_e ? make_float4(fmaf(sc, v[i], e[i]), fmaf(sc, v[i + 1], e[i + 1]),
+                                                          fmaf(sc, v[i + 2], e[i + 2]), fmaf(sc, v[i + 3], e[i + 3]))
+                                            : make_float4(sc * v[i], sc * v[i + 1], sc * v[i + 2], sc * v[i + 3]);
+                    st_dsmem_f4(reinterpret_cast<float4*>(dst + i), (unsigned)owner, w);
+                }
+            }
+            if (is_ec) st_dsmem_f32(recv_p + ks * TC_BM + row, (unsigned)(row / bno), pg_part);
+        }
+        tc_fence_before();
+        __syncwarp();
+        cluster_sync_all();
+        if (warp >= 2) {
+            const int row = (warp & 3) * 32 + lane;
+            if (is_ec) {
+                // Thread row = EC column j; tokens of this rank's share one by one.
+                const int j = row;
+                for (int c = 0; c < bno; ++c) {
+                    const int ml = ks * bno + c;
+                    float p = recv_p[ml];
+                    float tv = recv[j * rstride + c];
+                    for (int src = 1; src < KS; ++src) {
+                        p += recv_p[src * TC_BM + ml];
+                        tv += recv[(src * TC_BM + j) * rstride + c];
+                    }
+                    const int64_t m = m0 + ml;
+                    if (epi_ok && j < a.rank && m < a.M)
+                        a.u[m * a.rank + j] = __float2bfloat16_rn(tv / (1.0f + expf(-(p + a.b_g))));
+                }
+                asm volatile("fence.proxy.async.global;" ::: "memory");   // u is read by other CTAs' TMA
+                __threadfence();
+                named_bar_epi();
+                if (row == 0 && epi_ok)
+                    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&a.ec_ready[mb]) : "memory");
+            } else if (epi_ok) {
+                const int64_t n = n0 + row;
+                for (int c = 0; c < bno; c += 4) {
+                    float4 sum = *reinterpret_cast<const float4*>(recv + row * rstride + c);
+                    for (int src = 1; src < KS; ++src) {
+                        const float4 o = *reinterpret_cast<const float4*>(recv + (src * TC_BM + row) * rstride + c);
+                        sum.x += o.x;
+                        sum.y += o.y;
+                        sum.z += o.z;
+                        sum.w += o.w;
+                    }
+                    const float sv[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int64_t m = m0 + (int64_t)ks * bno + c + i;
+                        if (m >= a.M) continue;
+                        if (a.y_fp32)
+                            reinterpret_cast<float*>(a.y)[m * a.N + n] = sv[i];
+                        else
+                            reinterpret_cast<__nv_bfloat16*>(a.y)[m * a.N + n] = __float2bfloat16_rn(sv[i]);
+                    }
+                }
+            }
+        }
+        tc_fence_after();
+    }
     pdl_launch_dependents();
     if (warp == 1) {
         tc_fence_after();
@@ -479,9 +591,26 @@ cudaError_t opt_in_smem(const void* func, size_t bytes, std::once_flag* once, cu
     return status[dev];
 }
 
+// A K split of S: the tile's token columns split into S owners' shares of a multiple of 16, the
+// partial tiles fit in the stage area ([S][128][BN / S + 4] fp32; an EC tile's [S][128][128 / S + 4]
+// plus [S][128] gate pre-activations), and every split has the same number of 64-wide K stages.
 template <int BN, int STAGES, int SUB>
-static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream, bool pdl, int priority) {
+static bool split_fits(int split, int64_t K) {
     using L = TcSmem<BN, STAGES, SUB>;
+    if (split == 1) return true;
+    if (!(split == 2 || split == 4 || split == 8) || SUB != 1) return false;
+    if (BN % (16 * split) != 0 || (K / TC_BK) % split != 0) return false;
+    const int64_t stage_area = L::WG_OFF - L::X_OFF;
+    const int64_t ec_part = (int64_t)split * TC_BM * (TC_EB / split + 4) * 4 + (int64_t)split * TC_BM * 4;
+    return (int64_t)split * TC_BM * (BN / split + 4) * 4 <= stage_area && ec_part <= stage_area;
+}
+
+template <int BN, int STAGES, int SUB>
+static cudaError_t launch_tc_t(const TcArgs& a_in, cudaStream_t stream, bool pdl, int priority, int split) {
+    using L = TcSmem<BN, STAGES, SUB>;
+    if (!split_fits<BN, STAGES, SUB>(split, a_in.K) || (split > 1 && a_in.ec_only)) return cudaErrorInvalidValue;
+    TcArgs a = a_in;
+    a.split = split;
     CUtensorMap mx, mw, ma, mb, mu, mg, mx128;
     if (!make_map_2d(&mx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.K, (uint64_t)a.M, TC_BK, BN,
                      CU_TENSOR_MAP_SWIZZLE_128B))
@@ -522,14 +651,26 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream, bool pdl, i
     if (oe != cudaSuccess) return oe;
     const unsigned mblocks = (unsigned)((a.M + BN - 1) / BN);
     const unsigned eblocks = (unsigned)((a.M + TC_EB - 1) / TC_EB);
-    const unsigned tiles = a.ec_only ? eblocks : (unsigned)(a.N / (TC_BM * SUB)) * mblocks + (has_ec ? eblocks : 0u);
+    // EC CTAs first (split like the main tiles unless the MLP gate is on; padded to whole clusters),
+    // then the split CTAs of each main tile side by side.
+    const unsigned ec_ctas = has_ec ? eblocks * (a.mlp.w1 != nullptr ? 1u : (unsigned)split) : 0u;
+    const unsigned ec_pad = (ec_ctas + split - 1) / split * split;
+    const unsigned tiles =
+        a.ec_only ? eblocks : (unsigned)(a.N / (TC_BM * SUB)) * mblocks * (unsigned)split + ec_pad;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles);
     cfg.blockDim = dim3(TC_THREADS);
     cfg.dynamicSmemBytes = L::TOTAL;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[3];
     unsigned na = 0;
+    if (split > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)split;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
     if (pdl) {
         attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[na].val.programmaticStreamSerializationAllowed = 1;
@@ -545,14 +686,24 @@ static cudaError_t launch_tc_t(const TcArgs& a, cudaStream_t stream, bool pdl, i
     return cudaLaunchKernelEx(&cfg, w4_tc05_kernel<BN, STAGES, SUB>, mx, mw, ma, mb, mu, mg, mx128, my, a);
 }
 
-cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream, bool pdl, int priority) {
-    if (rows == 256) return bn == 128 ? launch_tc_t<128, 4, 2>(a, stream, pdl, priority) : cudaErrorInvalidValue;
+cudaError_t launch_tc05(const TcArgs& a, int bn, int rows, cudaStream_t stream, bool pdl, int priority, int split) {
+    if (rows == 256) return bn == 128 ? launch_tc_t<128, 4, 2>(a, stream, pdl, priority, split) : cudaErrorInvalidValue;
     if (rows != 128) return cudaErrorInvalidValue;
-    if (bn == 128) return launch_tc_t<128, 3, 1>(a, stream, pdl, priority);
-    if (bn == 160) return launch_tc_t<160, 4, 1>(a, stream, pdl, priority);
-    if (bn == 192) return launch_tc_t<192, 3, 1>(a, stream, pdl, priority);
-    if (bn == 256) return launch_tc_t<256, 4, 1>(a, stream, pdl, priority);
+    if (bn == 128) return launch_tc_t<128, 3, 1>(a, stream, pdl, priority, split);
+    if (bn == 160) return launch_tc_t<160, 4, 1>(a, stream, pdl, priority, split);
+    if (bn == 192) return launch_tc_t<192, 3, 1>(a, stream, pdl, priority, split);
+    if (bn == 256) return launch_tc_t<256, 4, 1>(a, stream, pdl, priority, split);
     return cudaErrorInvalidValue;
+}
+
+bool tc05_split_supported(int bn, int rows, int split, int64_t K) {
+    if (rows == 256) return bn == 128 && split_fits<128, 4, 2>(split, K);
+    if (rows != 128) return false;
+    if (bn == 128) return split_fits<128, 3, 1>(split, K);
+    if (bn == 160) return split_fits<160, 4, 1>(split, K);
+    if (bn == 192) return split_fits<192, 3, 1>(split, K);
+    if (bn == 256) return split_fits<256, 4, 1>(split, K);
+    return false;
 }
 
 }  // namespace spear
