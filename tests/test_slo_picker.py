@@ -2,6 +2,7 @@
 tables, the bisection against a brute-force scan, monotonicity, the effect of where compensators
 sit, and argument errors."""
 import math
+import os
 
 import pytest
 
@@ -52,6 +53,18 @@ def test_samples_are_made_monotone():
 def test_builtin_table_reads_back_and_is_monotone():
     table = spear.spear_latency_table()
     assert len(table) > 10 and all(M >= 1 and us > 0 for (M, _, _, _, us) in table)
+    # One row per shape: the fastest of the dispatcher's rows for it (both code orders).
+    keys = [(M, N, K, e) for (M, N, K, e, _) in table]
+    assert len(keys) == len(set(keys))
+    inc = os.path.join(os.path.dirname(spear.__file__), "csrc", "plan_table.inc")
+    fastest = {}
+    for line in open(inc):
+        if line.startswith("{"):
+            v = [float(t) for t in line.strip().strip("{},").split(",")]
+            k = tuple(int(t) for t in v[:4])
+            fastest[k] = min(fastest.get(k, math.inf), v[9])
+    assert {k: round(us, 3) for (*k, us) in map(tuple, table) for k in [tuple(k)]} == \
+        {k: round(us, 3) for k, us in fastest.items()}
     lin = model()
     prev = 0.0
     for M in range(0, 4097, 16):

@@ -92,27 +92,44 @@ struct Model {
     }
 };
 
-const spear_latency_entry* builtin_table() {
-    static spear_latency_entry* rows = [] {
-        auto* r = (spear_latency_entry*)calloc((size_t)kTableLen, sizeof(spear_latency_entry));
-        for (int32_t i = 0; r && i < kTableLen; ++i) {
-            r[i].M = kTable[i].M;
-            r[i].N = kTable[i].N;
-            r[i].K = kTable[i].K;
-            r[i].has_ec = kTable[i].has_ec;
-            r[i].us = kTable[i].us;
+// The dispatcher's table holds one row per shape and code order (row order, and the tile order of
+// spear_tile_w4 for the stream-K kernel); a layer that holds both orders runs the faster one, so
+// the latency table keeps, per (M, N, K, compensator or not), the fastest row.
+struct BuiltinTable {
+    spear_latency_entry* rows = nullptr;
+    int32_t len = 0;
+};
+const BuiltinTable& builtin() {
+    static BuiltinTable t = [] {
+        BuiltinTable b;
+        b.rows = (spear_latency_entry*)calloc((size_t)kTableLen, sizeof(spear_latency_entry));
+        for (int32_t i = 0; b.rows && i < kTableLen; ++i) {
+            int32_t j = 0;
+            while (j < b.len && !(b.rows[j].M == kTable[i].M && b.rows[j].N == kTable[i].N &&
+                                  b.rows[j].K == kTable[i].K && b.rows[j].has_ec == kTable[i].has_ec))
+                ++j;
+            if (j == b.len) {
+                b.rows[j].M = kTable[i].M;
+                b.rows[j].N = kTable[i].N;
+                b.rows[j].K = kTable[i].K;
+                b.rows[j].has_ec = kTable[i].has_ec;
+                b.rows[j].us = kTable[i].us;
+                ++b.len;
+            } else if (kTable[i].us < b.rows[j].us) {
+                b.rows[j].us = kTable[i].us;
+            }
         }
-        return r;
+        return b;
     }();
-    return rows;
+    return t;
 }
 
 spear_status build_model(const spear_linear_desc* linears, int32_t n, const spear_latency_entry* lut, int32_t lut_len,
                          double fixed_us, Model* m) {
     if (!linears || n <= 0 || !(fixed_us >= 0.0) || !isfinite(fixed_us)) return SPEAR_ERR_INVALID_ARG;
     if (!lut) {
-        lut = builtin_table();
-        lut_len = kTableLen;
+        lut = builtin().rows;
+        lut_len = builtin().len;
         if (!lut) return SPEAR_ERR_INVALID_ARG;
     } else if (lut_len <= 0) {
         return SPEAR_ERR_INVALID_ARG;
@@ -146,12 +163,12 @@ extern "C" {
 
 spear_status spear_latency_table(spear_latency_entry* out, int32_t capacity, int32_t* len_out) {
     if (!len_out) return SPEAR_ERR_INVALID_ARG;
-    *len_out = kTableLen;
+    const BuiltinTable& t = builtin();
+    if (!t.rows) return SPEAR_ERR_INVALID_ARG;
+    *len_out = t.len;
     if (!out) return SPEAR_OK;
-    if (capacity < kTableLen) return SPEAR_ERR_INVALID_ARG;
-    const spear_latency_entry* t = builtin_table();
-    if (!t) return SPEAR_ERR_INVALID_ARG;
-    for (int32_t i = 0; i < kTableLen; ++i) out[i] = t[i];
+    if (capacity < t.len) return SPEAR_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < t.len; ++i) out[i] = t.rows[i];
     return SPEAR_OK;
 }
 
