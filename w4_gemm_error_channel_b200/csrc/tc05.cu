@@ -446,7 +446,10 @@ w4_tc05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
             const float sc = is_ec ? 1.0f : __half2float(a.scale[n0 + row]);
             const bool with_e = ec_chunks > 0;
-            for (int c0 = 0; c0 < cols; c0 += 16) {
+            // Rank ks starts with the columns of owner ks + 1, so that at any time each owner
+            // receives from one rank rather than all ranks at once.
+            for (int q = 0; q < cols; q += 16) {
+                const int c0 = (q + (ks + 1) * bno) % cols;
                 float v[16], e[16];
                 tmem_ld16(tmem_d + lane_base + (uint32_t)c0, v);
                 if (with_e) tmem_ld16(tmem_e + lane_base + (uint32_t)c0, e);
