@@ -201,6 +201,39 @@ def test_plan_update_and_semifused_workspace():
         spear.spear_plan_update(q2, M, N, K, r)
 
 
+def _measured_rows():
+    inc = os.path.join(os.path.dirname(spear.__file__), "csrc", "plan_table.inc")
+    rows = []
+    for line in open(inc):
+        if line.startswith("{"):
+            v = line.strip().strip("{},").split(",")
+            rows.append(tuple(int(t) for t in v[:9]))
+    return rows
+
+
+def test_planner_returns_every_measured_plan():
+    # The dispatcher hands out, at each measured shape, the plan the table recorded for it (row-order
+    # codes), and every row -- tile-order rows included -- is a plan spear_plan_update accepts.
+    rows = _measured_rows()
+    assert len(rows) > 50
+    for (M, N, K, e, kern, tile_n, split, tile_m, flags) in rows:
+        r = 32 if e else 0
+        q = spear.spear_plan()
+        q.kernel_id, q.tile_n, q.split_k, q.tile_m, q.flags = kern, tile_n, split, tile_m, flags
+        if kern == spear.SPEAR_KERNEL_SPLITK:
+            q.tile_m = 8 if M <= 8 else (16 if M <= 16 else 32)
+        assert spear._lib.spear_plan_update(ctypes.byref(q), M, N, K, r) == OK, (M, N, K, e, kern, split)
+        if kern == spear.SPEAR_KERNEL_STREAM_RK:
+            continue
+        st, p = _plan(M, N, K, r)
+        assert st == OK
+        assert (p.kernel_id, p.split_k) == (kern, split), (M, N, K, e)
+        if kern == spear.SPEAR_KERNEL_SPLITK:
+            assert p.tile_n == tile_n
+        else:
+            assert p.tile_m == tile_m
+
+
 def test_tc05_k_split_plan_checks():
     # The tcgen05 kernel's K split: 2, 4 or 8 CTAs per tile (a cluster), 128 weight rows, token
     # tiles of 128 or 256, (K / 64) divisible by the split, fused compensator only.
