@@ -823,7 +823,7 @@ def slo_check(args):
 
 def kernel_name(spear, p):
     if p.kernel_id == spear.SPEAR_KERNEL_TC05:
-        return "tcgen05"
+        return "tcgen05" if p.split_k <= 1 else f"tcgen05, K split {p.split_k}"
     if p.kernel_id == spear.SPEAR_KERNEL_STREAM_RK:
         return "stream-K register path (tile order)"
     if p.kernel_id == spear.SPEAR_KERNEL_STREAM:
